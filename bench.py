@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Benchmark of PISA piecewise sparse attention on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan]
+                    [--impl pisa|reference] [--no-cpu-baseline] [--no-dense]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+block statistics -> selection -> fused piecewise attention, through the C ABI
+(`pisa_attention_ex` with a caller workspace).  `value` is the dense-equivalent
+throughput 4 B H L^2 d / step time in TFLOP/s, summed over ranks (weak
+scaling: every rank runs its own independent problem of the same shape; no
+collective is on the data path).  Inputs live in HBM when timing starts and
+are larger than L2 (126 MB), so no flush is needed between steps.
+
+The `roofline` object is for the dominant kernel (the fused attention kernel),
+timed per launch with CUDA events on the launching stream inside the timed
+region.  `e2e` is the same metric through `pisa_attention` with pinned host
+buffers: host->device copies of q, k, v and the device->host copy of the
+output are inside its timed region.  `cpu_baseline` is the fp64 oracle timed on
+the host cores on a bounded sample of the same workload, extrapolated.
+`--impl reference` times only that oracle, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, generate_head, generate_qkv  # noqa: E402
+
+METRIC = "PISA attention ms/call & dense-equiv TFLOP/s on 1 B200; fraction of roofline"
+UNIT = "dense-equiv TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the fused attention kernel, from an ncu capture,
+# keyed by the sha1 of the kernel source it was taken on (see profiles/).
+K3_TRAFFIC = {}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _k3_source_hash():
+    h = hashlib.sha1()
+    for n in ("k3_attention_mma.cuh",):
+        fn = os.path.join(ROOT, "block_sparse_attention_stats_b200", "csrc", n)
+        if os.path.exists(fn):
+            h.update(open(fn, "rb").read())
+    return h.hexdigest()[:12]
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work
+# ----------------------------------------------------------------------------
+
+def dense_flops(wl):
+    return 4.0 * wl.B * wl.H * wl.L * wl.L * wl.d
+
+
+def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
+    """4d sum_i n_i sum_{S_i} n_j + 4d sum_i n_i |U_i| + [hyd] 2 L d^2, per head, summed."""
+    b, L, d = wl.block_size, wl.L, wl.d
+    N = -(-L // b)
+    k_sel = idx.shape[-1]
+    n_last = L - (N - 1) * b
+    n_i = torch.full((N,), float(b), device=idx.device, dtype=torch.float64)
+    n_i[-1] = n_last
+    last_sel = (idx == N - 1).any(dim=-1).to(torch.float64)        # [B,H,N]
+    exact_keys = k_sel * b - (b - n_last) * last_sel                   # sum_{S_i} n_j
+    exact = 4.0 * d * float((n_i * exact_keys).sum())
+    tail = 4.0 * d * float(n_i.sum()) * (N - k_sel) * wl.B * wl.H
+    first = (2.0 * L * d * d * wl.B * wl.H) if wl.mode == "hyd" else 0.0
+    return exact + tail + first
+
+
+def k3_executed_flops(wl, k_sel: int, chunks_per_block: float) -> float:
+    """MMA flops the warp-MMA kernel issues: 64-row query tiles x 64-key tiles."""
+    b, d = wl.block_size, wl.d
+    N = -(-wl.L // b)
+    tiles = N * (k_sel + chunks_per_block) * wl.B * wl.H
+    first = (2.0 * N * 64 * d * d * wl.B * wl.H) if wl.mode == "hyd" else 0.0
+    return tiles * 4.0 * d * 64 * 64 + first
+
+
+def stats_bytes(wl):
+    e = 2 if wl.dtype == "bf16" else 4
+    base = 3.0 * wl.B * wl.H * wl.L * wl.d * e
+    return base + (2.0 * wl.B * wl.H * wl.L * wl.d * e if wl.cov_weight else 0.0)
+
+
+def k3_compulsory_bytes(wl):
+    e = 2 if wl.dtype == "bf16" else 4
+    N = -(-wl.L // wl.block_size)
+    return 4.0 * wl.B * wl.H * wl.L * wl.d * e + wl.B * wl.H * (2 * N * wl.d * 2 + wl.d * wl.d * 2)
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# the fp64 oracle on host cores
+# ----------------------------------------------------------------------------
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(wl, n_heads: int, n_blocks: int, seed: int = 7):
+    """Times the oracle on `n_heads` heads' statistics and `n_blocks` query blocks
+    (spread over those heads).  Returns (seconds per full workload extrapolated,
+    description)."""
+    import oracle as O
+    N = -(-wl.L // wl.block_size)
+    rng = np.random.default_rng(seed)
+    heads = [(0, h) for h in range(min(n_heads, wl.H))]
+    per_head = max(1, n_blocks // len(heads))
+    t_stats = t_rows = 0.0
+    rows_done = 0
+    for (b, h) in heads:
+        q, k, v = (x.double().numpy() for x in generate_head(wl, b, h, "cpu"))
+        blocks = sorted(set([0, N - 1] + list(rng.choice(N, size=min(per_head, N),
+                                                          replace=False))))[:per_head]
+        t0 = time.perf_counter()
+        st = O.block_stats(q, k, v, wl.block_size)
+        cov = None
+        if wl.cov_weight:
+            cov = O.covariance_norms(k, v, wl.block_size, st["kbar"], st["hbar"])
+        t1 = time.perf_counter()
+        k_sel = O.num_selected(N, wl.density)
+        sc = O.selection_scores(st["qbar"], st["kbar"], wl.scale, cov, wl.cov_weight, blocks)
+        idx = O.select_blocks(sc, k_sel, wl.sink_idx)
+        sel = np.zeros((N, k_sel), dtype=np.int64)
+        sel[blocks] = idx
+        O.piecewise_attention(q, k, v, wl.block_size, sel, st, wl.scale, wl.mode,
+                              query_blocks=blocks)
+        t2 = time.perf_counter()
+        t_stats += t1 - t0
+        t_rows += t2 - t1
+        rows_done += len(blocks)
+    BH = wl.B * wl.H
+    full = t_stats / len(heads) * BH + t_rows / rows_done * BH * N
+    desc = (f"oracle (fp64 numpy) on {len(heads)} head(s) of statistics and {rows_done} query "
+            f"blocks ({t_stats + t_rows:.1f} s), extrapolated linearly to {BH} heads x {N} "
+            f"query blocks")
+    return full, t_stats + t_rows, desc
+
+
+# ----------------------------------------------------------------------------
+# arms
+# ----------------------------------------------------------------------------
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, wl):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    cores = _blas_threads()
+    N = -(-wl.L // wl.block_size)
+    # one step = a bounded sample of the workload, extrapolated to the whole problem
+    n_blocks = 16 if wl.L > 20000 else 8
+    for _ in range(args.warmup):
+        oracle_sample(wl, 1, n_blocks)
+    times, wall = [], 0.0
+    desc = ""
+    for s in range(args.steps):
+        full, spent, desc = oracle_sample(wl, 1, n_blocks, seed=100 + s)
+        times.append(full)
+        wall += spent
+    t = statistics.median(times)
+    val = dense_flops(wl) / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(wl),
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(wl):
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "head_dim": wl.d,
+            "block_size": wl.block_size, "density": wl.density, "mode": wl.mode,
+            "sink_idx": wl.sink_idx, "cov_weight": wl.cov_weight, "io_dtype": wl.dtype,
+            "inputs": "seeded clustered Q/K (std 0.5 noise), V ~ N(0,1)",
+            "l2": "inputs larger than L2 (no flush)" if 3 * wl.B * wl.H * wl.L * wl.d * 2 > 126e6
+            else "L2 flushed between steps"}
+
+
+def run_pisa(args, wl):
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    from block_sparse_attention_stats_b200 import _lib
+    import block_sparse_attention_stats_b200 as P
+    _lib.load()
+
+    # independent problem per rank (weak scaling)
+    wl_r = wl.with_(seed=wl.seed + 1000 * rank) if rank else wl
+    Q, K, V = generate_qkv(wl_r, dev)
+    out = torch.empty_like(Q)
+    want_cov = wl.cov_weight != 0.0
+    ws_bytes = P.pisa_workspace_bytes(wl.B, wl.H, wl.L, wl.d, wl.block_size, wl.density,
+                                      wl.torch_dtype, want_cov)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    l2_flush = None
+    if 3 * Q.numel() * Q.element_size() <= 126e6:
+        l2_flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        P.pisa_attention_ex(Q, K, V, wl.density, wl.block_size, wl.sink_idx, wl.mode,
+                            cov_weight=wl.cov_weight, workspace=ws, out=out)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    P.pisa_device_status()
+    barrier()
+
+    # ---- timed region: the whole path ----------------------------------------
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    barrier()
+    for s in range(args.steps):
+        if l2_flush is not None:
+            l2_flush.zero_()
+        evs[2 * s].record(stream)
+        step()
+        evs[2 * s + 1].record(stream)
+    barrier()
+    step_ms = [evs[2 * s].elapsed_time(evs[2 * s + 1]) for s in range(args.steps)]
+    t_step = sum(step_ms) / len(step_ms)
+
+    # ---- per-kernel breakdown (same kernels, step by step through the C ABI) --
+    lib = _lib.load()
+    mk = lambda n: torch.empty(max(256, int(n)), dtype=torch.uint8, device=dev)
+    st_ws = mk(lib.pisa_block_stats_workspace_bytes(wl.B, wl.H, wl.L, wl.d, wl.block_size))
+    N_ = -(-wl.L // wl.block_size)
+    sel_ws = mk(lib.pisa_select_workspace_bytes(wl.B, wl.H, N_))
+    k3_ws = mk(lib.pisa_sparse_attention_workspace_bytes(wl.B, wl.H, wl.L, wl.d,
+                                                         wl.block_size,
+                                                         0 if wl.dtype == "bf16" else 1))
+    stt = P.pisa_block_stats(Q, K, V, wl.block_size, want_cov=want_cov, workspace=st_ws)
+    idx = P.pisa_select(stt["qbar"], stt["kbar"], wl.density, wl.sink_idx, cov=stt["cov"],
+                        cov_weight=wl.cov_weight, workspace=sel_ws)
+    torch.cuda.synchronize()
+    n_rep = max(3, min(args.steps, 10))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_rep)]
+    for s in range(n_rep):
+        if l2_flush is not None:
+            l2_flush.zero_()
+        e = ev[s]
+        e[0].record(stream)
+        P.pisa_block_stats(Q, K, V, wl.block_size, want_cov=want_cov, workspace=st_ws, out=stt)
+        e[1].record(stream)
+        P.pisa_select(stt["qbar"], stt["kbar"], wl.density, wl.sink_idx, cov=stt["cov"],
+                      cov_weight=wl.cov_weight, workspace=sel_ws, out=idx)
+        e[2].record(stream)
+        P.pisa_sparse_attention(Q, K, V, stt["kbar"], stt["vsum"], stt["hbar"], idx,
+                                mode=wl.mode, out=out, workspace=k3_ws)
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    parts = {"block_stats": [e[0].elapsed_time(e[1]) for e in ev],
+             "select": [e[1].elapsed_time(e[2]) for e in ev],
+             "sparse_attention": [e[2].elapsed_time(e[3]) for e in ev]}
+    clocks = clk.stop()
+    P.pisa_device_status()
+    part_ms = {k: sum(v) / len(v) for k, v in parts.items()}
+
+    # ---- dense attention kernel, same inputs -----------------------------------
+    dense = None
+    if not args.no_dense:
+        P.pisa_dense_attention(Q, K, V, out=out)
+        torch.cuda.synchronize()
+        reps = 2 if wl.L > 20000 else 10
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            P.pisa_dense_attention(Q, K, V, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dms = e0.elapsed_time(e1) / reps
+        dense = {"ms": dms, "tflops": dense_flops(wl) / (dms * 1e-3) / 1e12,
+                 "kernel": "pisa_dense_attention (all blocks exact, same kernel family)"}
+
+    # ---- e2e: public API with pinned host buffers ------------------------------
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+        hk = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+        hv = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+        ho = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+        hq.copy_(Q)
+        hk.copy_(K)
+        hv.copy_(V)
+        dq, dk, dv, do = (torch.empty_like(Q) for _ in range(4))
+        e2e_steps = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            P.pisa_attention(dq, dk, dv, wl.density, wl.block_size, wl.sink_idx, wl.mode,
+                             out=do)
+            ho.copy_(do, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b2.record(stream)
+        barrier()
+        t_e2e = a.elapsed_time(b2) / e2e_steps
+        nbytes = Q.numel() * Q.element_size()
+        e2e = {"t_ms": t_e2e, "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
+        del dq, dk, dv, do
+
+    # ---- max over ranks --------------------------------------------------------
+    t_vec = torch.tensor([t_step, part_ms["sparse_attention"],
+                          e2e["t_ms"] if e2e else 0.0], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t_vec, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+    t_step, t_k3, t_e2e = (float(x) for x in t_vec.tolist())
+
+    N = -(-wl.L // wl.block_size)
+    k_sel = idx.shape[-1]
+    f_alg = k3_algorithmic_flops(wl, idx)
+    n_chunks = -(-N // 64)
+    f_exec = k3_executed_flops(wl, k_sel, n_chunks)
+    peaks, peak_kind = _peaks()
+    p_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    p_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = f_alg / (t_k3 * 1e-3) / 1e12
+    src = _k3_source_hash()
+    traffic = K3_TRAFFIC.get(src)
+    launches_per_step = 2 + (1 if want_cov else 0) + 2 + 2 + (3 if wl.dtype == "f32" else 0)
+    line = {
+        "metric": METRIC,
+        "value": world * dense_flops(wl) / (t_step * 1e-3) / 1e12,
+        "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": t_step, "ms_per_call": t_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32-in/bf16-mma",
+        "data": "synthetic", "config": _config(wl),
+        "kernels_ms": part_ms,
+        "roofline": {
+            "kernel": "piecewise_attention (fused exact + centroid tail + first-order)",
+            "bound": "tensor", "achieved": achieved, "peak": p_sus,
+            "peak_kind": f"bf16 dense, sustained, {peak_kind}", "unit": "TFLOP/s",
+            "frac": achieved / p_sus, "frac_vs_burst": achieved / p_burst,
+            "traffic": traffic, "algorithmic_tflop_per_launch": f_alg / 1e12,
+            "executed_tflop_per_launch": f_exec / 1e12,
+            "executed_frac": f_exec / (t_k3 * 1e-3) / 1e12 / p_sus,
+            "kernel_src": src,
+        },
+        "step_roofline": {
+            "t_star_ms": 1e3 * max((f_alg + 2.0 * wl.L * wl.d ** 2 * wl.B * wl.H) / (p_burst * 1e12),
+                                   (stats_bytes(wl) + k3_compulsory_bytes(wl))
+                                   / (peaks.get("hbm_gbs", 6650.0) * 1e9)),
+        },
+        "dense_baseline": dense,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    line["step_roofline"]["frac"] = line["step_roofline"]["t_star_ms"] / t_step
+    if e2e:
+        line["e2e"] = {"value": world * dense_flops(wl) / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
+                       "ms_per_step": t_e2e, "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                       "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
+                       "api": "pisa_attention (C ABI) from pinned host buffers"}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        big = wl.L > 20000
+        full, spent, desc = oracle_sample(wl, 2 if big else wl.H,
+                                          1024 if big else wl.H * (-(-wl.L // wl.block_size)))
+        line["cpu_baseline"] = {"value": dense_flops(wl) / full / 1e12, "unit": UNIT,
+                                "cores": _blas_threads(), "kind": "oracle",
+                                "sample": desc, "extrapolated_s": full}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="wan", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="pisa", choices=["pisa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_pisa(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,18 @@
+"""PISA piecewise sparse attention on NVIDIA B200 (sm_100a).
+
+The compute lives in libpisa.so (hand-written CUDA kernels behind the C ABI of
+include/pisa.h); this package is its thin Python binding.
+"""
+from .api import (  # noqa: F401
+    PisaError,
+    pisa_attention,
+    pisa_attention_ex,
+    pisa_block_stats,
+    pisa_dense_attention,
+    pisa_device_status,
+    pisa_num_blocks,
+    pisa_num_selected,
+    pisa_select,
+    pisa_sparse_attention,
+    pisa_workspace_bytes,
+)

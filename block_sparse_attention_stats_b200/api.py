@@ -1,0 +1,207 @@
+"""Python binding of libpisa: argument marshalling only.
+
+Each function has the name of the C entry point it calls (include/pisa.h),
+takes CUDA torch tensors, passes their device pointers and the current CUDA
+stream, and raises PisaError on a non-OK status.  Every step of the path runs
+in libpisa's CUDA kernels; torch only provides device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+
+_DT = {torch.bfloat16: L.PISA_BF16, torch.float32: L.PISA_F32}
+_MODE = {"hyd": L.PISA_MODE_HYD, "0th": L.PISA_MODE_0TH}
+
+
+class PisaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        lib = L.load()
+        msg = lib.pisa_status_string(status).decode()
+        last = lib.pisa_last_error().decode()
+        super().__init__(f"{fn}: {msg} (status {status}){' - ' + last if last else ''}")
+        self.status = status
+
+
+def _check(fn: str, status: int):
+    if status != L.PISA_OK:
+        raise PisaError(fn, status)
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _sink(sink_idx: Optional[int]) -> int:
+    if sink_idx is None:
+        return L.PISA_SINK_NONE
+    if sink_idx not in (0, -1):
+        raise ValueError("sink_idx must be None, 0 or -1")
+    return sink_idx
+
+
+def _qkv_dims(q, k, v):
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must be [B, H, L, d] with equal shapes")
+    if q.dtype != k.dtype or q.dtype != v.dtype or q.dtype not in _DT:
+        raise ValueError("q, k, v must share dtype bf16 or float32")
+    return q.shape
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ---- sizes ------------------------------------------------------------------
+
+def pisa_num_blocks(L_: int, block_size: int = 64) -> int:
+    return L.load().pisa_num_blocks(L_, block_size)
+
+
+def pisa_num_selected(N: int, density: float) -> int:
+    return L.load().pisa_num_selected(N, float(density))
+
+
+def pisa_workspace_bytes(B, H, L_, d, block_size, density, dtype=torch.bfloat16,
+                         want_cov=False) -> int:
+    return L.load().pisa_workspace_bytes(B, H, L_, d, block_size, float(density), _DT[dtype],
+                                         int(bool(want_cov)))
+
+
+# ---- the three steps ----------------------------------------------------------
+
+def pisa_block_stats(q, k, v, block_size: int = 64, want_cov: bool = False,
+                     workspace: Optional[torch.Tensor] = None, out: Optional[dict] = None,
+                     stream=None):
+    """Returns dict(qbar, kbar, vsum [B,H,N,d], hbar [B,H,d,d], cov [B,H,N] or None).
+    `out` may pass a dict of preallocated outputs of those shapes."""
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    N = lib.pisa_num_blocks(Ln, block_size)
+    f = dict(dtype=torch.float32, device=q.device)
+    if out is not None:
+        qbar, kbar, vsum, hbar, cov = (out[n] for n in ("qbar", "kbar", "vsum", "hbar", "cov"))
+    else:
+        qbar, kbar, vsum = (torch.empty((B, H, N, d), **f) for _ in range(3))
+        hbar = torch.empty((B, H, d, d), **f)
+        cov = torch.empty((B, H, N), **f) if want_cov else None
+    need = lib.pisa_block_stats_workspace_bytes(B, H, Ln, d, block_size)
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check("pisa_block_stats", lib.pisa_block_stats(
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], B, H, Ln, d, block_size, int(want_cov),
+        _ptr(qbar), _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(cov), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return dict(qbar=qbar, kbar=kbar, vsum=vsum, hbar=hbar, cov=cov)
+
+
+def pisa_select(qbar, kbar, density: float, sink_idx: Optional[int] = None,
+                cov: Optional[torch.Tensor] = None, cov_weight: float = 0.0,
+                scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Returns idx [B, H, N, k_sel] int32, ascending per row."""
+    lib = L.load()
+    B, H, N, d = qbar.shape
+    s = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    k_sel = lib.pisa_num_selected(N, float(density))
+    if k_sel < 1:
+        raise ValueError("density must be in (0, 1]")
+    idx = torch.empty((B, H, N, k_sel), dtype=torch.int32, device=qbar.device) \
+        if out is None else out
+    need = lib.pisa_select_workspace_bytes(B, H, N)
+    ws = workspace if workspace is not None else _workspace(need, qbar.device)
+    _check("pisa_select", lib.pisa_select(
+        _ptr(qbar), _ptr(kbar), _ptr(cov), float(cov_weight), s, B, H, N, d, float(density),
+        _sink(sink_idx), _ptr(idx), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return idx
+
+
+def pisa_sparse_attention(q, k, v, kbar, vsum, hbar, idx, mode: str = "hyd",
+                          block_size: int = 64, scale: Optional[float] = None,
+                          out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None, stream=None):
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    k_sel = idx.shape[-1]
+    out = torch.empty_like(q) if out is None else out
+    need = lib.pisa_sparse_attention_workspace_bytes(B, H, Ln, d, block_size, _DT[q.dtype])
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check("pisa_sparse_attention", lib.pisa_sparse_attention(
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(idx),
+        k_sel, B, H, Ln, d, block_size, 0.0 if scale is None else float(scale), _MODE[mode],
+        _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+# ---- the whole path --------------------------------------------------------------
+
+def pisa_attention(q, k, v, density: float, block_size: int = 64,
+                   sink_idx: Optional[int] = None, mode: str = "hyd",
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16 piecewise sparse attention with default options (scratch memory is
+    allocated stream-ordered inside the library)."""
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    _check("pisa_attention", lib.pisa_attention(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Ln, d, block_size, float(density),
+        _sink(sink_idx), _MODE[mode], _stream(stream)))
+    return out
+
+
+def pisa_attention_ex(q, k, v, density: float, block_size: int = 64,
+                      sink_idx: Optional[int] = None, mode: str = "hyd",
+                      scale: Optional[float] = None, cov_weight: float = 0.0,
+                      workspace: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pisa_attention with options; the workspace (if given) is caller-owned scratch
+    of pisa_workspace_bytes(...) bytes and nothing is allocated by the library."""
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    opts = L.PisaOptions()
+    opts.scale = 0.0 if scale is None else float(scale)
+    opts.cov_weight = float(cov_weight)
+    opts.dtype = _DT[q.dtype]
+    if workspace is not None:
+        opts.workspace = _ptr(workspace)
+        opts.ws_bytes = workspace.numel() * workspace.element_size()
+    _check("pisa_attention_ex", lib.pisa_attention_ex(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Ln, d, block_size, float(density),
+        _sink(sink_idx), _MODE[mode], ctypes.byref(opts), _stream(stream)))
+    return out
+
+
+def pisa_dense_attention(q, k, v, scale: Optional[float] = None,
+                         out: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    need = lib.pisa_dense_attention_workspace_bytes(B, H, Ln, d, _DT[q.dtype])
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check("pisa_dense_attention", lib.pisa_dense_attention(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _DT[q.dtype], B, H, Ln, d,
+        0.0 if scale is None else float(scale), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    return out
+
+
+def pisa_device_status(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel flagged a device-side error."""
+    _check("pisa_device_status", L.load().pisa_device_status(_stream(stream)))

@@ -1,0 +1,412 @@
+// K1: block statistics of PISA (pre-computation phase).
+//
+// "Technical Summary: PISA" (gist.science), section 2: "Hardware
+// Implementation" step 1 (block centroids, value sums and the global statistic
+// Hbar), "Core Algorithm" (kbar_j, sum of values), "Global First-Order
+// Correction" (Hbar = mean of the block-wise first-order matrices) and
+// "Covariance-Aware Routing" (M_j = ||H_j - Hbar||).
+//
+// Per (b, h) and block j of n_j tokens:
+//   qbar_j = (1/n_j) sum_n q_n          kbar_j = (1/n_j) sum_n k_n
+//   vsum_j = sum_n v_n                   H_j = sum_n k_n^T v_n - kbar_j^T vsum_j
+//   hbar = (1/N) sum_j H_j               cov_j = ||H_j - hbar||_F
+// (sum_n (k_n - kbar_j)^T v_n = sum_n k_n^T v_n - n_j kbar_j^T vbar_j.)
+//
+// Pass 1 (stats_pass_*): one CTA per (chunk of consecutive blocks, head).  It
+// streams the Q/K/V tiles of its blocks once, writes qbar/kbar/vsum, and keeps
+// sum_j H_j of its chunk in registers; the chunk partial goes to scratch.
+// Pass 2 (hbar_reduce): sums the chunk partials in chunk order -> hbar.
+// Pass 3 (cov_pass_*, only with covariance-aware scoring): re-streams K/V,
+// rebuilds each H_j and reduces ||H_j - hbar||_F.
+// Reduction orders are fixed, so the results are bitwise reproducible.
+#pragma once
+
+#include "pisa_common.cuh"
+
+namespace pisa {
+
+constexpr int kStatsThreads = 256;
+constexpr int kBlk = 64;  // tokens per block (block_size)
+
+// Chunking of pass 1: about two CTAs per SM over the whole problem.
+__host__ __device__ inline int stats_num_chunks(int BH, int N) {
+  int want = (2 * 148 + BH - 1) / BH;
+  if (want < 1) want = 1;
+  return want < N ? want : N;
+}
+
+// ---------------------------------------------------------------------------
+// bf16 pass 1: tensor-core K_j^T V_j with mma.sync, cp.async double buffering.
+// ---------------------------------------------------------------------------
+template <int D> struct StatsMmaCfg {
+  static constexpr int kWarpsM = (D == 128) ? 4 : 2;
+  static constexpr int kWarpsN = 8 / kWarpsM;
+  static constexpr int kWarpRows = D / kWarpsM;  // 32
+  static constexpr int kWarpCols = D / kWarpsN;  // 64 (D=128) or 16 (D=64)
+  static constexpr int kMT = kWarpRows / 16;     // 2
+  static constexpr int kNT = kWarpCols / 8;      // 8 or 2
+  static constexpr int kTileBytes = kBlk * D * 2;
+};
+
+template <int D>
+__device__ __forceinline__ void stats_load_tile_bf16(uint32_t dst, const __nv_bfloat16 *src,
+                                                     int valid_rows) {
+  constexpr int kChunksPerRow = D / 8;
+  constexpr int kChunks = kBlk * kChunksPerRow;
+  for (int c = threadIdx.x; c < kChunks; c += kStatsThreads) {
+    int row = c / kChunksPerRow, col = (c % kChunksPerRow) * 8;
+    bool ok = row < valid_rows;
+    const __nv_bfloat16 *g = src + (size_t)(ok ? row : 0) * D + col;
+    cp_async_16(dst + SwizzledTile<D>::offset(row, col), g, ok ? 16 : 0);
+  }
+}
+
+// Accumulates acc += K^T V for one 64-token tile pair (swizzled smem tiles).
+template <int D>
+__device__ __forceinline__ void ktv_mma(float (&acc)[StatsMmaCfg<D>::kMT][StatsMmaCfg<D>::kNT][4],
+                                        uint32_t sK, uint32_t sV, int warp_m0, int warp_n0,
+                                        int lane) {
+  using C = StatsMmaCfg<D>;
+  const int mi = lane >> 3, r = lane & 7;
+#pragma unroll
+  for (int k0 = 0; k0 < kBlk; k0 += 16) {
+    uint32_t a[C::kMT][4];
+#pragma unroll
+    for (int mt = 0; mt < C::kMT; ++mt) {
+      int tok = k0 + r + 8 * (mi >> 1);
+      int dim = warp_m0 + mt * 16 + 8 * (mi & 1);
+      ldmatrix_x4_trans(sK + SwizzledTile<D>::offset(tok, dim), a[mt][0], a[mt][1], a[mt][2],
+                        a[mt][3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < C::kNT; nt += 2) {
+      int tok = k0 + r + 8 * (mi & 1);
+      int dim = warp_n0 + nt * 8 + 8 * (mi >> 1);
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(sV + SwizzledTile<D>::offset(tok, dim), b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < C::kMT; ++mt) {
+        mma_bf16_16816(acc[mt][nt], a[mt], b0, b1);
+        mma_bf16_16816(acc[mt][nt + 1], a[mt], b2, b3);
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kStatsThreads)
+    stats_pass_bf16_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+                           const __nv_bfloat16 *__restrict__ V, int L, int N, int nchunk,
+                           float *__restrict__ qbar, float *__restrict__ kbar,
+                           float *__restrict__ vsum, float *__restrict__ partial) {
+  using C = StatsMmaCfg<D>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  // [stage][Q,K,V] tiles, then column sums (3 x D floats)
+  float *colsum = reinterpret_cast<float *>(smem + 2 * 3 * C::kTileBytes);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int per = ceil_div(N, nchunk);
+  const int j0 = chunk * per, j1 = min(N, j0 + per);
+  const size_t head = (size_t)bh * L * D;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp_m0 = (warp / C::kWarpsN) * C::kWarpRows;
+  const int warp_n0 = (warp % C::kWarpsN) * C::kWarpCols;
+
+  float acc[C::kMT][C::kNT][4];
+#pragma unroll
+  for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < C::kNT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+
+  auto issue = [&](int j, int stage) {
+    int valid = min(kBlk, L - j * kBlk);
+    size_t off = head + (size_t)j * kBlk * D;
+    uint32_t st = sbase + stage * 3 * C::kTileBytes;
+    stats_load_tile_bf16<D>(st, Q + off, valid);
+    stats_load_tile_bf16<D>(st + C::kTileBytes, K + off, valid);
+    stats_load_tile_bf16<D>(st + 2 * C::kTileBytes, V + off, valid);
+  };
+
+  if (j0 < j1) issue(j0, 0);
+  cp_async_commit();
+  for (int j = j0; j < j1; ++j) {
+    const int stage = (j - j0) & 1;
+    if (j + 1 < j1) issue(j + 1, stage ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+
+    const unsigned char *tiles = smem + stage * 3 * C::kTileBytes;
+    const int n_j = min(kBlk, L - j * kBlk);
+    // column sums of Q, K, V (zero-filled rows past L add nothing)
+    for (int t = tid; t < 3 * D; t += kStatsThreads) {
+      const int which = t / D, col = t % D;
+      const unsigned char *tile = tiles + which * C::kTileBytes;
+      float s = 0.f;
+#pragma unroll 8
+      for (int row = 0; row < kBlk; ++row)
+        s += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+            tile + SwizzledTile<D>::offset(row, col)));
+      colsum[t] = s;
+    }
+    const uint32_t sK = sbase + stage * 3 * C::kTileBytes + C::kTileBytes;
+    ktv_mma<D>(acc, sK, sK + C::kTileBytes, warp_m0, warp_n0, lane);
+    __syncthreads();  // colsum visible
+
+    const float inv_n = 1.f / (float)n_j;
+    const size_t so = ((size_t)bh * N + j) * D;
+    for (int t = tid; t < 3 * D; t += kStatsThreads) {
+      const int which = t / D, col = t % D;
+      if (which == 0) qbar[so + col] = colsum[t] * inv_n;
+      else if (which == 1) kbar[so + col] = colsum[t] * inv_n;
+      else vsum[so + col] = colsum[t];
+    }
+    // acc -= kbar_j^T vsum_j
+    const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < C::kNT; ++nt) {
+        const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
+        const float ka = colsum[D + a0] * inv_n, kb = colsum[D + a0 + 8] * inv_n;
+        const float v0 = colsum[2 * D + c0], v1 = colsum[2 * D + c0 + 1];
+        acc[mt][nt][0] -= ka * v0;
+        acc[mt][nt][1] -= ka * v1;
+        acc[mt][nt][2] -= kb * v0;
+        acc[mt][nt][3] -= kb * v1;
+      }
+    __syncthreads();  // stage and colsum free for reuse
+  }
+  cp_async_wait<0>();
+
+  float *P = partial + ((size_t)bh * nchunk + chunk) * D * D;
+  const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < C::kNT; ++nt) {
+      const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
+      *reinterpret_cast<float2 *>(P + (size_t)a0 * D + c0) =
+          make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+      *reinterpret_cast<float2 *>(P + (size_t)(a0 + 8) * D + c0) =
+          make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// f32 pass 1: plain FMA version (small f32 workloads).
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kStatsThreads)
+    stats_pass_f32_kernel(const float *__restrict__ Q, const float *__restrict__ K,
+                          const float *__restrict__ V, int L, int N, int nchunk,
+                          float *__restrict__ qbar, float *__restrict__ kbar,
+                          float *__restrict__ vsum, float *__restrict__ partial) {
+  constexpr int kPer = D * D / kStatsThreads;
+  extern __shared__ __align__(128) unsigned char smem[];
+  float *sQ = reinterpret_cast<float *>(smem);
+  float *sK = sQ + kBlk * D;
+  float *sV = sK + kBlk * D;
+  float *colsum = sV + kBlk * D;  // 3 x D
+
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int per = ceil_div(N, nchunk);
+  const int j0 = chunk * per, j1 = min(N, j0 + per);
+  const size_t head = (size_t)bh * L * D;
+  const int tid = threadIdx.x;
+  float acc[kPer];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) acc[r] = 0.f;
+
+  for (int j = j0; j < j1; ++j) {
+    const int n_j = min(kBlk, L - j * kBlk);
+    const size_t off = head + (size_t)j * kBlk * D;
+    for (int e = tid; e < kBlk * D; e += kStatsThreads) {
+      const bool ok = e < n_j * D;
+      sQ[e] = ok ? Q[off + e] : 0.f;
+      sK[e] = ok ? K[off + e] : 0.f;
+      sV[e] = ok ? V[off + e] : 0.f;
+    }
+    __syncthreads();
+    for (int t = tid; t < 3 * D; t += kStatsThreads) {
+      const float *tile = (t < D) ? sQ : (t < 2 * D ? sK : sV);
+      const int col = t % D;
+      float s = 0.f;
+      for (int row = 0; row < kBlk; ++row) s += tile[row * D + col];
+      colsum[t] = s;
+    }
+    __syncthreads();
+    const float inv_n = 1.f / (float)n_j;
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int e = tid + r * kStatsThreads, a = e / D, c = e % D;
+      float s = 0.f;
+      for (int row = 0; row < kBlk; ++row) s += sK[row * D + a] * sV[row * D + c];
+      acc[r] += s - (colsum[D + a] * inv_n) * colsum[2 * D + c];
+    }
+    const size_t so = ((size_t)bh * N + j) * D;
+    for (int t = tid; t < 3 * D; t += kStatsThreads) {
+      const int col = t % D;
+      if (t < D) qbar[so + col] = colsum[t] * inv_n;
+      else if (t < 2 * D) kbar[so + col] = colsum[t] * inv_n;
+      else vsum[so + col] = colsum[t];
+    }
+    __syncthreads();
+  }
+  float *P = partial + ((size_t)bh * nchunk + chunk) * D * D;
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) P[tid + r * kStatsThreads] = acc[r];
+}
+
+// ---------------------------------------------------------------------------
+// pass 2: hbar = (1/N) sum over chunk partials, in chunk order.
+// ---------------------------------------------------------------------------
+__global__ void hbar_reduce_kernel(const float *__restrict__ partial, int nchunk, int DD, int N,
+                                   float *__restrict__ hbar) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= DD) return;
+  const float *p = partial + (size_t)bh * nchunk * DD + e;
+  float s = 0.f;
+  for (int c = 0; c < nchunk; ++c) s += p[(size_t)c * DD];
+  hbar[(size_t)bh * DD + e] = s / (float)N;
+}
+
+// ---------------------------------------------------------------------------
+// pass 3: cov_j = ||H_j - hbar||_F
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float block_reduce_sum(float v, float *red) {
+  // fixed-order reduction: butterfly inside each warp, then warp 0 over warps
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (warp == 0) {
+    t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  }
+  __syncthreads();
+  return t;  // valid in warp 0
+}
+
+template <int D>
+__global__ void __launch_bounds__(kStatsThreads)
+    cov_pass_bf16_kernel(const __nv_bfloat16 *__restrict__ K, const __nv_bfloat16 *__restrict__ V,
+                         int L, int N, int nchunk, const float *__restrict__ kbar,
+                         const float *__restrict__ vsum, const float *__restrict__ hbar,
+                         float *__restrict__ cov) {
+  using C = StatsMmaCfg<D>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  float *red = reinterpret_cast<float *>(smem + 2 * 2 * C::kTileBytes);
+  const uint32_t sbase = smem_u32(smem);
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int per = ceil_div(N, nchunk);
+  const int j0 = chunk * per, j1 = min(N, j0 + per);
+  const size_t head = (size_t)bh * L * D;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp_m0 = (warp / C::kWarpsN) * C::kWarpRows;
+  const int warp_n0 = (warp % C::kWarpsN) * C::kWarpCols;
+  const int g = lane >> 2, tq = lane & 3;
+
+  // hbar entries matching this thread's accumulator fragment
+  float hb[C::kMT][C::kNT][4];
+  const float *Hb = hbar + (size_t)bh * D * D;
+#pragma unroll
+  for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < C::kNT; ++nt) {
+      const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
+      hb[mt][nt][0] = Hb[a0 * D + c0];
+      hb[mt][nt][1] = Hb[a0 * D + c0 + 1];
+      hb[mt][nt][2] = Hb[(a0 + 8) * D + c0];
+      hb[mt][nt][3] = Hb[(a0 + 8) * D + c0 + 1];
+    }
+
+  auto issue = [&](int j, int stage) {
+    int valid = min(kBlk, L - j * kBlk);
+    size_t off = head + (size_t)j * kBlk * D;
+    uint32_t st = sbase + stage * 2 * C::kTileBytes;
+    stats_load_tile_bf16<D>(st, K + off, valid);
+    stats_load_tile_bf16<D>(st + C::kTileBytes, V + off, valid);
+  };
+  if (j0 < j1) issue(j0, 0);
+  cp_async_commit();
+  for (int j = j0; j < j1; ++j) {
+    const int stage = (j - j0) & 1;
+    if (j + 1 < j1) issue(j + 1, stage ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    float acc[C::kMT][C::kNT][4];
+#pragma unroll
+    for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < C::kNT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    const uint32_t sK = sbase + stage * 2 * C::kTileBytes;
+    ktv_mma<D>(acc, sK, sK + C::kTileBytes, warp_m0, warp_n0, lane);
+    const float *kb = kbar + ((size_t)bh * N + j) * D;
+    const float *vs = vsum + ((size_t)bh * N + j) * D;
+    float ss = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < C::kNT; ++nt) {
+        const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
+        const float ka = kb[a0], kc = kb[a0 + 8], v0 = vs[c0], v1 = vs[c0 + 1];
+        float e0 = acc[mt][nt][0] - ka * v0 - hb[mt][nt][0];
+        float e1 = acc[mt][nt][1] - ka * v1 - hb[mt][nt][1];
+        float e2 = acc[mt][nt][2] - kc * v0 - hb[mt][nt][2];
+        float e3 = acc[mt][nt][3] - kc * v1 - hb[mt][nt][3];
+        ss += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+      }
+    __syncthreads();  // tiles of this stage consumed
+    float tot = block_reduce_sum(ss, red);
+    if (tid == 0) cov[(size_t)bh * N + j] = sqrtf(tot);
+  }
+  cp_async_wait<0>();
+}
+
+template <int D>
+__global__ void __launch_bounds__(kStatsThreads)
+    cov_pass_f32_kernel(const float *__restrict__ K, const float *__restrict__ V, int L, int N,
+                        const float *__restrict__ kbar, const float *__restrict__ vsum,
+                        const float *__restrict__ hbar, float *__restrict__ cov) {
+  constexpr int kPer = D * D / kStatsThreads;
+  extern __shared__ __align__(128) unsigned char smem[];
+  float *sK = reinterpret_cast<float *>(smem);
+  float *sV = sK + kBlk * D;
+  float *red = sV + kBlk * D;
+  const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int n_j = min(kBlk, L - j * kBlk);
+  const size_t off = (size_t)bh * L * D + (size_t)j * kBlk * D;
+  for (int e = tid; e < kBlk * D; e += kStatsThreads) {
+    const bool ok = e < n_j * D;
+    sK[e] = ok ? K[off + e] : 0.f;
+    sV[e] = ok ? V[off + e] : 0.f;
+  }
+  __syncthreads();
+  const float *kb = kbar + ((size_t)bh * N + j) * D;
+  const float *vs = vsum + ((size_t)bh * N + j) * D;
+  const float *Hb = hbar + (size_t)bh * D * D;
+  float ss = 0.f;
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int e = tid + r * kStatsThreads, a = e / D, c = e % D;
+    float s = 0.f;
+    for (int row = 0; row < kBlk; ++row) s += sK[row * D + a] * sV[row * D + c];
+    const float h = s - kb[a] * vs[c] - Hb[e];
+    ss += h * h;
+  }
+  float tot = block_reduce_sum(ss, red);
+  if (tid == 0) cov[(size_t)bh * N + j] = sqrtf(tot);
+}
+
+}  // namespace pisa

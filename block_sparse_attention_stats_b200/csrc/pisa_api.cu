@@ -1,0 +1,494 @@
+// libpisa C ABI: argument checking, scratch layout and kernel launches.
+// One translation unit: every kernel header is included here.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <cmath>
+#include <string>
+
+#include "pisa.h"
+#include "pisa_common.cuh"
+#include "k1_block_stats.cuh"
+#include "k2_select.cuh"
+#include "k3_attention_mma.cuh"
+
+namespace pisa {
+
+static thread_local std::string t_last_error;
+
+void set_last_error(cudaError_t e) {
+  t_last_error = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
+}
+
+pisa_status check_launch() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error(e);
+    return PISA_ERR_CUDA;
+  }
+  return PISA_OK;
+}
+
+#define PISA_TRY(expr)                         \
+  do {                                         \
+    pisa_status _s = (expr);                   \
+    if (_s != PISA_OK) return _s;              \
+  } while (0)
+
+#define PISA_CUDA(expr)                        \
+  do {                                         \
+    cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) {                   \
+      set_last_error(_e);                      \
+      return PISA_ERR_CUDA;                    \
+    }                                          \
+  } while (0)
+
+static bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static pisa_status check_shape(int B, int H, int L, int d, int block_size) {
+  if (B < 1 || H < 1 || L < 1 || d < 1 || block_size < 1) return PISA_ERR_INVALID_ARG;
+  if ((long long)B * H > 65535) return PISA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return PISA_ERR_UNSUPPORTED;
+  if (block_size != 64) return PISA_ERR_UNSUPPORTED;
+  if ((long long)L > (1LL << 24)) return PISA_ERR_UNSUPPORTED;
+  return PISA_OK;
+}
+
+static int sink_block(int sink_idx, int N) {
+  if (sink_idx == PISA_SINK_NONE) return -1;
+  return sink_idx == 0 ? 0 : N - 1;
+}
+
+static bool sink_valid(int sink_idx) {
+  return sink_idx == PISA_SINK_NONE || sink_idx == 0 || sink_idx == -1;
+}
+
+// ---- scratch sizes --------------------------------------------------------
+static size_t stats_ws(int B, int H, int L, int d) {
+  const int N = ceil_div(L, 64), BH = B * H;
+  return align_up((size_t)BH * stats_num_chunks(BH, N) * d * d * sizeof(float), 256);
+}
+static size_t select_ws(int B, int H, int N) {
+  return align_up((size_t)B * H * N * N * sizeof(float), 256);
+}
+static size_t sparse_ws(int B, int H, int L, int d, pisa_dtype dt) {
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
+  const size_t BH = (size_t)B * H;
+  size_t s = 2 * align_up(BH * Npad * d * 2, 256) + align_up(BH * d * d * 2, 256);
+  if (dt == PISA_F32) s += 3 * align_up(BH * L * d * 2, 256);
+  return s;
+}
+
+struct PathLayout {
+  size_t qbar, kbar, vsum, hbar, cov, idx, scratch, total;
+};
+
+static PathLayout path_layout(int B, int H, int L, int d, double density, pisa_dtype dt,
+                              int want_cov) {
+  const int N = ceil_div(L, 64);
+  const size_t BH = (size_t)B * H;
+  const int k_sel = pisa_num_selected(N, density);
+  PathLayout p;
+  size_t o = 0;
+  const size_t st = align_up(BH * N * d * sizeof(float), 256);
+  p.qbar = o; o += st;
+  p.kbar = o; o += st;
+  p.vsum = o; o += st;
+  p.hbar = o; o += align_up(BH * d * d * sizeof(float), 256);
+  p.cov = o; o += want_cov ? align_up(BH * N * sizeof(float), 256) : 0;
+  p.idx = o; o += align_up(BH * N * (size_t)(k_sel > 0 ? k_sel : 1) * sizeof(int32_t), 256);
+  p.scratch = o;
+  size_t s = stats_ws(B, H, L, d);
+  s = s > select_ws(B, H, N) ? s : select_ws(B, H, N);
+  const size_t a = sparse_ws(B, H, L, d, dt);
+  s = s > a ? s : a;
+  o += s;
+  p.total = o;
+  return p;
+}
+
+static unsigned grid_1d(size_t n, int threads) {
+  size_t b = (n + threads - 1) / threads;
+  if (b > 148 * 32) b = 148 * 32;
+  return (unsigned)(b ? b : 1);
+}
+
+// ---- launches ---------------------------------------------------------------
+template <int D>
+static pisa_status launch_stats(const void *q, const void *k, const void *v, pisa_dtype dt,
+                                int BH, int L, int want_cov, float *qbar, float *kbar,
+                                float *vsum, float *hbar, float *cov, float *partial,
+                                cudaStream_t st) {
+  const int N = ceil_div(L, 64);
+  const int nchunk = stats_num_chunks(BH, N);
+  dim3 grid(nchunk, BH);
+  if (dt == PISA_BF16) {
+    const int smem = 2 * 3 * StatsMmaCfg<D>::kTileBytes + 3 * D * (int)sizeof(float);
+    PISA_CUDA(cudaFuncSetAttribute(stats_pass_bf16_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    stats_pass_bf16_kernel<D><<<grid, kStatsThreads, smem, st>>>(
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N,
+        nchunk, qbar, kbar, vsum, partial);
+  } else {
+    const int smem = 3 * kBlk * D * (int)sizeof(float) + 3 * D * (int)sizeof(float);
+    PISA_CUDA(cudaFuncSetAttribute(stats_pass_f32_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    stats_pass_f32_kernel<D><<<grid, kStatsThreads, smem, st>>>(
+        (const float *)q, (const float *)k, (const float *)v, L, N, nchunk, qbar, kbar, vsum,
+        partial);
+  }
+  PISA_TRY(check_launch());
+  hbar_reduce_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(partial, nchunk, D * D, N,
+                                                                      hbar);
+  PISA_TRY(check_launch());
+  if (want_cov) {
+    if (dt == PISA_BF16) {
+      const int smem = 2 * 2 * StatsMmaCfg<D>::kTileBytes + 32 * (int)sizeof(float);
+      PISA_CUDA(cudaFuncSetAttribute(cov_pass_bf16_kernel<D>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+      cov_pass_bf16_kernel<D><<<grid, kStatsThreads, smem, st>>>(
+          (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N, nchunk, kbar, vsum, hbar,
+          cov);
+    } else {
+      const int smem = 2 * kBlk * D * (int)sizeof(float) + 32 * (int)sizeof(float);
+      PISA_CUDA(cudaFuncSetAttribute(cov_pass_f32_kernel<D>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+      cov_pass_f32_kernel<D><<<dim3(N, BH), kStatsThreads, smem, st>>>(
+          (const float *)k, (const float *)v, L, N, kbar, vsum, hbar, cov);
+    }
+    PISA_TRY(check_launch());
+  }
+  return PISA_OK;
+}
+
+static pisa_status launch_select(const float *qbar, const float *kbar, const float *cov,
+                                 float cov_weight, float scale, int BH, int N, int d, int k_sel,
+                                 int sink, int32_t *idx, float *scores, cudaStream_t st) {
+  dim3 g1(ceil_div(N, kScoreTile), ceil_div(N, kScoreTile), BH);
+  scores_kernel<<<g1, 256, 0, st>>>(qbar, kbar, cov, cov_weight, scale, N, d, scores);
+  PISA_TRY(check_launch());
+  const int smem = N * (int)sizeof(uint32_t);
+  if (smem > 48 * 1024)
+    PISA_CUDA(cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  topk_kernel<<<(unsigned)((size_t)BH * N), kTopkThreads, smem, st>>>(scores, N, k_sel, sink,
+                                                                        idx);
+  return check_launch();
+}
+
+template <int D, bool DENSE>
+static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                                           const __nv_bfloat16 *v, const __nv_bfloat16 *kbar16,
+                                           const __nv_bfloat16 *vsum16,
+                                           const __nv_bfloat16 *hbar16, const int32_t *idx,
+                                           int k_sel, int BH, int L, float scale, int hyd,
+                                           void *out, int out_f32, cudaStream_t st) {
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
+  const int nwords = ceil_div(N, 32);
+  const int smem = AttnSmem<D>::kFixed +
+                   (DENSE ? 0 : (nwords + k_sel + ceil_div(N, 64)) * (int)sizeof(int));
+  if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
+  PISA_CUDA(cudaFuncSetAttribute(piecewise_attention_mma_kernel<D, DENSE>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  piecewise_attention_mma_kernel<D, DENSE><<<dim3(N, BH), kAttnThreads, smem, st>>>(
+      q, k, v, kbar16, vsum16, hbar16, idx, k_sel, L, N, Npad, scale, hyd, out, out_f32);
+  return check_launch();
+}
+
+static pisa_status to_bf16(const void *src, __nv_bfloat16 *dst, size_t n, cudaStream_t st) {
+  f32_to_bf16_kernel<<<grid_1d(n, 256), 256, 0, st>>>((const float *)src, dst, n);
+  return check_launch();
+}
+
+static pisa_status run_sparse_attention(const void *q, const void *k, const void *v,
+                                        pisa_dtype dt, const float *kbar, const float *vsum,
+                                        const float *hbar, const int32_t *idx, int k_sel, int BH,
+                                        int L, int d, float scale, pisa_mode mode, void *out,
+                                        unsigned char *ws, cudaStream_t st) {
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
+  __nv_bfloat16 *kbar16 = (__nv_bfloat16 *)ws;
+  __nv_bfloat16 *vsum16 = (__nv_bfloat16 *)(ws + align_up((size_t)BH * Npad * d * 2, 256));
+  __nv_bfloat16 *hbar16 = (__nv_bfloat16 *)(ws + 2 * align_up((size_t)BH * Npad * d * 2, 256));
+  unsigned char *next = ws + 2 * align_up((size_t)BH * Npad * d * 2, 256) +
+                        align_up((size_t)BH * d * d * 2, 256);
+  pack_stats_kernel<<<grid_1d((size_t)BH * (Npad * d + d * d), 256), 256, 0, st>>>(
+      kbar, vsum, hbar, N, Npad, d, BH, kbar16, vsum16, hbar16);
+  PISA_TRY(check_launch());
+  const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
+                      *v16 = (const __nv_bfloat16 *)v;
+  if (dt == PISA_F32) {
+    const size_t n = (size_t)BH * L * d, sz = align_up(n * 2, 256);
+    __nv_bfloat16 *a = (__nv_bfloat16 *)next, *b = (__nv_bfloat16 *)(next + sz),
+                  *c = (__nv_bfloat16 *)(next + 2 * sz);
+    PISA_TRY(to_bf16(q, a, n, st));
+    PISA_TRY(to_bf16(k, b, n, st));
+    PISA_TRY(to_bf16(v, c, n, st));
+    q16 = a;
+    k16 = b;
+    v16 = c;
+  }
+  const int hyd = mode == PISA_MODE_HYD;
+  const int of32 = dt == PISA_F32;
+  if (d == 128)
+    return launch_attention_kernel<128, false>(q16, k16, v16, kbar16, vsum16, hbar16, idx, k_sel,
+                                               BH, L, scale, hyd, out, of32, st);
+  return launch_attention_kernel<64, false>(q16, k16, v16, kbar16, vsum16, hbar16, idx, k_sel, BH,
+                                            L, scale, hyd, out, of32, st);
+}
+
+}  // namespace pisa
+
+using namespace pisa;
+
+// =============================================================================
+// C ABI
+// =============================================================================
+extern "C" {
+
+int pisa_num_blocks(int L, int block_size) {
+  if (L < 1 || block_size < 1) return -1;
+  return ceil_div(L, block_size);
+}
+
+int pisa_num_selected(int N, double density) {
+  if (N < 1 || !(density > 0.0) || density > 1.0) return -1;
+  double k = std::floor(density * (double)N + 1e-6);
+  if (k < 1.0) k = 1.0;
+  if (k > (double)N) k = (double)N;
+  return (int)k;
+}
+
+size_t pisa_block_stats_workspace_bytes(int B, int H, int L, int d, int block_size) {
+  if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
+  return stats_ws(B, H, L, d);
+}
+
+size_t pisa_select_workspace_bytes(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  return select_ws(B, H, N);
+}
+
+size_t pisa_sparse_attention_workspace_bytes(int B, int H, int L, int d, int block_size,
+                                             pisa_dtype dtype) {
+  if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
+  return sparse_ws(B, H, L, d, dtype);
+}
+
+size_t pisa_workspace_bytes(int B, int H, int L, int d, int block_size, double density,
+                            pisa_dtype dtype, int want_cov) {
+  if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
+  if (pisa_num_selected(ceil_div(L, 64), density) < 1) return 0;
+  return path_layout(B, H, L, d, density, dtype, want_cov).total;
+}
+
+pisa_status pisa_block_stats(const void *q, const void *k, const void *v, pisa_dtype dtype,
+                             int B, int H, int L, int d, int block_size, int want_cov,
+                             float *qbar, float *kbar, float *vsum, float *hbar, float *cov,
+                             void *workspace, size_t ws_bytes, pisa_stream_t stream) {
+  PISA_TRY(check_shape(B, H, L, d, block_size));
+  if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qbar) || !aligned16(kbar) ||
+      !aligned16(vsum) || !aligned16(hbar) || !aligned16(workspace))
+    return PISA_ERR_INVALID_ARG;
+  if (want_cov && !aligned16(cov)) return PISA_ERR_INVALID_ARG;
+  if (ws_bytes < stats_ws(B, H, L, d)) return PISA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  float *partial = (float *)workspace;
+  if (d == 128)
+    return launch_stats<128>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
+                             partial, st);
+  return launch_stats<64>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
+                          partial, st);
+}
+
+pisa_status pisa_select(const float *qbar, const float *kbar, const float *cov, float cov_weight,
+                        float scale, int B, int H, int N, int d, double density, int sink_idx,
+                        int32_t *idx, void *workspace, size_t ws_bytes, pisa_stream_t stream) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return PISA_ERR_INVALID_ARG;
+  if ((long long)B * H > 65535) return PISA_ERR_UNSUPPORTED;
+  if ((long long)N * 4 > 200 * 1024) return PISA_ERR_UNSUPPORTED;
+  if (!sink_valid(sink_idx) || !std::isfinite(scale) || !std::isfinite(cov_weight))
+    return PISA_ERR_INVALID_ARG;
+  const int k_sel = pisa_num_selected(N, density);
+  if (k_sel < 1) return PISA_ERR_INVALID_ARG;
+  if (!aligned16(qbar) || !aligned16(kbar) || !idx || !aligned16(workspace))
+    return PISA_ERR_INVALID_ARG;
+  if (cov_weight != 0.f && !cov) return PISA_ERR_INVALID_ARG;
+  if (ws_bytes < select_ws(B, H, N)) return PISA_ERR_WORKSPACE;
+  return launch_select(qbar, kbar, cov, cov_weight, scale, B * H, N, d, k_sel,
+                       sink_block(sink_idx, N), idx, (float *)workspace, (cudaStream_t)stream);
+}
+
+pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, pisa_dtype dtype,
+                                  const float *kbar, const float *vsum, const float *hbar,
+                                  const int32_t *idx, int k_sel, int B, int H, int L, int d,
+                                  int block_size, float scale, pisa_mode mode, void *out,
+                                  void *workspace, size_t ws_bytes, pisa_stream_t stream) {
+  PISA_TRY(check_shape(B, H, L, d, block_size));
+  if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
+  if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH) return PISA_ERR_INVALID_ARG;
+  const int N = ceil_div(L, 64);
+  if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kbar) ||
+      !aligned16(vsum) || !aligned16(hbar) || !idx || !aligned16(workspace))
+    return PISA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return PISA_ERR_INVALID_ARG;
+  if (ws_bytes < sparse_ws(B, H, L, d, dtype)) return PISA_ERR_WORKSPACE;
+  const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
+  return run_sparse_attention(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B * H, L, d, s, mode,
+                              out, (unsigned char *)workspace, (cudaStream_t)stream);
+}
+
+pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void *out, int B,
+                              int H, int L, int d, int block_size, double density, int sink_idx,
+                              pisa_mode mode, const pisa_options *opts, pisa_stream_t stream) {
+  pisa_options o;
+  memset(&o, 0, sizeof(o));
+  if (opts) o = *opts;
+  PISA_TRY(check_shape(B, H, L, d, block_size));
+  if (o.dtype != PISA_BF16 && o.dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
+  if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH) return PISA_ERR_INVALID_ARG;
+  if (!sink_valid(sink_idx)) return PISA_ERR_INVALID_ARG;
+  if (!(o.scale >= 0.f) || !std::isfinite(o.scale) || !std::isfinite(o.cov_weight))
+    return PISA_ERR_INVALID_ARG;
+  const int N = ceil_div(L, 64);
+  const int k_sel = pisa_num_selected(N, density);
+  if (k_sel < 1) return PISA_ERR_INVALID_ARG;
+  if ((long long)N * 4 > 200 * 1024) return PISA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return PISA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return PISA_ERR_INVALID_ARG;
+  const int want_cov = o.cov_weight != 0.f;
+  const PathLayout p = path_layout(B, H, L, d, density, o.dtype, want_cov);
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned char *ws = (unsigned char *)o.workspace;
+  bool owned = false;
+  if (ws) {
+    if (!aligned16(ws)) return PISA_ERR_INVALID_ARG;
+    if (o.ws_bytes < p.total) return PISA_ERR_WORKSPACE;
+  } else {
+    void *mem = nullptr;
+    PISA_CUDA(cudaMallocAsync(&mem, p.total, st));
+    ws = (unsigned char *)mem;
+    owned = true;
+  }
+  const float s = o.scale == 0.f ? 1.f / std::sqrt((float)d) : o.scale;
+  const int BH = B * H;
+  float *qbar = (float *)(ws + p.qbar), *kbar = (float *)(ws + p.kbar),
+        *vsum = (float *)(ws + p.vsum), *hbar = (float *)(ws + p.hbar),
+        *cov = want_cov ? (float *)(ws + p.cov) : nullptr;
+  int32_t *idx = (int32_t *)(ws + p.idx);
+  unsigned char *scratch = ws + p.scratch;
+  pisa_status r;
+  if (d == 128)
+    r = launch_stats<128>(q, k, v, o.dtype, BH, L, want_cov, qbar, kbar, vsum, hbar, cov,
+                          (float *)scratch, st);
+  else
+    r = launch_stats<64>(q, k, v, o.dtype, BH, L, want_cov, qbar, kbar, vsum, hbar, cov,
+                         (float *)scratch, st);
+  if (r == PISA_OK)
+    r = launch_select(qbar, kbar, cov, o.cov_weight, s, BH, N, d, k_sel,
+                      sink_block(sink_idx, N), idx, (float *)scratch, st);
+  if (r == PISA_OK)
+    r = run_sparse_attention(q, k, v, o.dtype, kbar, vsum, hbar, idx, k_sel, BH, L, d, s, mode,
+                             out, scratch, st);
+  if (owned) {
+    cudaError_t e = cudaFreeAsync(ws, st);
+    if (e != cudaSuccess && r == PISA_OK) {
+      set_last_error(e);
+      r = PISA_ERR_CUDA;
+    }
+  }
+  return r;
+}
+
+pisa_status pisa_attention(const void *q, const void *k, const void *v, void *out, int B, int H,
+                           int L, int d, int block_size, double density, int sink_idx,
+                           pisa_mode mode, pisa_stream_t stream) {
+  return pisa_attention_ex(q, k, v, out, B, H, L, d, block_size, density, sink_idx, mode, nullptr,
+                           stream);
+}
+
+size_t pisa_dense_attention_workspace_bytes(int B, int H, int L, int d, pisa_dtype dtype) {
+  if (check_shape(B, H, L, d, 64) != PISA_OK) return 0;
+  return dtype == PISA_F32 ? 3 * align_up((size_t)B * H * L * d * 2, 256) : 0;
+}
+
+pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, void *out,
+                                 pisa_dtype dtype, int B, int H, int L, int d, float scale,
+                                 void *workspace, size_t ws_bytes, pisa_stream_t stream) {
+  PISA_TRY(check_shape(B, H, L, d, 64));
+  if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return PISA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return PISA_ERR_INVALID_ARG;
+  const size_t need = pisa_dense_attention_workspace_bytes(B, H, L, d, dtype);
+  if (ws_bytes < need) return PISA_ERR_WORKSPACE;
+  if (need && !aligned16(workspace)) return PISA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int BH = B * H;
+  const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
+  const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
+                      *v16 = (const __nv_bfloat16 *)v;
+  if (dtype == PISA_F32) {
+    const size_t n = (size_t)BH * L * d, sz = align_up(n * 2, 256);
+    unsigned char *w = (unsigned char *)workspace;
+    PISA_TRY(to_bf16(q, (__nv_bfloat16 *)w, n, st));
+    PISA_TRY(to_bf16(k, (__nv_bfloat16 *)(w + sz), n, st));
+    PISA_TRY(to_bf16(v, (__nv_bfloat16 *)(w + 2 * sz), n, st));
+    q16 = (const __nv_bfloat16 *)w;
+    k16 = (const __nv_bfloat16 *)(w + sz);
+    v16 = (const __nv_bfloat16 *)(w + 2 * sz);
+  }
+  const int of32 = dtype == PISA_F32;
+  if (d == 128)
+    return launch_attention_kernel<128, true>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr,
+                                              0, BH, L, s, 0, out, of32, st);
+  return launch_attention_kernel<64, true>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, 0,
+                                           BH, L, s, 0, out, of32, st);
+}
+
+pisa_status pisa_device_status(pisa_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    set_last_error(e);
+    return PISA_ERR_CUDA;
+  }
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
+  if (e != cudaSuccess) {
+    set_last_error(e);
+    return PISA_ERR_CUDA;
+  }
+  if (v) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) {
+      set_last_error(e);
+      return PISA_ERR_CUDA;
+    }
+  }
+  if (v & kDevErrTimeout) return PISA_ERR_TIMEOUT;
+  if (v & kDevErrRange) return PISA_ERR_DEVICE;
+  return PISA_OK;
+}
+
+const char *pisa_status_string(pisa_status s) {
+  switch (s) {
+    case PISA_OK: return "ok";
+    case PISA_ERR_INVALID_ARG: return "invalid argument";
+    case PISA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PISA_ERR_CUDA: return "CUDA error";
+    case PISA_ERR_WORKSPACE: return "workspace too small";
+    case PISA_ERR_TIMEOUT: return "device-side bounded wait timed out";
+    case PISA_ERR_DEVICE: return "device-side range check failed";
+  }
+  return "unknown status";
+}
+
+const char *pisa_last_error(void) { return t_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+/*
+ * pisa.h -- C ABI of libpisa: PISA piecewise sparse attention (forward) on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("PISA: Piecewise Sparse Attention Is Wiser for Efficient
+ * Diffusion Transformers"; the gist.science "Technical Summary", section 2
+ * "Methodology"): every query block i attends exactly to its selected key/value
+ * blocks S_i, and every unselected block j in U_i enters the same softmax
+ * numerator N_t and denominator D_t through a block-wise zeroth-order Taylor
+ * term (block centroid kbar_j, value sum SigmaV_j) plus, in the paper ("hyd")
+ * variant, one shared global first-order correction Hbar, the mean of the
+ * block first-order matrices.  o_t = N_t / D_t.
+ *
+ * Conventions shared by every call:
+ *  - Tensors are dense row-major.  Q, K, V and the output are [B, H, L, d]
+ *    (token rows of d elements, heads and batches outermost).  Statistics are
+ *    float32: qbar/kbar/vsum [B, H, N, d], hbar [B, H, d, d], cov [B, H, N].
+ *    Selected block indices are int32 [B, H, N, k_sel], ascending per row.
+ *    N = ceil(L / block_size); only the last block may be partial.
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *    where stated.  The library keeps no pointer after a call returns.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and performs no host synchronisation, except
+ *    pisa_device_status.
+ *  - Arguments are validated on the host before anything is launched.  A
+ *    failed check returns PISA_ERR_INVALID_ARG or PISA_ERR_UNSUPPORTED and
+ *    launches nothing.  A failed launch returns PISA_ERR_CUDA.  Errors found
+ *    by the kernels themselves (an index out of range, a bounded wait that ran
+ *    out) are recorded in a device status word that pisa_device_status reads.
+ *  - Supported now: d in {64, 128}; block_size = 64; dtype bf16 or f32 (f32
+ *    inputs are rounded to bf16 for the tensor-core products; statistics are
+ *    accumulated in float32 from the inputs as given); all data pointers
+ *    16-byte aligned.
+ *  - There is no CPU fallback: every step runs in this library's CUDA kernels.
+ *
+ * Softmax scale: s multiplies every q.k product (exact logits, centroid
+ * logits, selection scores and the first-order term s q Hbar); 0 selects the
+ * default 1/sqrt(d).
+ */
+#ifndef PISA_H
+#define PISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pisa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  PISA_OK = 0,
+  PISA_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment or option */
+  PISA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d = 96) */
+  PISA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  PISA_ERR_WORKSPACE = 4,   /* caller workspace too small */
+  PISA_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (device word) */
+  PISA_ERR_DEVICE = 6       /* a kernel's range check failed (device word) */
+} pisa_status;
+
+typedef enum {
+  PISA_MODE_HYD = 0, /* zeroth-order tail + global first-order term ("_hyd") */
+  PISA_MODE_0TH = 1  /* zeroth-order tail only ("_0th") */
+} pisa_mode;
+
+typedef enum { PISA_BF16 = 0, PISA_F32 = 1 } pisa_dtype;
+
+/* sink_idx values: the authors' README, "Attention sink for MMDiT": 0 or -1
+ * force the first or the last K/V block into the exact set of every query
+ * block; PISA_SINK_NONE forces nothing. */
+#define PISA_SINK_NONE INT32_MIN
+
+/* Options of pisa_attention_ex.  Zero-initialise, then set what you need. */
+typedef struct {
+  float scale;        /* softmax scale s; 0 = 1/sqrt(d) */
+  float cov_weight;   /* lambda of covariance-aware scoring; 0 = off */
+  pisa_dtype dtype;   /* dtype of q, k, v and out */
+  void *workspace;    /* device scratch; NULL = allocate per call (stream-ordered) */
+  size_t ws_bytes;    /* size of `workspace` */
+} pisa_options;
+
+/* ---- sizes ------------------------------------------------------------- */
+
+/* N = ceil(L / block_size); -1 on invalid arguments. */
+int pisa_num_blocks(int L, int block_size);
+
+/* Exact blocks per query block: density is the fraction of K/V blocks kept
+ * exact (the authors' README `density`; 0.15 is "85% sparsity").
+ * k_sel = clamp(floor(density * N + 1e-6), 1, N), computed in double; the sink
+ * block counts inside k_sel.  -1 on invalid arguments. */
+int pisa_num_selected(int N, double density);
+
+/* Workspace bytes that pisa_attention_ex needs for these arguments (the sum
+ * of the three calls' needs below, plus bf16 copies for f32 inputs). */
+size_t pisa_workspace_bytes(int B, int H, int L, int d, int block_size,
+                            double density, pisa_dtype dtype, int want_cov);
+size_t pisa_block_stats_workspace_bytes(int B, int H, int L, int d, int block_size);
+size_t pisa_select_workspace_bytes(int B, int H, int N);
+size_t pisa_sparse_attention_workspace_bytes(int B, int H, int L, int d, int block_size,
+                                             pisa_dtype dtype);
+
+/* ---- the three steps of the path -------------------------------------- */
+
+/* Block statistics (gist.science summary, "Hardware Implementation" step 1,
+ * "Core Algorithm", "Global First-Order Correction", "Covariance-Aware
+ * Routing"):
+ *   qbar_i = mean query of block i            [B,H,N,d]
+ *   kbar_j = mean key of block j (centroid)   [B,H,N,d]
+ *   vsum_j = sum of the values of block j     [B,H,N,d]
+ *   hbar   = (1/N) sum_j H_j, H_j = sum_n (k_{j,n} - kbar_j)^T v_{j,n}  [B,H,d,d]
+ *   cov_j  = || H_j - hbar ||_F               [B,H,N]   (only if want_cov;
+ *                                                         cov may be NULL otherwise)
+ * q, k, v: [B,H,L,d] in `dtype`.  All outputs float32.  `workspace` must
+ * hold pisa_block_stats_workspace_bytes(...) bytes (deterministic partial
+ * sums; no atomics, so results are bitwise reproducible). */
+pisa_status pisa_block_stats(const void *q, const void *k, const void *v, pisa_dtype dtype,
+                             int B, int H, int L, int d, int block_size, int want_cov,
+                             float *qbar, float *kbar, float *vsum, float *hbar, float *cov,
+                             void *workspace, size_t ws_bytes, pisa_stream_t stream);
+
+/* Covariance-aware top-k routing with sink forcing (gist.science summary,
+ * "Covariance-Aware Routing"; authors' README "Attention sink for MMDiT"):
+ *   score_ij = scale * qbar_i . kbar_j + cov_weight * cov_j   (float32)
+ * keeps, per query block i, the k_sel = pisa_num_selected(N, density) highest
+ * scores, ties going to the lower block index; with sink_idx 0 / -1 the block
+ * 0 / N-1 is always kept and the other k_sel-1 are the best of the rest.
+ * idx [B,H,N,k_sel] int32, each row ascending.  cov may be NULL when
+ * cov_weight == 0.  `workspace`: pisa_select_workspace_bytes(B,H,N) bytes. */
+pisa_status pisa_select(const float *qbar, const float *kbar, const float *cov,
+                        float cov_weight, float scale, int B, int H, int N, int d,
+                        double density, int sink_idx, int32_t *idx,
+                        void *workspace, size_t ws_bytes, pisa_stream_t stream);
+
+/* Fused exact-or-approximate attention (gist.science summary, "Core
+ * Algorithm" numerator equation and "Hardware Implementation" phases 1-3): for
+ * token t of query block i,
+ *   D_t = sum_{j in S_i} sum_n e^{s q_t k_{j,n}} + sum_{j in U_i} n_j alpha_tj
+ *   N_t = sum_{j in S_i} sum_n e^{s q_t k_{j,n}} v_{j,n} + sum_{j in U_i} alpha_tj vsum_j
+ *         + [hyd] (s q_t hbar) sum_{j in U_i} alpha_tj,     alpha_tj = e^{s q_t kbar_j}
+ *   out_t = N_t / D_t
+ * with S_i = idx row i (k_sel ascending, distinct indices < N) and U_i its
+ * complement.  kbar, vsum, hbar as written by pisa_block_stats.  out
+ * [B,H,L,d] in `dtype`; it must not overlap any input.  `workspace`:
+ * pisa_sparse_attention_workspace_bytes(...) bytes. */
+pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v,
+                                  pisa_dtype dtype, const float *kbar, const float *vsum,
+                                  const float *hbar, const int32_t *idx, int k_sel,
+                                  int B, int H, int L, int d, int block_size, float scale,
+                                  pisa_mode mode, void *out, void *workspace,
+                                  size_t ws_bytes, pisa_stream_t stream);
+
+/* ---- the whole path ----------------------------------------------------- */
+
+/* The authors' `piecewise_sparse_attention_{hyd,0th}(q, k, v, density,
+ * block_size, sink_idx)`: statistics -> selection -> fused attention, bf16
+ * I/O, scale 1/sqrt(d), covariance weight 0.  Scratch memory is allocated and
+ * freed stream-ordered (cudaMallocAsync / cudaFreeAsync) on `stream`. */
+pisa_status pisa_attention(const void *q, const void *k, const void *v, void *out,
+                           int B, int H, int L, int d, int block_size, double density,
+                           int sink_idx, pisa_mode mode, pisa_stream_t stream);
+
+/* pisa_attention with options (scale, covariance weight, f32 I/O, caller
+ * workspace).  With opts->workspace non-NULL nothing is allocated; it must
+ * hold pisa_workspace_bytes(...) bytes, else PISA_ERR_WORKSPACE.  opts may be
+ * NULL (defaults). */
+pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void *out,
+                              int B, int H, int L, int d, int block_size, double density,
+                              int sink_idx, pisa_mode mode, const pisa_options *opts,
+                              pisa_stream_t stream);
+
+/* Dense softmax attention out = softmax(s q k^T) v over all L keys, same
+ * layout and dtypes: the dense baseline timed beside the sparse path. */
+pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, void *out,
+                                 pisa_dtype dtype, int B, int H, int L, int d, float scale,
+                                 void *workspace, size_t ws_bytes, pisa_stream_t stream);
+size_t pisa_dense_attention_workspace_bytes(int B, int H, int L, int d, pisa_dtype dtype);
+
+/* ---- errors -------------------------------------------------------------- */
+
+/* Synchronises `stream`, then reads and clears the device status word set by
+ * the kernels.  Returns PISA_OK, PISA_ERR_TIMEOUT, PISA_ERR_DEVICE, or
+ * PISA_ERR_CUDA if the stream itself reported an error. */
+pisa_status pisa_device_status(pisa_stream_t stream);
+
+/* Static description of a status code. */
+const char *pisa_status_string(pisa_status s);
+
+/* Text of the last CUDA error seen by this library on the calling thread
+ * ("" if none). */
+const char *pisa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PISA_H */

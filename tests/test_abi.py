@@ -1,0 +1,90 @@
+"""C-ABI library: loads, exports every declared symbol, host-side logic.
+
+No compute call is made here (these run without a GPU): only size helpers and
+argument checks that fail before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+from block_sparse_attention_stats_b200 import _lib as L
+from block_sparse_attention_stats_b200.build import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "pisa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return L.load()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pisa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in L.SIGNATURES, f"binding lacks a prototype for {n}"
+
+
+def test_num_blocks_and_selected_match_oracle(lib):
+    for L_, b in ((1, 64), (64, 64), (65, 64), (75600, 64), (119056, 64)):
+        assert lib.pisa_num_blocks(L_, b) == O.block_partition(L_, b)[0]
+    for N in (1, 2, 7, 16, 72, 1182, 1861):
+        for dens in (0.01, 0.05, 0.1, 0.125, 0.15, 0.25, 0.5, 1.0):
+            assert lib.pisa_num_selected(N, dens) == O.num_selected(N, dens)
+    assert lib.pisa_num_selected(10, 0.0) == -1
+    assert lib.pisa_num_selected(10, 1.01) == -1
+    assert lib.pisa_num_blocks(0, 64) == -1
+
+
+def test_workspace_sizes(lib):
+    w = lib.pisa_workspace_bytes(1, 40, 75600, 128, 64, 0.125, L.PISA_BF16, 0)
+    assert w > 0 and w % 256 == 0
+    # covariance and f32 inputs need more scratch
+    assert lib.pisa_workspace_bytes(1, 24, 4608, 128, 64, 0.15, L.PISA_BF16, 1) > \
+        lib.pisa_workspace_bytes(1, 24, 4608, 128, 64, 0.15, L.PISA_BF16, 0)
+    assert lib.pisa_workspace_bytes(1, 2, 1024, 64, 64, 0.25, L.PISA_F32, 0) > \
+        lib.pisa_workspace_bytes(1, 2, 1024, 64, 64, 0.25, L.PISA_BF16, 0)
+    # unsupported shapes report 0
+    assert lib.pisa_workspace_bytes(1, 1, 1024, 96, 64, 0.25, L.PISA_BF16, 0) == 0
+    assert lib.pisa_workspace_bytes(1, 1, 1024, 128, 32, 0.25, L.PISA_BF16, 0) == 0
+
+
+def _attn(lib, q=0x1000, k=0x2000, v=0x3000, out=0x4000, B=1, H=1, Ln=128, d=128, bs=64,
+          dens=0.5, sink=L.PISA_SINK_NONE, mode=L.PISA_MODE_HYD, opts=None):
+    return lib.pisa_attention_ex(q, k, v, out, B, H, Ln, d, bs, dens, sink, mode,
+                                 ctypes.byref(opts) if opts else None, None)
+
+
+def test_argument_checks_fail_before_any_launch(lib):
+    assert _attn(lib, q=None) == L.PISA_ERR_INVALID_ARG
+    assert _attn(lib, q=0x1001) == L.PISA_ERR_INVALID_ARG          # misaligned
+    assert _attn(lib, out=0x1000) == L.PISA_ERR_INVALID_ARG        # out aliases q
+    assert _attn(lib, d=96) == L.PISA_ERR_UNSUPPORTED
+    assert _attn(lib, bs=128) == L.PISA_ERR_UNSUPPORTED
+    assert _attn(lib, Ln=0) == L.PISA_ERR_INVALID_ARG
+    assert _attn(lib, dens=0.0) == L.PISA_ERR_INVALID_ARG
+    assert _attn(lib, dens=1.5) == L.PISA_ERR_INVALID_ARG
+    assert _attn(lib, sink=3) == L.PISA_ERR_INVALID_ARG
+    assert _attn(lib, mode=7) == L.PISA_ERR_INVALID_ARG
+    o = L.PisaOptions()
+    o.workspace = 0x10000
+    o.ws_bytes = 16
+    assert _attn(lib, opts=o) == L.PISA_ERR_WORKSPACE
+    o = L.PisaOptions()
+    o.scale = float("nan")
+    assert _attn(lib, opts=o) == L.PISA_ERR_INVALID_ARG
+    assert lib.pisa_select(None, None, None, 0.0, 0.1, 1, 1, 4, 64, 0.5, 0, None, None, 0,
+                           None) == L.PISA_ERR_INVALID_ARG
+    assert lib.pisa_status_string(L.PISA_ERR_TIMEOUT).decode().startswith("device-side")
