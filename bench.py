@@ -47,7 +47,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of the fused attention kernel, from an ncu capture,
 # keyed by the sha1 of the kernel source it was taken on (see profiles/).
-K3_TRAFFIC = {}
+K3_TRAFFIC = {
+    # warp-MMA kernel, Wan-like H=4 capture (302.8 MB) scaled by heads to H=40
+    "0c3ca42da25c": {"wan": 3.028e9},
+}
 
 
 def _peaks():
@@ -433,7 +436,7 @@ def run_pisa(args, wl):
     p_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     achieved = f_alg / (t_k3 * 1e-3) / 1e12
     src = _k3_source_hash()
-    traffic = K3_TRAFFIC.get(src)
+    traffic = K3_TRAFFIC.get(src, {}).get(wl.name)
     launches_per_step = 2 + (1 if want_cov else 0) + 2 + 2 + (3 if wl.dtype == "f32" else 0)
     line = {
         "metric": METRIC,
@@ -494,8 +497,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (small cases for profiling only)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
+    if args.heads:
+        wl = wl.with_(H=args.heads, name=f"{wl.name}-h{args.heads}")
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_pisa(args, wl)
