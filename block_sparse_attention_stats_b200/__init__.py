@@ -8,6 +8,7 @@ from .api import (  # noqa: F401
     pisa_attention,
     pisa_attention_ex,
     pisa_block_stats,
+    pisa_block_stats_noalloc,
     pisa_dense_attention,
     pisa_device_status,
     pisa_num_blocks,

@@ -110,6 +110,28 @@ def pisa_block_stats(q, k, v, block_size: int = 64, want_cov: bool = False,
     return dict(qbar=qbar, kbar=kbar, vsum=vsum, hbar=hbar, cov=cov)
 
 
+def pisa_block_stats_noalloc(q, k, v, block_size: int = 64, want_cov: bool = False,
+                             out: Optional[dict] = None, stream=None):
+    """pisa_block_stats for callers that must not allocate device memory: the
+    library keeps the scratch partial sums in its own static device array
+    (shapes needing more than PISA_NOALLOC_SCRATCH_BYTES are refused).  Calls
+    on one device share that array, so order them on one stream."""
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    N = lib.pisa_num_blocks(Ln, block_size)
+    f = dict(dtype=torch.float32, device=q.device)
+    if out is not None:
+        qbar, kbar, vsum, hbar, cov = (out[n] for n in ("qbar", "kbar", "vsum", "hbar", "cov"))
+    else:
+        qbar, kbar, vsum = (torch.empty((B, H, N, d), **f) for _ in range(3))
+        hbar = torch.empty((B, H, d, d), **f)
+        cov = torch.empty((B, H, N), **f) if want_cov else None
+    _check("pisa_block_stats_noalloc", lib.pisa_block_stats_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], B, H, Ln, d, block_size, int(want_cov),
+        _ptr(qbar), _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(cov), _stream(stream)))
+    return dict(qbar=qbar, kbar=kbar, vsum=vsum, hbar=hbar, cov=cov)
+
+
 def pisa_select(qbar, kbar, density: float, sink_idx: Optional[int] = None,
                 cov: Optional[torch.Tensor] = None, cov_weight: float = 0.0,
                 scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,

@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <cmath>
+#include <mutex>
 #include <string>
 
 #include "pisa.h"
@@ -241,6 +242,45 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
 
 using namespace pisa;
 
+// ---------------------------------------------------------------------------
+// pisa_block_stats_noalloc: scratch in a static device array
+// ---------------------------------------------------------------------------
+// Chunk partial sums of the statistics pass live here instead of in a caller
+// workspace.  The host-side symbol is only a stand-in: kernels must be given
+// the device address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PISA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the first call on a device does the lookup).
+pisa_status noalloc_scratch(void **out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_last_error(e);
+    return PISA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return PISA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      set_last_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      return PISA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return PISA_OK;
+}
+}  // namespace
+
+
 // =============================================================================
 // C ABI
 // =============================================================================
@@ -449,6 +489,35 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
                                               0, BH, L, s, 0, out, of32, st);
   return launch_attention_kernel<64, true>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, 0,
                                            BH, L, s, 0, out, of32, st);
+}
+
+pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v,
+                                     pisa_dtype dtype, int B, int H, int L, int d,
+                                     int block_size, int want_cov, float *qbar, float *kbar,
+                                     float *vsum, float *hbar, float *cov,
+                                     pisa_stream_t stream) {
+  PISA_TRY(check_shape(B, H, L, d, block_size));
+  if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qbar) || !aligned16(kbar) ||
+      !aligned16(vsum) || !aligned16(hbar))
+    return PISA_ERR_INVALID_ARG;
+  if (want_cov && !aligned16(cov)) return PISA_ERR_INVALID_ARG;
+  const size_t need = stats_ws(B, H, L, d);
+  if (need > (size_t)PISA_NOALLOC_SCRATCH_BYTES) {
+    t_last_error = "pisa_block_stats_noalloc: this shape needs " + std::to_string(need) +
+                   " bytes of scratch; the static array holds " +
+                   std::to_string((size_t)PISA_NOALLOC_SCRATCH_BYTES);
+    return PISA_ERR_WORKSPACE;
+  }
+  void *scratch = nullptr;
+  PISA_TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = (cudaStream_t)stream;
+  float *partial = (float *)scratch;
+  if (d == 128)
+    return launch_stats<128>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
+                             partial, st);
+  return launch_stats<64>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
+                          partial, st);
 }
 
 pisa_status pisa_device_status(pisa_stream_t stream) {

@@ -176,6 +176,44 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
                                  void *workspace, size_t ws_bytes, pisa_stream_t stream);
 size_t pisa_dense_attention_workspace_bytes(int B, int H, int L, int d, pisa_dtype dtype);
 
+/* ---- block statistics without any allocation ----------------------------- */
+
+/* Largest scratch, in bytes, that pisa_block_stats_noalloc can use. */
+#define PISA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* pisa_block_stats for callers that cannot allocate device memory.  The
+ * paper has no counterpart: this is a packaging variant, not part of the
+ * method.  Some hosts give a library only the buffers of one call and forbid
+ * cudaMalloc (plugin interfaces of inference runtimes, frameworks whose own
+ * allocator has reserved the device), and some loops cannot afford the device
+ * synchronisation that cudaMalloc / cudaFree may cause.  Such callers cannot
+ * provide the workspace that pisa_block_stats needs.
+ *
+ * This call computes exactly what pisa_block_stats computes (same kernels,
+ * same reduction order, bitwise the same results), with the same argument
+ * meaning, layout and ownership, but keeps its chunk partial sums in one
+ * static device array of PISA_NOALLOC_SCRATCH_BYTES bytes inside libpisa.
+ * Every GPU that loads the library holds that array until the process exits.
+ *  - It allocates nothing and calls no allocating routine.
+ *  - Shapes whose scratch need, pisa_block_stats_workspace_bytes(B, H, L, d,
+ *    block_size), exceeds PISA_NOALLOC_SCRATCH_BYTES are rejected with
+ *    PISA_ERR_WORKSPACE before anything is launched (pisa_last_error gives the
+ *    sizes).  Example: the Wan2.1-like shape (B=1, H=40, L=75600, d=128)
+ *    needs 20 MiB.
+ *  - The first call on each device looks up that device's address of the
+ *    array (cudaGetSymbolAddress) with the device current; make that first
+ *    call before any stream capture begins on the device.
+ *  - All calls on a device share the one array, which keeps whatever the last
+ *    call left there.  Nothing in it needs to start at zero: each call writes
+ *    every partial it later reads.  Calls whose kernels may overlap on the GPU
+ *    (different streams without ordering, or several host threads) race on
+ *    the array and give wrong results; order them on one stream. */
+pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v,
+                                     pisa_dtype dtype, int B, int H, int L, int d,
+                                     int block_size, int want_cov, float *qbar, float *kbar,
+                                     float *vsum, float *hbar, float *cov,
+                                     pisa_stream_t stream);
+
 /* ---- errors -------------------------------------------------------------- */
 
 /* Synchronises `stream`, then reads and clears the device status word set by
