@@ -64,7 +64,7 @@ def _peaks():
 
 def _k3_source_hash():
     h = hashlib.sha1()
-    for n in ("k3_attention_mma.cuh",):
+    for n in ("k3_attention_tc.cuh", "k3_pack.cuh", "sm100_primitives.cuh"):
         fn = os.path.join(ROOT, "block_sparse_attention_stats_b200", "csrc", n)
         if os.path.exists(fn):
             h.update(open(fn, "rb").read())
@@ -95,13 +95,60 @@ def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
     return exact + tail + first
 
 
-def k3_executed_flops(wl, k_sel: int, chunks_per_block: float) -> float:
-    """MMA flops the warp-MMA kernel issues: 64-row query tiles x 64-key tiles."""
+PAIR_WINDOW = 16
+
+
+def _pairs_like_kernel(bits: np.ndarray):
+    """The fused kernel's query-block pairing (greedy, largest overlap of exact
+    sets within the next 16 blocks, nearer on ties), replayed on the host only to
+    count the tensor-core tiles it issues."""
+    N = bits.shape[0]
+    used = np.zeros(N, dtype=bool)
+    pairs = []
+    for i in range(N):
+        if used[i]:
+            continue
+        used[i] = True
+        best, bo = -1, -1
+        for j in range(i + 1, min(N, i + 1 + PAIR_WINDOW)):
+            if not used[j]:
+                o = int((bits[i] & bits[j]).sum())
+                if o > bo:
+                    bo, best = o, j
+        if best < 0:
+            rest = np.nonzero(~used[i + 1:])[0]
+            best = i + 1 + int(rest[0]) if rest.size else -1
+        if best >= 0:
+            used[best] = True
+        pairs.append((i, best))
+    return pairs
+
+
+def k3_executed_flops(wl, idx: torch.Tensor, heads: int = 2) -> float:
+    """MMA flops of the fused kernel: 128-row tiles x 64-key tiles over the union
+    of each pair's exact sets plus the centroid chunks, and Q Hbar; counted on
+    `heads` heads and scaled to all heads."""
     b, d = wl.block_size, wl.d
     N = -(-wl.L // b)
-    tiles = N * (k_sel + chunks_per_block) * wl.B * wl.H
-    first = (2.0 * N * 64 * d * d * wl.B * wl.H) if wl.mode == "hyd" else 0.0
-    return tiles * 4.0 * d * 64 * 64 + first
+    nch = -(-N // 64)
+    tile = 4.0 * d * 128 * 64
+    tot = 0.0
+    idx_np = idx.reshape(-1, N, idx.shape[-1]).cpu().numpy()
+    use = min(heads, idx_np.shape[0])
+    for h in range(use):
+        bits = np.zeros((N, N), dtype=bool)
+        np.put_along_axis(bits, idx_np[h].astype(np.int64), True, axis=1)
+        for (i, j) in _pairs_like_kernel(bits):
+            sel = bits[i] | (bits[j] if j >= 0 else False)
+            chunks = 0
+            for c in range(nch):
+                lo, hi = c * 64, min(N, c * 64 + 64)
+                need = (~bits[i, lo:hi]).any() or (j >= 0 and (~bits[j, lo:hi]).any())
+                chunks += int(need)
+            tot += (int(sel.sum()) + chunks) * tile
+            if wl.mode == "hyd":
+                tot += 2.0 * 128 * d * d
+    return tot * (wl.B * wl.H) / use
 
 
 def stats_bytes(wl):
@@ -429,8 +476,7 @@ def run_pisa(args, wl):
     N = -(-wl.L // wl.block_size)
     k_sel = idx.shape[-1]
     f_alg = k3_algorithmic_flops(wl, idx)
-    n_chunks = -(-N // 64)
-    f_exec = k3_executed_flops(wl, k_sel, n_chunks)
+    f_exec = k3_executed_flops(wl, idx)
     peaks, peak_kind = _peaks()
     p_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     p_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])

@@ -1,0 +1,505 @@
+// K3 (tcgen05 version): fused exact-or-approximate attention on sm_100a.
+//
+// "Technical Summary: PISA" (gist.science), section 2: "Core Algorithm" (the
+// numerator N_t equation, alpha_{t,j} = exp(q_t kbar_j^T), o_t = N_t / D_t),
+// "Key Insights" 2 (both approximations enter the same softmax numerator and
+// denominator) and "Hardware Implementation" (one fused kernel running the
+// exact phase over selected blocks, the zeroth-order scan over aggregated
+// block vectors of unselected blocks and the global first-order correction
+// inside one online softmax).
+//
+// Work unit: one CTA = two adjacent query blocks (2p, 2p+1) of one head, i.e.
+// 128 query rows, so every tensor-core product is an M = 128 tcgen05 MMA.
+// The exact tiles are the union S_2p u S_2p+1 (ascending); each carries two
+// flags saying which half selected it.  A half that did not select a tile
+// gives it zero probability (and spends no exp on it); that block then reaches
+// that half through its centroid, as in the method.  After the exact tiles
+// come the centroid chunks: 64 consecutive block centroids kbar_j as keys and
+// value sums vsum_j as values, masked per half to that half's unselected
+// blocks U_i, with weight n_j in the denominator; their probabilities are also
+// summed into a_t = sum_{U_i} alpha_tj.  In the paper ("hyd") mode a last MMA
+// forms Q Hbar and the epilogue adds s a_t (q_t Hbar) to the numerator.
+//
+// Roles (192 threads):
+//   warp 0      TMA producer: Q once, then the K/V (or kbar/vsum) tile of every
+//               list entry into a 2-stage ring, then Hbar;
+//   warp 1      TMEM allocation; one thread issues every tcgen05.mma:
+//               S_b = Q K^T (two S buffers), O += P V with P read from TMEM,
+//               and Q Hbar at the end;
+//   warps 2-5   softmax: one thread per query row (= TMEM lane); reads S, keeps
+//               the running max m (log2 domain), denominator l and tail weight
+//               a in registers, writes P (bf16) into the S columns, rescales
+//               the O row in TMEM only when the max grows by more than 2^8,
+//               and runs the epilogue o = (O + s a QHbar) / l.
+// TMEM columns: O [0, D), S buffers [D, D+64) and [D+64, D+128); Q Hbar
+// reuses [D, 2D) after the last P V.
+// Every mbarrier wait is bounded (sm100::mbar_wait); on a timeout the CTA
+// records the error, stops issuing work, waits for its own copies and MMAs,
+// frees TMEM and exits.
+#pragma once
+
+#include "pisa_common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace pisa {
+
+template <int D> struct TcCfg {
+  static constexpr int kThreads = 192;
+  static constexpr int kRows = 128;
+  static constexpr int kKeys = 64;
+  static constexpr int kStages = 2;
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kBoxQBytes = kRows * 128;   // one 64-column box of Q
+  static constexpr int kBoxKBytes = kKeys * 128;   // one 64-column box of a K/V tile
+  static constexpr int kTileBytes = kKeys * D * 2;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kHbarBytes = D * D * 2;
+  static_assert(kHbarBytes <= kStageBytes, "Hbar must fit in one stage");
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffStage = kQBytes;
+  static constexpr int kOffBar = kOffStage + kStages * kStageBytes;
+  static constexpr int kNumBars = 16;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kOffMisc = kOffTmemSlot + 16;
+  static constexpr int kOffDyn = kOffMisc + 16;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kColO = 0;
+  static constexpr uint32_t kColS = D;
+  static constexpr uint32_t kColQH = D;
+  // barrier indices
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKvFull = 1;                  // + stage
+  static constexpr int kBarKvEmpty = 1 + kStages;       // + stage
+  static constexpr int kBarSFull = 1 + 2 * kStages;     // + buffer
+  static constexpr int kBarPFull = 3 + 2 * kStages;     // + buffer
+  static constexpr int kBarODone = 5 + 2 * kStages;
+  static constexpr int kBarFinal = 6 + 2 * kStages;     // after the last MMA
+  static constexpr int kBarTeardown = 7 + 2 * kStages;
+  static_assert(kBarTeardown < kNumBars, "barrier slots");
+
+  __host__ __device__ static int smem_bytes(int N) {
+    const int nwords = (N + 31) / 32;
+    return kOffDyn + (2 * nwords + N + (N + 63) / 64) * 4 + 1024;  // + alignment slack
+  }
+};
+
+__device__ __forceinline__ uint32_t valid_bits(int w, int N) {
+  const int lo = w * 32;
+  if (lo + 32 <= N) return 0xffffffffu;
+  if (lo >= N) return 0u;
+  return (1u << (N - lo)) - 1u;
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 2)
+    piecewise_attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                  const __grid_constant__ CUtensorMap tm_k,
+                                  const __grid_constant__ CUtensorMap tm_v,
+                                  const __grid_constant__ CUtensorMap tm_kbar,
+                                  const __grid_constant__ CUtensorMap tm_vsum,
+                                  const __grid_constant__ CUtensorMap tm_hbar,
+                                  const int32_t *__restrict__ idx,
+                                  const int2 *__restrict__ pairs, int k_sel, int L, int N,
+                                  float scale, int hyd, int dense, void *__restrict__ out,
+                                  int out_f32) {
+  using C = TcCfg<D>;
+  using namespace sm100;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  unsigned char *smem = smem_raw + (sbase - raw);
+  auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
+  volatile int *misc = reinterpret_cast<volatile int *>(smem + C::kOffMisc);  // [0] tiles, [1] abort
+  const int nwords = (N + 31) / 32;
+  uint32_t *bm_lo = reinterpret_cast<uint32_t *>(smem + C::kOffDyn);
+  uint32_t *bm_hi = bm_lo + nwords;
+  int *tiles = reinterpret_cast<int *>(bm_hi + nwords);
+
+  const int pair = blockIdx.x, bh = blockIdx.y;
+  // query blocks of the two halves (rows 0-63 and 64-127 of the tile)
+  int qb0 = 2 * pair, qb1 = 2 * pair + 1 < N ? 2 * pair + 1 : -1;
+  if (pairs) {
+    const int2 pr = pairs[(size_t)bh * ((N + 1) / 2) + pair];
+    qb0 = pr.x;
+    qb1 = pr.y;
+  }
+  const bool has_hi = qb1 >= 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- set-up ---------------------------------------------------------------
+  if (warp == 1) {
+    tmem_alloc(sbase + C::kOffTmemSlot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar(C::kBarQ), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(C::kBarKvFull + s), 1);
+      mbar_init(bar(C::kBarKvEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::kBarSFull + b), 1);
+      mbar_init(bar(C::kBarPFull + b), 128);
+    }
+    mbar_init(bar(C::kBarODone), 1);
+    mbar_init(bar(C::kBarFinal), 1);
+    mbar_init(bar(C::kBarTeardown), 1);
+    fence_mbar_init();
+    misc[1] = 0;
+  }
+  if (tid == 32) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_kbar);
+    prefetch_tmap(&tm_vsum);
+    prefetch_tmap(&tm_hbar);
+  }
+  for (int w = tid; w < 2 * nwords; w += C::kThreads) bm_lo[w] = 0u;
+  __syncthreads();
+  if (dense) {
+    for (int w = tid; w < nwords; w += C::kThreads) {
+      bm_lo[w] = valid_bits(w, N);
+      bm_hi[w] = has_hi ? valid_bits(w, N) : 0u;
+    }
+  } else {
+    const int32_t *r0 = idx + ((size_t)bh * N + qb0) * k_sel;
+    const int32_t *r1 = idx + ((size_t)bh * N + (has_hi ? qb1 : qb0)) * k_sel;
+    for (int t = tid; t < (has_hi ? 2 : 1) * k_sel; t += C::kThreads) {
+      const int j = t < k_sel ? r0[t] : r1[t - k_sel];
+      uint32_t *bm = t < k_sel ? bm_lo : bm_hi;
+      if (j >= 0 && j < N) atomicOr(&bm[j >> 5], 1u << (j & 31));
+      else report_device_error(kDevErrRange);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exact tiles: ascending union of both halves' sets, with per-half flags
+    int base = 0;
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t lo = w < nwords ? bm_lo[w] : 0u, hi = w < nwords ? bm_hi[w] : 0u;
+      uint32_t u = lo | hi;
+      const int cnt = __popc(u);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int pos = base + incl - cnt;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1u;
+        tiles[pos++] = ((w * 32 + bit) << 2) | ((lo >> bit) & 1u) | (((hi >> bit) & 1u) << 1);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    // centroid chunks that hold an unselected block for either half
+    if (!dense) {
+      const int nch = (N + 63) / 64;
+      for (int c0 = 0; c0 < nch; c0 += 32) {
+        const int c = c0 + lane;
+        bool need = false;
+        if (c < nch) {
+          for (int h = 0; h < (has_hi ? 2 : 1); ++h) {
+            const uint32_t *bm = h ? bm_hi : bm_lo;
+            const uint32_t m0 = ~bm[2 * c] & valid_bits(2 * c, N);
+            const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & valid_bits(2 * c + 1, N)) : 0u;
+            need = need || ((m0 | m1) != 0u);
+          }
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, need);
+        if (need) tiles[base + __popc(bal & ((1u << lane) - 1u))] = -(c + 1);
+        base += __popc(bal);
+      }
+    }
+    if (lane == 0) misc[0] = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + C::kOffTmemSlot);
+  const int T = misc[0];
+
+  if (warp == 0) {
+    // ======================= TMA producer =====================================
+    if (lane == 0) {
+      const int total = T + (hyd ? 1 : 0);
+      int issued = 0;
+      // Q rows of both query blocks (an absent upper block reads as zeros)
+      mbar_expect_tx(bar(C::kBarQ), C::kQBytes);
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b) {
+        const uint32_t dst = sbase + C::kOffQ + b * C::kBoxQBytes;
+        tma_load_3d(dst, &tm_q, bar(C::kBarQ), 64 * b, qb0 * 64, bh);
+        tma_load_3d(dst + 64 * 128, &tm_q, bar(C::kBarQ), 64 * b, has_hi ? qb1 * 64 : L, bh);
+      }
+      for (int t = 0; t < total; ++t) {
+        if (misc[1]) break;
+        const int s = t % C::kStages;
+        if (t >= C::kStages && !mbar_wait(bar(C::kBarKvEmpty + s), ((t / C::kStages) - 1) & 1)) {
+          misc[1] = 1;
+          break;
+        }
+        const uint32_t st = sbase + C::kOffStage + s * C::kStageBytes;
+        const uint32_t full = bar(C::kBarKvFull + s);
+        if (t < T) {
+          const int e = tiles[t];
+          const CUtensorMap *mk = e >= 0 ? &tm_k : &tm_kbar;
+          const CUtensorMap *mv = e >= 0 ? &tm_v : &tm_vsum;
+          const int row = e >= 0 ? (e >> 2) * 64 : (-e - 1) * 64;
+          mbar_expect_tx(full, C::kStageBytes);
+#pragma unroll
+          for (int b = 0; b < D / 64; ++b) {
+            tma_load_3d(st + b * C::kBoxKBytes, mk, full, 64 * b, row, bh);
+            tma_load_3d(st + C::kTileBytes + b * C::kBoxKBytes, mv, full, 64 * b, row, bh);
+          }
+        } else {
+          mbar_expect_tx(full, C::kHbarBytes);
+#pragma unroll
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_3d(st + b * (D * 128), &tm_hbar, full, 64 * b, 0, bh);
+        }
+        issued = t + 1;
+      }
+      if (misc[1]) {
+        // let the copies already in flight land before the CTA exits
+        mbar_wait(bar(C::kBarQ), 0);
+        for (int t = issued - C::kStages; t < issued; ++t)
+          if (t >= 0) mbar_wait(bar(C::kBarKvFull + t % C::kStages), (t / C::kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================================
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+      bool ok = mbar_wait(bar(C::kBarQ), 0);
+      tc_fence_after();
+      auto q_desc = [&](int k) -> uint64_t {
+        return smem_desc_sw128(sbase + C::kOffQ + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
+      };
+      auto issue_pv = [&](int u) -> bool {
+        const int bu = u & 1, su = u % C::kStages;
+        if (!mbar_wait(bar(C::kBarPFull + bu), (u >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t vst = sbase + C::kOffStage + su * C::kStageBytes + C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + C::kColO, tmem + C::kColS + 64 * bu + kk * 8,
+                 smem_desc_sw128(vst + kk * 2048, C::kBoxKBytes, 1024), kIdPV,
+                 (u > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(C::kBarKvEmpty + su));
+        tc_commit(bar(C::kBarODone));
+        return true;
+      };
+      for (int t = 0; ok && t < T; ++t) {
+        if (misc[1]) { ok = false; break; }
+        const int s = t % C::kStages, b = t & 1;
+        if (!mbar_wait(bar(C::kBarKvFull + s), (t / C::kStages) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kst = sbase + C::kOffStage + s * C::kStageBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + C::kColS + 64 * b, q_desc(k),
+                 smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024), kIdQK,
+                 k > 0 ? 1u : 0u);
+        tc_commit(bar(C::kBarSFull + b));
+        if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+      }
+      if (ok && T >= 1) ok = issue_pv(T - 1);
+      if (ok && !hyd) tc_commit(bar(C::kBarFinal));
+      if (ok && hyd) {
+        const int s = T % C::kStages;
+        if (mbar_wait(bar(C::kBarKvFull + s), (T / C::kStages) & 1)) {
+          tc_fence_after();
+          const uint32_t hst = sbase + C::kOffStage + s * C::kStageBytes;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k)
+            mma_ss(tmem + C::kColQH, q_desc(k), smem_desc_sw128(hst + k * 2048, D * 128, 1024),
+                   kIdPV, k > 0 ? 1u : 0u);
+          tc_commit(bar(C::kBarFinal));
+        } else {
+          ok = false;
+        }
+      }
+      if (!ok) {
+        misc[1] = 1;
+        // every MMA issued so far must finish before TMEM is released
+        tc_commit(bar(C::kBarTeardown));
+        mbar_wait(bar(C::kBarTeardown), 0);
+      }
+    }
+  } else {
+    // ======================= softmax warps ====================================
+    const int sp = warp & 3;                 // TMEM sub-partition of this warp
+    const int row = sp * 32 + lane;          // query row in the tile = TMEM lane
+    const int half = row >> 6;               // warp-uniform
+    const bool exists = half == 0 || has_hi;
+    const uint32_t *bm = half ? bm_hi : bm_lo;
+    const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
+    const float sl2 = scale * kLog2e;
+    const int n_last = L - (N - 1) * 64;
+    float m_run = -INFINITY, l_run = 0.f, a_run = 0.f;
+    bool ok = true;
+    // waits and abort checks are made warp-uniform: TMEM access is warp-collective
+    auto warp_wait = [&](uint32_t b_addr, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(b_addr, parity));
+    };
+    for (int t = 0; t < T; ++t) {
+      if (__any_sync(0xffffffffu, misc[1] != 0)) { ok = false; break; }
+      const int b = t & 1;
+      if (!warp_wait(bar(C::kBarSFull + b), (t >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const int e = tiles[t];
+      const bool centroid = e < 0;
+      uint64_t cmask = 0;
+      bool active;
+      if (!exists) {
+        active = false;
+      } else if (!centroid) {
+        active = ((e >> half) & 1) != 0;
+      } else {
+        const int c = -e - 1;
+        const uint32_t m0 = ~bm[2 * c] & valid_bits(2 * c, N);
+        const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & valid_bits(2 * c + 1, N)) : 0u;
+        cmask = (uint64_t)m0 | ((uint64_t)m1 << 32);
+        active = cmask != 0;
+      }
+      float sv[64];
+      float tmax = -INFINITY;
+      const uint32_t s_addr = lane_addr + C::kColS + 64 * b;
+      uint32_t pk[32];
+      if (active) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_x32(s_addr, r0);
+        tmem_ld_x32(s_addr + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = __uint_as_float(r0[i]);
+          sv[i + 32] = __uint_as_float(r1[i]);
+        }
+        // columns that are not keys of this row: past the sequence end in the
+        // partial last block, or centroids of blocks this half selected
+        uint64_t keep = ~0ull;
+        if (centroid) keep = cmask;
+        else if ((e >> 2) == N - 1 && n_last < 64) keep = (1ull << n_last) - 1ull;
+        if (keep != ~0ull) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) sv[i] = ((keep >> i) & 1ull) ? sv[i] : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, sv[i]);
+        const float m_t = tmax * sl2;                  // finite: the row has a key here
+        const bool grow = m_t > m_run + 8.0f;          // lazy rescale threshold 2^8
+        const bool need_o = grow && m_run != -INFINITY;
+        const float f = grow ? ex2_approx(m_run - m_t) : 1.0f;  // 0 when m_run = -inf
+        if (__any_sync(0xffffffffu, need_o)) {
+          // O is stable once P V of the previous tile is done (P V of the tile
+          // before that finished before S of this tile, by commit order)
+          if (!warp_wait(bar(C::kBarODone), (t - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_x32(lane_addr + C::kColO + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st_x32(lane_addr + C::kColO + 32 * c, o);
+          }
+        }
+        if (grow) {
+          m_run = m_t;
+          l_run *= f;
+          a_run *= f;
+        }
+        const float neg = -m_run;
+        float ps = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2_approx(fmaf(sv[2 * i], sl2, neg));
+          const float p1 = ex2_approx(fmaf(sv[2 * i + 1], sl2, neg));
+          ps += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        if (centroid) {
+          // weight n_j = 64 except for the last block, which holds n_last tokens
+          float pl = 0.f;
+          if ((-e - 1) == (N - 1) / 64 && n_last < 64) {
+            const int col = (N - 1) % 64;
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (i == col) pl = ex2_approx(fmaf(sv[i], sl2, neg));
+          }
+          a_run += ps;
+          l_run += 64.f * ps - (64.f - (float)n_last) * pl;
+        } else {
+          l_run += ps;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+      }
+      tmem_st_x32(s_addr, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarPFull + b));
+    }
+    // ---- epilogue -----------------------------------------------------------
+    if (ok && T >= 1 && !__any_sync(0xffffffffu, misc[1] != 0)) {
+      const bool ready = warp_wait(bar(C::kBarFinal), 0);
+      if (!ready) {
+        misc[1] = 1;
+      } else {
+        tc_fence_after();
+        const int grow_row = (half ? qb1 : qb0) * 64 + (row & 63);
+        const bool store = exists && grow_row < L;
+        const float inv = 1.f / l_run;
+        const float fa = hyd ? scale * a_run : 0.f;
+        const size_t obase = ((size_t)bh * L + (size_t)(store ? grow_row : 0)) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32], qh[32];
+          tmem_ld_x32(lane_addr + C::kColO + 32 * c, o);
+          if (hyd) tmem_ld_x32(lane_addr + C::kColQH + 32 * c, qh);
+          tmem_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float acc = __uint_as_float(o[i]);
+            if (hyd) acc = fmaf(fa, __uint_as_float(qh[i]), acc);
+            v[i] = acc * inv;
+          }
+          if (store) {
+            if (out_f32) {
+              float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + obase + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(out) + obase + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                    pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+            }
+          }
+        }
+      }
+    }
+    if (!ok) misc[1] = 1;
+  }
+
+  // ---- teardown -----------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace pisa

@@ -1,0 +1,126 @@
+// Packing kernels of the fused-attention step: float32 statistics -> bf16
+// operands laid out for the tensor-memory-accelerator loads, and f32 -> bf16
+// copies of f32 inputs (the tensor-core products run on bf16).
+#pragma once
+
+#include "pisa_common.cuh"
+
+namespace pisa {
+
+// ---------------------------------------------------------------------------
+// packing helpers for K3
+// ---------------------------------------------------------------------------
+// kbar16/vsum16 [BH, Npad, D] (rows >= N zero), hbar16 [BH, D, D]
+__global__ void pack_stats_kernel(const float *__restrict__ kbar, const float *__restrict__ vsum,
+                                  const float *__restrict__ hbar, int N, int Npad, int D, int BH,
+                                  __nv_bfloat16 *__restrict__ kbar16,
+                                  __nv_bfloat16 *__restrict__ vsum16,
+                                  __nv_bfloat16 *__restrict__ hbar16) {
+  const size_t nrow = (size_t)BH * Npad * D;
+  const size_t nh = (size_t)BH * D * D;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < nrow + nh;
+       e += (size_t)gridDim.x * blockDim.x) {
+    if (e < nrow) {
+      const size_t bh = e / ((size_t)Npad * D), rem = e % ((size_t)Npad * D);
+      const int j = (int)(rem / D), c = (int)(rem % D);
+      const bool ok = j < N;
+      const size_t src = (bh * N + j) * D + c;
+      kbar16[e] = __float2bfloat16_rn(ok ? kbar[src] : 0.f);
+      vsum16[e] = __float2bfloat16_rn(ok ? vsum[src] : 0.f);
+    } else {
+      const size_t h = e - nrow;
+      hbar16[h] = __float2bfloat16_rn(hbar[h]);
+    }
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst,
+                                   size_t n) {
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
+       e += (size_t)gridDim.x * blockDim.x)
+    dst[e] = __float2bfloat16_rn(src[e]);
+}
+
+// ---------------------------------------------------------------------------
+// Pairing of query blocks for the 128-row attention tiles.
+//
+// The fused kernel runs two query blocks per CTA and loads the union of their
+// exact sets, so a partner whose selected set overlaps more costs fewer
+// tensor-core tiles.  Each query block i is paired greedily (ascending i) with
+// the still-unpaired block among i+1 .. i+kPairWindow whose exact set shares
+// the most blocks with S_i (ties: the nearer one); when all of those are taken,
+// with the next unpaired block.  Only the schedule changes: every row still
+// sees exactly its own S_i and U_i.
+// ---------------------------------------------------------------------------
+constexpr int kPairWindow = 16;
+
+// bm[bh][i][w]: bit j of word w set iff block 32w + j is in S_i.
+__global__ void selection_bitmap_kernel(const int32_t *__restrict__ idx, int N, int k_sel,
+                                        int nwords, uint32_t *__restrict__ bm) {
+  extern __shared__ uint32_t words[];
+  const size_t row = (size_t)blockIdx.y * N + blockIdx.x;
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) words[w] = 0u;
+  __syncthreads();
+  for (int t = threadIdx.x; t < k_sel; t += blockDim.x) {
+    const int j = idx[row * k_sel + t];
+    if (j >= 0 && j < N) atomicOr(&words[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) bm[row * nwords + w] = words[w];
+}
+
+// ov[bh][i][d-1] = |S_i n S_{i+d}| for d = 1 .. kPairWindow (0 past the end).
+__global__ void pair_overlap_kernel(const uint32_t *__restrict__ bm, int N, int nwords,
+                                    uint16_t *__restrict__ ov) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int bh = blockIdx.y;
+  if (i >= N || lane >= kPairWindow) return;
+  const int j = i + 1 + lane;
+  int cnt = 0;
+  if (j < N) {
+    const uint32_t *a = bm + ((size_t)bh * N + i) * nwords;
+    const uint32_t *b = bm + ((size_t)bh * N + j) * nwords;
+    for (int w = 0; w < nwords; ++w) cnt += __popc(a[w] & b[w]);
+  }
+  ov[((size_t)bh * N + i) * kPairWindow + lane] = (uint16_t)cnt;
+}
+
+// One warp per head; pairs[bh][p] = (i0, i1), i1 = -1 for an unpaired block.
+// Writes exactly ceil(N / 2) entries.
+__global__ void pairing_kernel(const uint16_t *__restrict__ ov, int N, int2 *__restrict__ pairs) {
+  extern __shared__ unsigned char used[];
+  const int bh = blockIdx.x, lane = threadIdx.x;
+  for (int i = lane; i < N; i += 32) used[i] = 0;
+  __syncwarp();
+  const uint16_t *o = ov + (size_t)bh * N * kPairWindow;
+  int2 *out = pairs + (size_t)bh * ((N + 1) / 2);
+  int np = 0;
+  for (int i = 0; i < N; ++i) {
+    if (used[i]) continue;  // uniform: every lane reads the same byte
+    const int j = i + 1 + lane;
+    const bool cand = lane < kPairWindow && j < N && !used[j];
+    // key: overlap high, then nearer partner first
+    const int key = cand ? ((int)o[(size_t)i * kPairWindow + lane] << 8) | (255 - lane) : -1;
+    int best = key;
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, s));
+    int partner = -1;
+    if (best >= 0) {
+      partner = i + 1 + (255 - (best & 255));
+    } else {
+      for (int jj = i + 1 + kPairWindow; jj < N; ++jj)
+        if (!used[jj]) { partner = jj; break; }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      used[i] = 1;
+      if (partner >= 0) used[partner] = 1;
+      out[np] = make_int2(i, partner);
+    }
+    __syncwarp();
+    ++np;
+  }
+}
+
+}  // namespace pisa

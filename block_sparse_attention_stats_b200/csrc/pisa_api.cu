@@ -1,5 +1,7 @@
 // libpisa C ABI: argument checking, scratch layout and kernel launches.
 // One translation unit: every kernel header is included here.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -12,7 +14,8 @@
 #include "pisa_common.cuh"
 #include "k1_block_stats.cuh"
 #include "k2_select.cuh"
-#include "k3_attention_mma.cuh"
+#include "k3_pack.cuh"
+#include "k3_attention_tc.cuh"
 
 namespace pisa {
 
@@ -74,12 +77,28 @@ static size_t stats_ws(int B, int H, int L, int d) {
 static size_t select_ws(int B, int H, int N) {
   return align_up((size_t)B * H * N * N * sizeof(float), 256);
 }
-static size_t sparse_ws(int B, int H, int L, int d, pisa_dtype dt) {
-  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
+// scratch of the fused-attention step: bf16 kbar/vsum/hbar, query-block
+// pairing (selection bitmaps, overlaps, pairs), bf16 copies of f32 inputs
+struct SparseLayout {
+  size_t kbar16, vsum16, hbar16, bm, ov, pairs, qkv16, total;
+};
+static SparseLayout sparse_layout(int B, int H, int L, int d, pisa_dtype dt) {
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
   const size_t BH = (size_t)B * H;
-  size_t s = 2 * align_up(BH * Npad * d * 2, 256) + align_up(BH * d * d * 2, 256);
-  if (dt == PISA_F32) s += 3 * align_up(BH * L * d * 2, 256);
-  return s;
+  SparseLayout p;
+  size_t o = 0;
+  p.kbar16 = o; o += align_up(BH * Npad * d * 2, 256);
+  p.vsum16 = o; o += align_up(BH * Npad * d * 2, 256);
+  p.hbar16 = o; o += align_up(BH * d * d * 2, 256);
+  p.bm = o; o += align_up(BH * N * nwords * 4, 256);
+  p.ov = o; o += align_up(BH * N * kPairWindow * 2, 256);
+  p.pairs = o; o += align_up(BH * ((N + 1) / 2) * 8, 256);
+  p.qkv16 = o; o += dt == PISA_F32 ? 3 * align_up(BH * L * d * 2, 256) : 0;
+  p.total = o;
+  return p;
+}
+static size_t sparse_ws(int B, int H, int L, int d, pisa_dtype dt) {
+  return sparse_layout(B, H, L, d, dt).total;
 }
 
 struct PathLayout {
@@ -178,22 +197,75 @@ static pisa_status launch_select(const float *qbar, const float *kbar, const flo
   return check_launch();
 }
 
-template <int D, bool DENSE>
+// ---- tensor maps for the tensor-memory-accelerator loads ------------------------
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor [planes][rows][cols] (cols contiguous, cols multiple of 64), read
+// in boxes of 64 columns x box_rows rows with the 128-byte swizzle; rows past
+// `rows` read as zero.
+static pisa_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                            uint64_t planes, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) {
+    t_last_error = "cuTensorMapEncodeTiled is not available from the driver";
+    return PISA_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {cols, rows, planes};
+  cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
+    return PISA_ERR_CUDA;
+  }
+  return PISA_OK;
+}
+
+template <int D>
 static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                            const __nv_bfloat16 *v, const __nv_bfloat16 *kbar16,
                                            const __nv_bfloat16 *vsum16,
                                            const __nv_bfloat16 *hbar16, const int32_t *idx,
-                                           int k_sel, int BH, int L, float scale, int hyd,
-                                           void *out, int out_f32, cudaStream_t st) {
+                                           const int2 *pairs, int k_sel, int BH, int L,
+                                           float scale, int hyd, int dense, void *out,
+                                           int out_f32, cudaStream_t st) {
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
-  const int nwords = ceil_div(N, 32);
-  const int smem = AttnSmem<D>::kFixed +
-                   (DENSE ? 0 : (nwords + k_sel + ceil_div(N, 64)) * (int)sizeof(int));
+  const int smem = TcCfg<D>::smem_bytes(N);
   if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
-  PISA_CUDA(cudaFuncSetAttribute(piecewise_attention_mma_kernel<D, DENSE>,
+  CUtensorMap mq, mk, mv, mkb, mvs, mh;
+  PISA_TRY(make_map(&mq, q, D, L, BH, 64));
+  PISA_TRY(make_map(&mk, k, D, L, BH, 64));
+  PISA_TRY(make_map(&mv, v, D, L, BH, 64));
+  if (dense) {
+    mkb = mk;
+    mvs = mv;
+    mh = mk;
+  } else {
+    PISA_TRY(make_map(&mkb, kbar16, D, Npad, BH, 64));
+    PISA_TRY(make_map(&mvs, vsum16, D, Npad, BH, 64));
+    PISA_TRY(make_map(&mh, hbar16, D, D, BH, D));
+  }
+  PISA_CUDA(cudaFuncSetAttribute(piecewise_attention_tc_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  piecewise_attention_mma_kernel<D, DENSE><<<dim3(N, BH), kAttnThreads, smem, st>>>(
-      q, k, v, kbar16, vsum16, hbar16, idx, k_sel, L, N, Npad, scale, hyd, out, out_f32);
+  piecewise_attention_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), TcCfg<D>::kThreads, smem, st>>>(
+      mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, scale, hyd, dense, out, out_f32);
   return check_launch();
 }
 
@@ -207,19 +279,32 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
                                         const float *hbar, const int32_t *idx, int k_sel, int BH,
                                         int L, int d, float scale, pisa_mode mode, void *out,
                                         unsigned char *ws, cudaStream_t st) {
-  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
-  __nv_bfloat16 *kbar16 = (__nv_bfloat16 *)ws;
-  __nv_bfloat16 *vsum16 = (__nv_bfloat16 *)(ws + align_up((size_t)BH * Npad * d * 2, 256));
-  __nv_bfloat16 *hbar16 = (__nv_bfloat16 *)(ws + 2 * align_up((size_t)BH * Npad * d * 2, 256));
-  unsigned char *next = ws + 2 * align_up((size_t)BH * Npad * d * 2, 256) +
-                        align_up((size_t)BH * d * d * 2, 256);
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+  const SparseLayout lay = sparse_layout(1, BH, L, d, dt);
+  __nv_bfloat16 *kbar16 = (__nv_bfloat16 *)(ws + lay.kbar16);
+  __nv_bfloat16 *vsum16 = (__nv_bfloat16 *)(ws + lay.vsum16);
+  __nv_bfloat16 *hbar16 = (__nv_bfloat16 *)(ws + lay.hbar16);
+  uint32_t *bm = (uint32_t *)(ws + lay.bm);
+  uint16_t *ov = (uint16_t *)(ws + lay.ov);
+  int2 *pairs = (int2 *)(ws + lay.pairs);
   pack_stats_kernel<<<grid_1d((size_t)BH * (Npad * d + d * d), 256), 256, 0, st>>>(
       kbar, vsum, hbar, N, Npad, d, BH, kbar16, vsum16, hbar16);
+  PISA_TRY(check_launch());
+  // schedule: pair query blocks whose exact sets overlap most
+  selection_bitmap_kernel<<<dim3(N, BH), 64, nwords * sizeof(uint32_t), st>>>(idx, N, k_sel,
+                                                                              nwords, bm);
+  PISA_TRY(check_launch());
+  pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, nwords, ov);
+  PISA_TRY(check_launch());
+  if (N > 48 * 1024)
+    PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, N));
+  pairing_kernel<<<BH, 32, N, st>>>(ov, N, pairs);
   PISA_TRY(check_launch());
   const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
                       *v16 = (const __nv_bfloat16 *)v;
   if (dt == PISA_F32) {
     const size_t n = (size_t)BH * L * d, sz = align_up(n * 2, 256);
+    unsigned char *next = ws + lay.qkv16;
     __nv_bfloat16 *a = (__nv_bfloat16 *)next, *b = (__nv_bfloat16 *)(next + sz),
                   *c = (__nv_bfloat16 *)(next + 2 * sz);
     PISA_TRY(to_bf16(q, a, n, st));
@@ -232,10 +317,10 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   const int hyd = mode == PISA_MODE_HYD;
   const int of32 = dt == PISA_F32;
   if (d == 128)
-    return launch_attention_kernel<128, false>(q16, k16, v16, kbar16, vsum16, hbar16, idx, k_sel,
-                                               BH, L, scale, hyd, out, of32, st);
-  return launch_attention_kernel<64, false>(q16, k16, v16, kbar16, vsum16, hbar16, idx, k_sel, BH,
-                                            L, scale, hyd, out, of32, st);
+    return launch_attention_kernel<128>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel,
+                                        BH, L, scale, hyd, 0, out, of32, st);
+  return launch_attention_kernel<64>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel, BH,
+                                     L, scale, hyd, 0, out, of32, st);
 }
 
 }  // namespace pisa
@@ -485,10 +570,10 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
   }
   const int of32 = dtype == PISA_F32;
   if (d == 128)
-    return launch_attention_kernel<128, true>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr,
-                                              0, BH, L, s, 0, out, of32, st);
-  return launch_attention_kernel<64, true>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, 0,
-                                           BH, L, s, 0, out, of32, st);
+    return launch_attention_kernel<128>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr,
+                                        nullptr, 0, BH, L, s, 0, 1, out, of32, st);
+  return launch_attention_kernel<64>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                     0, BH, L, s, 0, 1, out, of32, st);
 }
 
 pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v,
