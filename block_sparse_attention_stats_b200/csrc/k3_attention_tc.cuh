@@ -47,18 +47,19 @@ template <int D> struct TcCfg {
   static constexpr int kThreads = 192;
   static constexpr int kRows = 128;
   static constexpr int kKeys = 64;
-  static constexpr int kStages = 2;
+  static constexpr int kKStages = 2;                // K ring: a slot frees when its S MMA is done
+  static constexpr int kVStages = 2;                // V ring: a slot frees when its P V MMA is done
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kBoxQBytes = kRows * 128;   // one 64-column box of Q
   static constexpr int kBoxKBytes = kKeys * 128;   // one 64-column box of a K/V tile
   static constexpr int kTileBytes = kKeys * D * 2;
-  static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kHbarBytes = D * D * 2;
-  static_assert(kHbarBytes <= kStageBytes, "Hbar must fit in one stage");
+  static_assert(kHbarBytes <= kKStages * kTileBytes, "Hbar must fit in the K ring");
   static constexpr int kOffQ = 0;
-  static constexpr int kOffStage = kQBytes;
-  static constexpr int kOffBar = kOffStage + kStages * kStageBytes;
-  static constexpr int kNumBars = 16;
+  static constexpr int kOffK = kQBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kNumBars = 24;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffMisc = kOffTmemSlot + 16;
   static constexpr int kOffDyn = kOffMisc + 16;
@@ -68,14 +69,17 @@ template <int D> struct TcCfg {
   static constexpr uint32_t kColQH = D;
   // barrier indices
   static constexpr int kBarQ = 0;
-  static constexpr int kBarKvFull = 1;                  // + stage
-  static constexpr int kBarKvEmpty = 1 + kStages;       // + stage
-  static constexpr int kBarSFull = 1 + 2 * kStages;     // + buffer
-  static constexpr int kBarPFull = 3 + 2 * kStages;     // + buffer
-  static constexpr int kBarODone = 5 + 2 * kStages;
-  static constexpr int kBarFinal = 6 + 2 * kStages;     // after the last MMA
-  static constexpr int kBarTeardown = 7 + 2 * kStages;
-  static_assert(kBarTeardown < kNumBars, "barrier slots");
+  static constexpr int kBarKFull = 1;                   // + slot
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;
+  static constexpr int kBarVEmpty = kBarVFull + kVStages;
+  static constexpr int kBarSFull = kBarVEmpty + kVStages;  // + S buffer
+  static constexpr int kBarPFull = kBarSFull + 2;          // + S buffer
+  static constexpr int kBarODone = kBarPFull + 2;
+  static constexpr int kBarFinal = kBarODone + 1;          // after the last MMA
+  static constexpr int kBarTeardown = kBarFinal + 1;
+  static constexpr int kBarHFull = kBarTeardown + 1;
+  static_assert(kBarHFull < kNumBars, "barrier slots");
 
   __host__ __device__ static int smem_bytes(int N) {
     const int nwords = (N + 31) / 32;
@@ -133,10 +137,15 @@ __global__ void __launch_bounds__(192, 2)
   }
   if (tid == 0) {
     mbar_init(bar(C::kBarQ), 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(bar(C::kBarKvFull + s), 1);
-      mbar_init(bar(C::kBarKvEmpty + s), 1);
+    for (int s = 0; s < C::kKStages; ++s) {
+      mbar_init(bar(C::kBarKFull + s), 1);
+      mbar_init(bar(C::kBarKEmpty + s), 1);
     }
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(bar(C::kBarVFull + s), 1);
+      mbar_init(bar(C::kBarVEmpty + s), 1);
+    }
+    mbar_init(bar(C::kBarHFull), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(C::kBarSFull + b), 1);
       mbar_init(bar(C::kBarPFull + b), 128);
@@ -225,8 +234,6 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 0) {
     // ======================= TMA producer =====================================
     if (lane == 0) {
-      const int total = T + (hyd ? 1 : 0);
-      int issued = 0;
       // Q rows of both query blocks (an absent upper block reads as zeros)
       mbar_expect_tx(bar(C::kBarQ), C::kQBytes);
 #pragma unroll
@@ -235,39 +242,57 @@ __global__ void __launch_bounds__(192, 2)
         tma_load_3d(dst, &tm_q, bar(C::kBarQ), 64 * b, qb0 * 64, bh);
         tma_load_3d(dst + 64 * 128, &tm_q, bar(C::kBarQ), 64 * b, has_hi ? qb1 * 64 : L, bh);
       }
-      for (int t = 0; t < total; ++t) {
-        if (misc[1]) break;
-        const int s = t % C::kStages;
-        if (t >= C::kStages && !mbar_wait(bar(C::kBarKvEmpty + s), ((t / C::kStages) - 1) & 1)) {
-          misc[1] = 1;
-          break;
-        }
-        const uint32_t st = sbase + C::kOffStage + s * C::kStageBytes;
-        const uint32_t full = bar(C::kBarKvFull + s);
-        if (t < T) {
-          const int e = tiles[t];
-          const CUtensorMap *mk = e >= 0 ? &tm_k : &tm_kbar;
-          const CUtensorMap *mv = e >= 0 ? &tm_v : &tm_vsum;
-          const int row = e >= 0 ? (e >> 2) * 64 : (-e - 1) * 64;
-          mbar_expect_tx(full, C::kStageBytes);
+      int k_issued = 0, v_issued = 0;
+      bool h_issued = false, ok = true;
+      // tile t of the list: exact block j (K, V rows) or centroid chunk c (kbar, vsum rows)
+      auto load = [&](int t, bool is_k) -> bool {
+        const int ns = is_k ? C::kKStages : C::kVStages;
+        const int sl = t % ns;
+        const uint32_t empty = bar((is_k ? C::kBarKEmpty : C::kBarVEmpty) + sl);
+        const uint32_t full = bar((is_k ? C::kBarKFull : C::kBarVFull) + sl);
+        if (t >= ns && !mbar_wait(empty, ((t / ns) - 1) & 1)) return false;
+        const int e = tiles[t];
+        const CUtensorMap *m = e >= 0 ? (is_k ? &tm_k : &tm_v) : (is_k ? &tm_kbar : &tm_vsum);
+        const int row = e >= 0 ? (e >> 2) * 64 : (-e - 1) * 64;
+        const uint32_t dst = sbase + (is_k ? C::kOffK : C::kOffV) + sl * C::kTileBytes;
+        mbar_expect_tx(full, C::kTileBytes);
 #pragma unroll
-          for (int b = 0; b < D / 64; ++b) {
-            tma_load_3d(st + b * C::kBoxKBytes, mk, full, 64 * b, row, bh);
-            tma_load_3d(st + C::kTileBytes + b * C::kBoxKBytes, mv, full, 64 * b, row, bh);
-          }
-        } else {
-          mbar_expect_tx(full, C::kHbarBytes);
+        for (int b = 0; b < D / 64; ++b) tma_load_3d(dst + b * C::kBoxKBytes, m, full, 64 * b, row, bh);
+        return true;
+      };
+      // K runs one tile ahead of V: K_t is due at S_t, V_t only after softmax_t
+      for (int t = 0; ok && t <= T; ++t) {
+        if (misc[1]) { ok = false; break; }
+        if (t < T) {
+          if (!load(t, true)) { ok = false; break; }
+          k_issued = t + 1;
+        }
+        if (t >= 1) {
+          if (!load(t - 1, false)) { ok = false; break; }
+          v_issued = t;
+        }
+      }
+      if (ok && hyd) {
+        // Hbar goes into the K ring once every S = Q K^T has completed
+        for (int u = (T >= C::kKStages ? T - C::kKStages : 0); ok && u < T; ++u)
+          ok = mbar_wait(bar(C::kBarKEmpty + u % C::kKStages), (u / C::kKStages) & 1);
+        if (ok) {
+          mbar_expect_tx(bar(C::kBarHFull), C::kHbarBytes);
 #pragma unroll
           for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(st + b * (D * 128), &tm_hbar, full, 64 * b, 0, bh);
+            tma_load_3d(sbase + C::kOffK + b * (D * 128), &tm_hbar, bar(C::kBarHFull), 64 * b, 0, bh);
+          h_issued = true;
         }
-        issued = t + 1;
       }
-      if (misc[1]) {
+      if (!ok) {
+        misc[1] = 1;
         // let the copies already in flight land before the CTA exits
         mbar_wait(bar(C::kBarQ), 0);
-        for (int t = issued - C::kStages; t < issued; ++t)
-          if (t >= 0) mbar_wait(bar(C::kBarKvFull + t % C::kStages), (t / C::kStages) & 1);
+        for (int t = k_issued - C::kKStages; t < k_issued; ++t)
+          if (t >= 0) mbar_wait(bar(C::kBarKFull + t % C::kKStages), (t / C::kKStages) & 1);
+        for (int t = v_issued - C::kVStages; t < v_issued; ++t)
+          if (t >= 0) mbar_wait(bar(C::kBarVFull + t % C::kVStages), (t / C::kVStages) & 1);
+        if (h_issued) mbar_wait(bar(C::kBarHFull), 0);
       }
     }
   } else if (warp == 1) {
@@ -281,40 +306,41 @@ __global__ void __launch_bounds__(192, 2)
         return smem_desc_sw128(sbase + C::kOffQ + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
       };
       auto issue_pv = [&](int u) -> bool {
-        const int bu = u & 1, su = u % C::kStages;
+        const int bu = u & 1, sv = u % C::kVStages;
         if (!mbar_wait(bar(C::kBarPFull + bu), (u >> 1) & 1)) return false;
+        if (!mbar_wait(bar(C::kBarVFull + sv), (u / C::kVStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t vst = sbase + C::kOffStage + su * C::kStageBytes + C::kTileBytes;
+        const uint32_t vst = sbase + C::kOffV + sv * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tmem + C::kColO, tmem + C::kColS + 64 * bu + kk * 8,
                  smem_desc_sw128(vst + kk * 2048, C::kBoxKBytes, 1024), kIdPV,
                  (u > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C::kBarKvEmpty + su));
+        tc_commit(bar(C::kBarVEmpty + sv));
         tc_commit(bar(C::kBarODone));
         return true;
       };
       for (int t = 0; ok && t < T; ++t) {
         if (misc[1]) { ok = false; break; }
-        const int s = t % C::kStages, b = t & 1;
-        if (!mbar_wait(bar(C::kBarKvFull + s), (t / C::kStages) & 1)) { ok = false; break; }
+        const int sk = t % C::kKStages, b = t & 1;
+        if (!mbar_wait(bar(C::kBarKFull + sk), (t / C::kKStages) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t kst = sbase + C::kOffStage + s * C::kStageBytes;
+        const uint32_t kst = sbase + C::kOffK + sk * C::kTileBytes;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem + C::kColS + 64 * b, q_desc(k),
                  smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024), kIdQK,
                  k > 0 ? 1u : 0u);
         tc_commit(bar(C::kBarSFull + b));
+        tc_commit(bar(C::kBarKEmpty + sk));
         if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
       }
       if (ok && T >= 1) ok = issue_pv(T - 1);
       if (ok && !hyd) tc_commit(bar(C::kBarFinal));
       if (ok && hyd) {
-        const int s = T % C::kStages;
-        if (mbar_wait(bar(C::kBarKvFull + s), (T / C::kStages) & 1)) {
+        if (mbar_wait(bar(C::kBarHFull), 0)) {
           tc_fence_after();
-          const uint32_t hst = sbase + C::kOffStage + s * C::kStageBytes;
+          const uint32_t hst = sbase + C::kOffK;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             mma_ss(tmem + C::kColQH, q_desc(k), smem_desc_sw128(hst + k * 2048, D * 128, 1024),
@@ -390,8 +416,18 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
           for (int i = 0; i < 64; ++i) sv[i] = ((keep >> i) & 1ull) ? sv[i] : -INFINITY;
         }
+        {
+          float mx[8];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, sv[i]);
+          for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+          for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+#pragma unroll
+          for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+            for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+          tmax = mx[0];
+        }
         const float m_t = tmax * sl2;                  // finite: the row has a key here
         const bool grow = m_t > m_run + 8.0f;          // lazy rescale threshold 2^8
         const bool need_o = grow && m_run != -INFINITY;
@@ -417,14 +453,15 @@ __global__ void __launch_bounds__(192, 2)
           a_run *= f;
         }
         const float neg = -m_run;
-        float ps = 0.f;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float p0 = ex2_approx(fmaf(sv[2 * i], sl2, neg));
           const float p1 = ex2_approx(fmaf(sv[2 * i + 1], sl2, neg));
-          ps += p0 + p1;
+          acc[i & 7] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
+        const float ps = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         if (centroid) {
           // weight n_j = 64 except for the last block, which holds n_last tokens
           float pl = 0.f;
