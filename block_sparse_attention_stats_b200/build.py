@@ -46,7 +46,7 @@ def needs_build() -> bool:
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+def build(force: bool = False, ptxas_verbose: bool = False, log: str = "") -> str:
     if not force and not needs_build():
         return LIB
     cmd = [_nvcc(), *ARCH_FLAGS, "-O3", "-std=c++17", "-lineinfo", "--shared",
@@ -58,7 +58,11 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
     if ptxas_verbose:
-        sys.stderr.write(r.stderr)
+        if log:
+            with open(log, "w") as f:
+                f.write(r.stderr)
+        else:
+            sys.stderr.write(r.stderr)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

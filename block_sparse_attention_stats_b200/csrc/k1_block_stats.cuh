@@ -28,9 +28,9 @@ namespace pisa {
 constexpr int kStatsThreads = 256;
 constexpr int kBlk = 64;  // tokens per block (block_size)
 
-// Chunking of pass 1: about two CTAs per SM over the whole problem.
+// Chunking of pass 1: at most two CTAs per SM over the whole problem (one wave).
 __host__ __device__ inline int stats_num_chunks(int BH, int N) {
-  int want = (2 * 148 + BH - 1) / BH;
+  int want = (2 * 148) / BH;
   if (want < 1) want = 1;
   return want < N ? want : N;
 }
@@ -93,6 +93,49 @@ __device__ __forceinline__ void ktv_mma(float (&acc)[StatsMmaCfg<D>::kMT][StatsM
   }
 }
 
+// Column sums of the Q, K and V tiles (3 x D columns, 64 rows each) on the
+// tensor cores: C = 1^T X with an all-ones A operand; every row of C holds the
+// column sums.  Warp w handles n-tiles 6w .. 6w+5 of the 3D/8 tiles.
+template <int D>
+__device__ __forceinline__ void colsum_mma(uint32_t tiles, float *colsum, int warp, int lane) {
+  using C = StatsMmaCfg<D>;
+  constexpr int kNT = 3 * D / 8;           // 8-column tiles over Q, K, V
+  constexpr int kPerWarp = kNT / 8;        // 6 (D=128) or 3 (D=64)
+  const uint32_t one2 = 0x3F803F80u;       // two bf16 1.0
+  const uint32_t ones[4] = {one2, one2, one2, one2};
+  float acc[kPerWarp][4];
+#pragma unroll
+  for (int i = 0; i < kPerWarp; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+  const int mi = lane >> 3, r = lane & 7;
+#pragma unroll
+  for (int k0 = 0; k0 < kBlk; k0 += 16) {
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+      const int nt = warp * kPerWarp + i;
+      const int which = nt / (D / 8), col = (nt % (D / 8)) * 8;
+      // B fragment (16 tokens x 8 columns) of tile `which`, via ldmatrix.trans
+      const int tok = k0 + r + 8 * (mi & 1);
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(tiles + which * C::kTileBytes + SwizzledTile<D>::offset(tok, col), b0, b1,
+                        b2, b3);
+      (void)b2;
+      (void)b3;
+      mma_bf16_16816(acc[i], ones, b0, b1);
+    }
+  }
+  if (lane < 4) {
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+      const int nt = warp * kPerWarp + i;
+      const int which = nt / (D / 8), col = (nt % (D / 8)) * 8 + 2 * lane;
+      colsum[which * D + col] = acc[i][0];
+      colsum[which * D + col + 1] = acc[i][1];
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kStatsThreads)
     stats_pass_bf16_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
@@ -139,19 +182,9 @@ __global__ void __launch_bounds__(kStatsThreads)
     cp_async_wait<1>();
     __syncthreads();
 
-    const unsigned char *tiles = smem + stage * 3 * C::kTileBytes;
     const int n_j = min(kBlk, L - j * kBlk);
     // column sums of Q, K, V (zero-filled rows past L add nothing)
-    for (int t = tid; t < 3 * D; t += kStatsThreads) {
-      const int which = t / D, col = t % D;
-      const unsigned char *tile = tiles + which * C::kTileBytes;
-      float s = 0.f;
-#pragma unroll 8
-      for (int row = 0; row < kBlk; ++row)
-        s += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-            tile + SwizzledTile<D>::offset(row, col)));
-      colsum[t] = s;
-    }
+    colsum_mma<D>(sbase + stage * 3 * C::kTileBytes, colsum, warp, lane);
     const uint32_t sK = sbase + stage * 3 * C::kTileBytes + C::kTileBytes;
     ktv_mma<D>(acc, sK, sK + C::kTileBytes, warp_m0, warp_n0, lane);
     __syncthreads();  // colsum visible

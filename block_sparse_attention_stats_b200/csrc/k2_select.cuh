@@ -10,73 +10,87 @@
 //
 // Pass 1 (scores_kernel): a float32 FMA GEMM per head, 64 x 64 output tiles,
 // each score summed over the head dimension in ascending order.
-// Pass 2 (topk_kernel): one CTA per query block.  Scores become 32-bit keys
+// Pass 2 (topk_kernel): one warp per query block.  Scores become 32-bit keys
 // whose unsigned order is the float order; an MSB-first radix select (4 x 8
 // bits) finds the k-th largest key T; every key > T is kept, and of the keys
 // equal to T the lowest block indices are kept (ties go to the lower index).
 // The sink block is set aside first and always kept.  Indices come out
-// ascending via a block-wide prefix sum.
+// ascending via warp ballots.
 #pragma once
 
 #include "pisa_common.cuh"
 
 namespace pisa {
 
-constexpr int kScoreTile = 64;
-constexpr int kScoreK = 32;
+// Scores: C = scale * Qbar Kbar^T + lambda * cov over 128 x 128 tiles, 256
+// threads with 8 x 8 outputs each; operands staged in shared memory as
+// [dim][row] so every thread reads its 8 rows / 8 columns as two float4.
+// Each score is accumulated over the head dimension in ascending order.
+constexpr int kScoreTile = 128;
+constexpr int kScoreK = 16;
+constexpr int kScorePad = 4;
 
 __global__ void __launch_bounds__(256)
     scores_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar,
                   const float *__restrict__ cov, float cov_weight, float scale, int N, int D,
                   float *__restrict__ scores) {
-  __shared__ __align__(16) float As[kScoreK][kScoreTile];
-  __shared__ __align__(16) float Bs[kScoreK][kScoreTile];
+  __shared__ __align__(16) float As[kScoreK][kScoreTile + kScorePad];
+  __shared__ __align__(16) float Bs[kScoreK][kScoreTile + kScorePad];
   const int bh = blockIdx.z;
   const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
   const float *qb = qbar + (size_t)bh * N * D;
   const float *kb = kbar + (size_t)bh * N * D;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  float acc[4][4];
+  float acc[8][8];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
 
   for (int e0 = 0; e0 < D; e0 += kScoreK) {
-    // load 64 rows x 32 dims of qbar and kbar, transposed into [dim][row]
-    for (int t = tid; t < kScoreTile * kScoreK; t += 256) {
-      const int row = t / kScoreK, e = t % kScoreK;
+    // 128 rows x 16 dims of each operand: two float4 per thread per operand
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int t = tid + 256 * h;
+      const int row = t >> 2, e4 = (t & 3) * 4;
       const int gi = i0 + row, gj = j0 + row;
-      As[e][row] = gi < N ? qb[(size_t)gi * D + e0 + e] : 0.f;
-      Bs[e][row] = gj < N ? kb[(size_t)gj * D + e0 + e] : 0.f;
+      const float4 a = gi < N ? *reinterpret_cast<const float4 *>(qb + (size_t)gi * D + e0 + e4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 b = gj < N ? *reinterpret_cast<const float4 *>(kb + (size_t)gj * D + e0 + e4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      As[e4 + 0][row] = a.x; As[e4 + 1][row] = a.y; As[e4 + 2][row] = a.z; As[e4 + 3][row] = a.w;
+      Bs[e4 + 0][row] = b.x; Bs[e4 + 1][row] = b.y; Bs[e4 + 2][row] = b.z; Bs[e4 + 3][row] = b.w;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll
     for (int e = 0; e < kScoreK; ++e) {
-      const float4 a = *reinterpret_cast<const float4 *>(&As[e][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4 *>(&Bs[e][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[e][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[e][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[e][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[e][tx * 8 + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
     }
     __syncthreads();
   }
-  float cw[4];
+  float cw[8];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const int gj = j0 + tx * 4 + c;
+  for (int c = 0; c < 8; ++c) {
+    const int gj = j0 + tx * 8 + c;
     cw[c] = (cov_weight != 0.f && gj < N) ? cov_weight * cov[(size_t)bh * N + gj] : 0.f;
   }
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int gi = i0 + ty * 4 + r;
+  for (int r = 0; r < 8; ++r) {
+    const int gi = i0 + ty * 8 + r;
     if (gi >= N) continue;
     float *out = scores + ((size_t)bh * N + gi) * N;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int gj = j0 + tx * 4 + c;
+    for (int c = 0; c < 8; ++c) {
+      const int gj = j0 + tx * 8 + c;
       if (gj < N) out[gj] = scale * acc[r][c] + cw[c];
     }
   }
@@ -89,126 +103,108 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-constexpr int kTopkThreads = 256;
+constexpr int kTopkThreads = 256;  // 8 warps, one query block per warp
 
-// Block-wide exclusive prefix sum of 0/1 flags in thread order; returns this
-// thread's prefix and writes the block total to *total.
-__device__ __forceinline__ int block_exclusive_scan(int flag, int *warp_tot, int *total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned bal = __ballot_sync(0xffffffffu, flag);
-  const int in_warp = __popc(bal & ((1u << lane) - 1u));
-  if (lane == 0) warp_tot[warp] = __popc(bal);
-  __syncthreads();
-  int before = 0, all = 0;
-#pragma unroll
-  for (int w = 0; w < kTopkThreads / 32; ++w) {
-    const int c = warp_tot[w];
-    before += (w < warp) ? c : 0;
-    all += c;
-  }
-  __syncthreads();
-  *total = all;
-  return before + in_warp;
-}
-
+// One warp selects the exact set of one query block.  The row's scores stay
+// in global memory (L2) and are re-read on every pass.
 __global__ void __launch_bounds__(kTopkThreads)
-    topk_kernel(const float *__restrict__ scores, int N, int k_sel, int sink,
+    topk_kernel(const float *__restrict__ scores, int N, int k_sel, int sink, size_t rows,
                 int32_t *__restrict__ idx) {
-  extern __shared__ uint32_t keys[];  // N
-  __shared__ unsigned hist[256];
-  __shared__ int warp_tot[kTopkThreads / 32];
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_remaining;
-
-  const size_t row = blockIdx.x;
+  __shared__ unsigned hist_all[kTopkThreads / 32][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * (kTopkThreads / 32) + warp;
+  if (row >= rows) return;
+  unsigned *hist = hist_all[warp];
   const float *sc = scores + row * N;
   int32_t *out = idx + row * k_sel;
-  const int tid = threadIdx.x;
-
-  for (int j = tid; j < N; j += kTopkThreads) keys[j] = float_key(sc[j]);
-  if (tid == 0) {
-    s_prefix = 0u;
-    s_mask = 0u;
-    s_remaining = k_sel - (sink >= 0 ? 1 : 0);
-  }
-  __syncthreads();
-
+  const int need = k_sel - (sink >= 0 ? 1 : 0);
   const int candidates = N - (sink >= 0 ? 1 : 0);
-  const bool take_all = s_remaining >= candidates;
-  if (!take_all && s_remaining > 0) {
+  const bool take_all = need >= candidates;
+
+  uint32_t prefix = 0u, mask = 0u;
+  int rem = need;
+  if (!take_all && need > 0) {
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
-      hist[tid] = 0u;  // kTopkThreads == 256 bins
-      __syncthreads();
-      const uint32_t prefix = s_prefix, mask = s_mask;
-      for (int j = tid; j < N; j += kTopkThreads) {
-        const uint32_t key = keys[j];
-        if (j != sink && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (tid < 32) {
-        // lane l owns digits 255-8l down to 248-8l (largest digits first)
-        const int lane = tid;
-        unsigned own = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) own += hist[255 - 8 * lane - q];
-        unsigned incl = own;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
+      for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0u;
+      __syncwarp();
+      for (int j0 = 0; j0 < N; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = j < N ? float_key(sc[j]) : 0u;
+        const bool part = j < N && j != sink && (key & mask) == prefix;
+        const unsigned act = __ballot_sync(0xffffffffu, part);
+        if (part) {
+          // aggregate lanes that hit the same bin into one shared-memory atomic
+          const unsigned digit = (key >> shift) & 255u;
+          const unsigned peers = __match_any_sync(act, digit);
+          if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
         }
-        const unsigned excl = incl - own;
-        const int rem = s_remaining;
-        const bool here = excl < (unsigned)rem && (unsigned)rem <= incl;
-        const unsigned who = __ballot_sync(0xffffffffu, here);
-        if (here && lane == __ffs(who) - 1) {
-          unsigned cum = excl;
-          for (int q = 0; q < 8; ++q) {
-            const int digit = 255 - 8 * lane - q;
-            const unsigned c = hist[digit];
-            if ((unsigned)rem <= cum + c) {
-              s_remaining = rem - (int)cum;
-              s_prefix = prefix | ((uint32_t)digit << shift);
-              s_mask = mask | (255u << shift);
-              break;
-            }
-            cum += c;
+      }
+      __syncwarp();
+      // lane l owns digits 255-8l .. 248-8l (largest first)
+      unsigned own = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) own += hist[255 - 8 * lane - q];
+      unsigned incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const unsigned excl = incl - own;
+      const bool here = excl < (unsigned)rem && (unsigned)rem <= incl;
+      const unsigned who = __ballot_sync(0xffffffffu, here);
+      const int src = __ffs(who) - 1;
+      int digit_sel = 0, new_rem = 0;
+      if (lane == src) {
+        unsigned cum = excl;
+        for (int q = 0; q < 8; ++q) {
+          const int digit = 255 - 8 * lane - q;
+          const unsigned c = hist[digit];
+          if ((unsigned)rem <= cum + c) {
+            digit_sel = digit;
+            new_rem = rem - (int)cum;
+            break;
           }
+          cum += c;
         }
       }
-      __syncthreads();
+      digit_sel = __shfl_sync(0xffffffffu, digit_sel, src);
+      new_rem = __shfl_sync(0xffffffffu, new_rem, src);
+      prefix |= (uint32_t)digit_sel << shift;
+      mask |= 255u << shift;
+      rem = new_rem;
+      __syncwarp();
     }
   }
-  const uint32_t T = s_prefix;
-  const int take_eq = s_remaining;
-
-  // selection flags in index order, then ascending compaction
+  // keep: the sink, every key > T, and the lowest-index `rem` keys equal to T
+  const uint32_t T = prefix;
   int eq_base = 0, out_base = 0;
-  for (int j0 = 0; j0 < N; j0 += kTopkThreads) {
-    const int j = j0 + tid;
+  for (int j0 = 0; j0 < N; j0 += 32) {
+    const int j = j0 + lane;
     const bool valid = j < N;
-    const uint32_t key = valid ? keys[j] : 0u;
+    const uint32_t key = valid ? float_key(sc[j]) : 0u;
     const bool cand = valid && j != sink;
-    const int is_eq = (cand && !take_all && key == T) ? 1 : 0;
-    int eq_tot;
-    const int eq_rank = eq_base + block_exclusive_scan(is_eq, warp_tot, &eq_tot);
+    const bool is_eq = cand && !take_all && need > 0 && key == T;
+    const unsigned eq_bal = __ballot_sync(0xffffffffu, is_eq);
+    const int eq_rank = eq_base + __popc(eq_bal & ((1u << lane) - 1u));
     bool sel;
     if (!valid) sel = false;
     else if (j == sink) sel = true;
     else if (take_all) sel = true;
-    else if (k_sel - (sink >= 0 ? 1 : 0) <= 0) sel = false;
-    else sel = key > T || (is_eq && eq_rank < take_eq);
-    int sel_tot;
-    const int pos = out_base + block_exclusive_scan(sel ? 1 : 0, warp_tot, &sel_tot);
+    else if (need <= 0) sel = false;
+    else sel = key > T || (is_eq && eq_rank < rem);
+    const unsigned sel_bal = __ballot_sync(0xffffffffu, sel);
+    const int pos = out_base + __popc(sel_bal & ((1u << lane) - 1u));
     if (sel) {
       if (pos < k_sel) out[pos] = j;
       else report_device_error(kDevErrRange);
     }
-    eq_base += eq_tot;
-    out_base += sel_tot;
+    eq_base += __popc(eq_bal);
+    out_base += __popc(sel_bal);
   }
-  if (tid == 0 && out_base != k_sel) report_device_error(kDevErrRange);
+  if (lane == 0 && out_base != k_sel) report_device_error(kDevErrRange);
 }
 
 }  // namespace pisa

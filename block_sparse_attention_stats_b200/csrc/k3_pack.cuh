@@ -87,13 +87,28 @@ __global__ void pair_overlap_kernel(const uint32_t *__restrict__ bm, int N, int 
 }
 
 // One warp per head; pairs[bh][p] = (i0, i1), i1 = -1 for an unpaired block.
-// Writes exactly ceil(N / 2) entries.
-__global__ void pairing_kernel(const uint16_t *__restrict__ ov, int N, int2 *__restrict__ pairs) {
-  extern __shared__ unsigned char used[];
+// Writes exactly ceil(N / 2) entries.  The head's overlap table is staged in
+// shared memory first (N * kPairWindow * 2 bytes), then the greedy pass runs
+// from shared memory only.
+// With staged == 0 (tables too large for shared memory) the table is read
+// from global memory instead.
+__global__ void pairing_kernel(const uint16_t *__restrict__ ov, int N, int staged,
+                               int2 *__restrict__ pairs) {
+  extern __shared__ __align__(16) unsigned char pair_smem[];
   const int bh = blockIdx.x, lane = threadIdx.x;
+  const uint16_t *head = ov + (size_t)bh * N * kPairWindow;
+  const uint16_t *o = head;
+  unsigned char *used = pair_smem;
+  if (staged) {
+    uint16_t *t = reinterpret_cast<uint16_t *>(pair_smem);
+    const uint4 *src = reinterpret_cast<const uint4 *>(head);
+    uint4 *dst = reinterpret_cast<uint4 *>(t);
+    for (int i = lane; i < N * kPairWindow / 8; i += 32) dst[i] = src[i];
+    o = t;
+    used = pair_smem + (size_t)N * kPairWindow * 2;
+  }
   for (int i = lane; i < N; i += 32) used[i] = 0;
   __syncwarp();
-  const uint16_t *o = ov + (size_t)bh * N * kPairWindow;
   int2 *out = pairs + (size_t)bh * ((N + 1) / 2);
   int np = 0;
   for (int i = 0; i < N; ++i) {

@@ -189,11 +189,10 @@ static pisa_status launch_select(const float *qbar, const float *kbar, const flo
   dim3 g1(ceil_div(N, kScoreTile), ceil_div(N, kScoreTile), BH);
   scores_kernel<<<g1, 256, 0, st>>>(qbar, kbar, cov, cov_weight, scale, N, d, scores);
   PISA_TRY(check_launch());
-  const int smem = N * (int)sizeof(uint32_t);
-  if (smem > 48 * 1024)
-    PISA_CUDA(cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  topk_kernel<<<(unsigned)((size_t)BH * N), kTopkThreads, smem, st>>>(scores, N, k_sel, sink,
-                                                                        idx);
+  const size_t rows = (size_t)BH * N;
+  const int per_cta = kTopkThreads / 32;
+  topk_kernel<<<(unsigned)((rows + per_cta - 1) / per_cta), kTopkThreads, 0, st>>>(
+      scores, N, k_sel, sink, rows, idx);
   return check_launch();
 }
 
@@ -296,9 +295,12 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   PISA_TRY(check_launch());
   pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, nwords, ov);
   PISA_TRY(check_launch());
-  if (N > 48 * 1024)
-    PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, N));
-  pairing_kernel<<<BH, 32, N, st>>>(ov, N, pairs);
+  const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
+  const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
+  if (pair_smem > 48 * 1024)
+    PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   pair_smem));
+  pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
   PISA_TRY(check_launch());
   const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
                       *v16 = (const __nv_bfloat16 *)v;
