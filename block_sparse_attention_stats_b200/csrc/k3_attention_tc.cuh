@@ -419,14 +419,14 @@ __global__ void __launch_bounds__(192, 2)
         {
           float mx[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+          for (int i = 0; i < 8; ++i) mx[i] = max3f(sv[i], sv[i + 8], sv[i + 16]);
 #pragma unroll
-          for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+          for (int i = 0; i < 8; ++i) mx[i] = max3f(mx[i], sv[i + 24], sv[i + 32]);
 #pragma unroll
-          for (int w = 4; w > 0; w >>= 1)
+          for (int i = 0; i < 8; ++i) mx[i] = max3f(mx[i], sv[i + 40], sv[i + 48]);
 #pragma unroll
-            for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-          tmax = mx[0];
+          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], sv[i + 56]);
+          tmax = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         }
         const float m_t = tmax * sl2;                  // finite: the row has a key here
         const bool grow = m_t > m_run + 8.0f;          // lazy rescale threshold 2^8
@@ -453,15 +453,18 @@ __global__ void __launch_bounds__(192, 2)
           a_run *= f;
         }
         const float neg = -m_run;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float2 sl2x2 = make_float2(sl2, sl2), neg2 = make_float2(neg, neg);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[2 * i], sl2, neg));
-          const float p1 = ex2_approx(fmaf(sv[2 * i + 1], sl2, neg));
-          acc[i & 7] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          const float2 x = fma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2x2, neg2);
+          const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          acc[i & 3] = add2(acc[i & 3], p);
+          pk[i] = pack_bf16x2(p.x, p.y);
         }
-        const float ps = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        const float2 s2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+        const float ps = s2.x + s2.y;
         if (centroid) {
           // weight n_j = 64 except for the last block, which holds n_last tokens
           float pl = 0.f;
