@@ -128,7 +128,11 @@ __global__ void __launch_bounds__(192, 2)
     qb1 = pr.y;
   }
   const bool has_hi = qb1 >= 0;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // warp index through a shuffle so the compiler knows it is warp-uniform: the
+  // producer and MMA warps then run converged and keep their descriptors in
+  // uniform registers (one elected lane issues each TMA copy / MMA)
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
 
   // ---- set-up ---------------------------------------------------------------
   if (warp == 1) {
@@ -231,10 +235,16 @@ __global__ void __launch_bounds__(192, 2)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + C::kOffTmemSlot);
   const int T = misc[0];
 
+  // warp-uniform bounded wait (every lane polls; all agree on the outcome)
+  auto uwait = [&](uint32_t b_addr, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(b_addr, parity));
+  };
+  auto aborted = [&]() -> bool { return __any_sync(0xffffffffu, misc[1] != 0); };
+
   if (warp == 0) {
     // ======================= TMA producer =====================================
-    if (lane == 0) {
-      // Q rows of both query blocks (an absent upper block reads as zeros)
+    // Q rows of both query blocks (an absent upper block reads as zeros)
+    if (elect_one()) {
       mbar_expect_tx(bar(C::kBarQ), C::kQBytes);
 #pragma unroll
       for (int b = 0; b < D / 64; ++b) {
@@ -242,75 +252,82 @@ __global__ void __launch_bounds__(192, 2)
         tma_load_3d(dst, &tm_q, bar(C::kBarQ), 64 * b, qb0 * 64, bh);
         tma_load_3d(dst + 64 * 128, &tm_q, bar(C::kBarQ), 64 * b, has_hi ? qb1 * 64 : L, bh);
       }
-      int k_issued = 0, v_issued = 0;
-      bool h_issued = false, ok = true;
-      // tile t of the list: exact block j (K, V rows) or centroid chunk c (kbar, vsum rows)
-      auto load = [&](int t, bool is_k) -> bool {
-        const int ns = is_k ? C::kKStages : C::kVStages;
-        const int sl = t % ns;
-        const uint32_t empty = bar((is_k ? C::kBarKEmpty : C::kBarVEmpty) + sl);
-        const uint32_t full = bar((is_k ? C::kBarKFull : C::kBarVFull) + sl);
-        if (t >= ns && !mbar_wait(empty, ((t / ns) - 1) & 1)) return false;
-        const int e = tiles[t];
-        const CUtensorMap *m = e >= 0 ? (is_k ? &tm_k : &tm_v) : (is_k ? &tm_kbar : &tm_vsum);
-        const int row = e >= 0 ? (e >> 2) * 64 : (-e - 1) * 64;
-        const uint32_t dst = sbase + (is_k ? C::kOffK : C::kOffV) + sl * C::kTileBytes;
+    }
+    __syncwarp();
+    int k_issued = 0, v_issued = 0;
+    bool h_issued = false, ok = true;
+    // tile t of the list: exact block j (K, V rows) or centroid chunk c (kbar, vsum rows)
+    auto load = [&](int t, bool is_k) -> bool {
+      const int ns = is_k ? C::kKStages : C::kVStages;
+      const int sl = t % ns;
+      const uint32_t empty = bar((is_k ? C::kBarKEmpty : C::kBarVEmpty) + sl);
+      const uint32_t full = bar((is_k ? C::kBarKFull : C::kBarVFull) + sl);
+      if (t >= ns && !uwait(empty, ((t / ns) - 1) & 1)) return false;
+      const int e = tiles[t];
+      const CUtensorMap *m = e >= 0 ? (is_k ? &tm_k : &tm_v) : (is_k ? &tm_kbar : &tm_vsum);
+      const int row = e >= 0 ? (e >> 2) * 64 : (-e - 1) * 64;
+      const uint32_t dst = sbase + (is_k ? C::kOffK : C::kOffV) + sl * C::kTileBytes;
+      if (elect_one()) {
         mbar_expect_tx(full, C::kTileBytes);
 #pragma unroll
         for (int b = 0; b < D / 64; ++b) tma_load_3d(dst + b * C::kBoxKBytes, m, full, 64 * b, row, bh);
-        return true;
-      };
-      // K runs one tile ahead of V: K_t is due at S_t, V_t only after softmax_t
-      for (int t = 0; ok && t <= T; ++t) {
-        if (misc[1]) { ok = false; break; }
-        if (t < T) {
-          if (!load(t, true)) { ok = false; break; }
-          k_issued = t + 1;
-        }
-        if (t >= 1) {
-          if (!load(t - 1, false)) { ok = false; break; }
-          v_issued = t;
-        }
       }
-      if (ok && hyd) {
-        // Hbar goes into the K ring once every S = Q K^T has completed
-        for (int u = (T >= C::kKStages ? T - C::kKStages : 0); ok && u < T; ++u)
-          ok = mbar_wait(bar(C::kBarKEmpty + u % C::kKStages), (u / C::kKStages) & 1);
-        if (ok) {
+      __syncwarp();
+      return true;
+    };
+    // K runs one tile ahead of V: K_t is due at S_t, V_t only after softmax_t
+    for (int t = 0; ok && t <= T; ++t) {
+      if (aborted()) { ok = false; break; }
+      if (t < T) {
+        if (!load(t, true)) { ok = false; break; }
+        k_issued = t + 1;
+      }
+      if (t >= 1) {
+        if (!load(t - 1, false)) { ok = false; break; }
+        v_issued = t;
+      }
+    }
+    if (ok && hyd) {
+      // Hbar goes into the K ring once every S = Q K^T has completed
+      for (int u = (T >= C::kKStages ? T - C::kKStages : 0); ok && u < T; ++u)
+        ok = uwait(bar(C::kBarKEmpty + u % C::kKStages), (u / C::kKStages) & 1);
+      if (ok) {
+        if (elect_one()) {
           mbar_expect_tx(bar(C::kBarHFull), C::kHbarBytes);
 #pragma unroll
           for (int b = 0; b < D / 64; ++b)
             tma_load_3d(sbase + C::kOffK + b * (D * 128), &tm_hbar, bar(C::kBarHFull), 64 * b, 0, bh);
-          h_issued = true;
         }
+        __syncwarp();
+        h_issued = true;
       }
-      if (!ok) {
-        misc[1] = 1;
-        // let the copies already in flight land before the CTA exits
-        mbar_wait(bar(C::kBarQ), 0);
-        for (int t = k_issued - C::kKStages; t < k_issued; ++t)
-          if (t >= 0) mbar_wait(bar(C::kBarKFull + t % C::kKStages), (t / C::kKStages) & 1);
-        for (int t = v_issued - C::kVStages; t < v_issued; ++t)
-          if (t >= 0) mbar_wait(bar(C::kBarVFull + t % C::kVStages), (t / C::kVStages) & 1);
-        if (h_issued) mbar_wait(bar(C::kBarHFull), 0);
-      }
+    }
+    if (!ok) {
+      misc[1] = 1;
+      // let the copies already in flight land before the CTA exits
+      uwait(bar(C::kBarQ), 0);
+      for (int t = k_issued - C::kKStages; t < k_issued; ++t)
+        if (t >= 0) uwait(bar(C::kBarKFull + t % C::kKStages), (t / C::kKStages) & 1);
+      for (int t = v_issued - C::kVStages; t < v_issued; ++t)
+        if (t >= 0) uwait(bar(C::kBarVFull + t % C::kVStages), (t / C::kVStages) & 1);
+      if (h_issued) uwait(bar(C::kBarHFull), 0);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================================
-    if (lane == 0) {
-      constexpr uint32_t kIdQK = idesc_bf16_f32(128, 64, 0, 0);
-      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
-      bool ok = mbar_wait(bar(C::kBarQ), 0);
+    constexpr uint32_t kIdQK = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+    bool ok = uwait(bar(C::kBarQ), 0);
+    tc_fence_after();
+    auto q_desc = [&](int k) -> uint64_t {
+      return smem_desc_sw128(sbase + C::kOffQ + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
+    };
+    auto issue_pv = [&](int u) -> bool {
+      const int bu = u & 1, sv = u % C::kVStages;
+      if (!uwait(bar(C::kBarPFull + bu), (u >> 1) & 1)) return false;
+      if (!uwait(bar(C::kBarVFull + sv), (u / C::kVStages) & 1)) return false;
       tc_fence_after();
-      auto q_desc = [&](int k) -> uint64_t {
-        return smem_desc_sw128(sbase + C::kOffQ + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
-      };
-      auto issue_pv = [&](int u) -> bool {
-        const int bu = u & 1, sv = u % C::kVStages;
-        if (!mbar_wait(bar(C::kBarPFull + bu), (u >> 1) & 1)) return false;
-        if (!mbar_wait(bar(C::kBarVFull + sv), (u / C::kVStages) & 1)) return false;
-        tc_fence_after();
-        const uint32_t vst = sbase + C::kOffV + sv * C::kTileBytes;
+      const uint32_t vst = sbase + C::kOffV + sv * C::kTileBytes;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tmem + C::kColO, tmem + C::kColS + 64 * bu + kk * 8,
@@ -318,14 +335,17 @@ __global__ void __launch_bounds__(192, 2)
                  (u > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(C::kBarVEmpty + sv));
         tc_commit(bar(C::kBarODone));
-        return true;
-      };
-      for (int t = 0; ok && t < T; ++t) {
-        if (misc[1]) { ok = false; break; }
-        const int sk = t % C::kKStages, b = t & 1;
-        if (!mbar_wait(bar(C::kBarKFull + sk), (t / C::kKStages) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kst = sbase + C::kOffK + sk * C::kTileBytes;
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int t = 0; ok && t < T; ++t) {
+      if (aborted()) { ok = false; break; }
+      const int sk = t % C::kKStages, b = t & 1;
+      if (!uwait(bar(C::kBarKFull + sk), (t / C::kKStages) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t kst = sbase + C::kOffK + sk * C::kTileBytes;
+      if (elect_one()) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem + C::kColS + 64 * b, q_desc(k),
@@ -333,29 +353,37 @@ __global__ void __launch_bounds__(192, 2)
                  k > 0 ? 1u : 0u);
         tc_commit(bar(C::kBarSFull + b));
         tc_commit(bar(C::kBarKEmpty + sk));
-        if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
       }
-      if (ok && T >= 1) ok = issue_pv(T - 1);
-      if (ok && !hyd) tc_commit(bar(C::kBarFinal));
-      if (ok && hyd) {
-        if (mbar_wait(bar(C::kBarHFull), 0)) {
-          tc_fence_after();
-          const uint32_t hst = sbase + C::kOffK;
+      __syncwarp();
+      if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+    }
+    if (ok && T >= 1) ok = issue_pv(T - 1);
+    if (ok && !hyd) {
+      if (elect_one()) tc_commit(bar(C::kBarFinal));
+      __syncwarp();
+    }
+    if (ok && hyd) {
+      if (uwait(bar(C::kBarHFull), 0)) {
+        tc_fence_after();
+        const uint32_t hst = sbase + C::kOffK;
+        if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             mma_ss(tmem + C::kColQH, q_desc(k), smem_desc_sw128(hst + k * 2048, D * 128, 1024),
                    kIdPV, k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarFinal));
-        } else {
-          ok = false;
         }
+        __syncwarp();
+      } else {
+        ok = false;
       }
-      if (!ok) {
-        misc[1] = 1;
-        // every MMA issued so far must finish before TMEM is released
-        tc_commit(bar(C::kBarTeardown));
-        mbar_wait(bar(C::kBarTeardown), 0);
-      }
+    }
+    if (!ok) {
+      misc[1] = 1;
+      // every MMA issued so far must finish before TMEM is released
+      if (elect_one()) tc_commit(bar(C::kBarTeardown));
+      __syncwarp();
+      uwait(bar(C::kBarTeardown), 0);
     }
   } else {
     // ======================= softmax warps ====================================
