@@ -48,8 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the fused attention kernel, from an ncu capture,
 # keyed by the sha1 of the kernel source it was taken on (see profiles/).
 K3_TRAFFIC = {
-    # warp-MMA kernel, Wan-like H=4 capture (302.8 MB) scaled by heads to H=40
-    "0c3ca42da25c": {"wan": 3.028e9},
+    # tcgen05 kernel, Wan-like H=4 ncu capture (303.2 MB read+write) scaled by heads
+    "8de7c1645474": {"wan": 3.032e9},
 }
 
 
