@@ -276,6 +276,21 @@ def oracle_sample(wl, n_heads: int, n_blocks: int, seed: int = 7):
 # arms
 # ----------------------------------------------------------------------------
 
+def max_over_ranks(values, world: int, device="cpu"):
+    """Element-wise maximum of per-rank timings (ms) over all ranks (the slowest
+    rank defines the step time); a no-op with one rank."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_value(world: int, flops_per_rank: float, t_ms: float) -> float:
+    """Whole-job throughput in TFLOP/s: every rank processed its own problem of
+    `flops_per_rank` within the max-over-ranks time `t_ms`."""
+    return world * flops_per_rank / (t_ms * 1e-3) / 1e12
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -466,12 +481,10 @@ def run_pisa(args, wl):
         del dq, dk, dv, do
 
     # ---- max over ranks --------------------------------------------------------
-    t_vec = torch.tensor([t_step, part_ms["sparse_attention"],
-                          e2e["t_ms"] if e2e else 0.0], dtype=torch.float64, device=dev)
+    t_step, t_k3, t_e2e = max_over_ranks(
+        [t_step, part_ms["sparse_attention"], e2e["t_ms"] if e2e else 0.0], world, dev)
     if world > 1:
-        torch.distributed.all_reduce(t_vec, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
-    t_step, t_k3, t_e2e = (float(x) for x in t_vec.tolist())
 
     N = -(-wl.L // wl.block_size)
     k_sel = idx.shape[-1]
@@ -486,7 +499,7 @@ def run_pisa(args, wl):
     launches_per_step = 2 + (1 if want_cov else 0) + 2 + 2 + (3 if wl.dtype == "f32" else 0)
     line = {
         "metric": METRIC,
-        "value": world * dense_flops(wl) / (t_step * 1e-3) / 1e12,
+        "value": weak_scaling_value(world, dense_flops(wl), t_step),
         "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": t_step, "ms_per_call": t_step,
@@ -515,7 +528,7 @@ def run_pisa(args, wl):
     }
     line["step_roofline"]["frac"] = line["step_roofline"]["t_star_ms"] / t_step
     if e2e:
-        line["e2e"] = {"value": world * dense_flops(wl) / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
+        line["e2e"] = {"value": weak_scaling_value(world, dense_flops(wl), t_e2e), "unit": UNIT,
                        "ms_per_step": t_e2e, "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                        "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
                        "api": "pisa_attention (C ABI) from pinned host buffers"}

@@ -14,6 +14,7 @@ from .api import (  # noqa: F401
     pisa_num_blocks,
     pisa_num_selected,
     pisa_select,
+    pisa_selftest_timeout,
     pisa_sparse_attention,
     pisa_workspace_bytes,
 )

@@ -54,6 +54,7 @@ SIGNATURES = {
     "pisa_dense_attention_workspace_bytes": (_Z, [_I, _I, _I, _I, _I]),
     "pisa_block_stats_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                       _P, _P, _P, _P, _P, _P]),
+    "pisa_selftest_timeout": (_I, [ctypes.c_uint64, _P]),
     "pisa_device_status": (_I, [_P]),
     "pisa_status_string": (ctypes.c_char_p, [_I]),
     "pisa_last_error": (ctypes.c_char_p, []),

@@ -224,6 +224,12 @@ def pisa_dense_attention(q, k, v, scale: Optional[float] = None,
     return out
 
 
+def pisa_selftest_timeout(limit_ns: int = 10_000_000, stream=None) -> None:
+    """Run the bounded-wait self-test kernel (see include/pisa.h); the following
+    pisa_device_status call raises PisaError with status PISA_ERR_TIMEOUT."""
+    _check("pisa_selftest_timeout", L.load().pisa_selftest_timeout(int(limit_ns), _stream(stream)))
+
+
 def pisa_device_status(stream=None) -> None:
     """Synchronise the stream and raise if a kernel flagged a device-side error."""
     _check("pisa_device_status", L.load().pisa_device_status(_stream(stream)))

@@ -4,6 +4,7 @@
 #pragma once
 
 #include "pisa_common.cuh"
+#include "sm100_primitives.cuh"
 
 namespace pisa {
 
@@ -136,6 +137,20 @@ __global__ void pairing_kernel(const uint16_t *__restrict__ ov, int N, int stage
     __syncwarp();
     ++np;
   }
+}
+
+// Self-test of the error path of the bounded waits: one warp waits on an
+// mbarrier that nothing ever completes, with a short limit.  The wait gives up,
+// records the timeout in the device status word and the kernel returns.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t barrier;
+  const uint32_t b = smem_u32(&barrier);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncwarp();
+  sm100::mbar_wait(b, 0, limit_ns);
 }
 
 }  // namespace pisa

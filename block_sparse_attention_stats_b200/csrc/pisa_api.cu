@@ -607,6 +607,12 @@ pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v
                           partial, st);
 }
 
+pisa_status pisa_selftest_timeout(uint64_t limit_ns, pisa_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return PISA_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns);
+  return check_launch();
+}
+
 pisa_status pisa_device_status(pisa_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) {

@@ -110,12 +110,13 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // kWaitLimitNs of wall time (far beyond any legitimate wait of these kernels),
 // records a timeout in the device status word and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 0 && global_timer_ns() - t0 > limit_ns) {
       report_device_error(kDevErrTimeout);
       return false;
     }

@@ -221,6 +221,15 @@ pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v
  * PISA_ERR_CUDA if the stream itself reported an error. */
 pisa_status pisa_device_status(pisa_stream_t stream);
 
+/* Self-test of the failure path (no counterpart in the paper).  Launches one
+ * warp that waits, with the same bounded mbarrier wait every kernel of this
+ * library uses, on a barrier that nothing ever completes, giving up after
+ * limit_ns nanoseconds (1 .. 1e9).  The kernel then records PISA_ERR_TIMEOUT in
+ * the device status word and returns, so a following pisa_device_status
+ * reports PISA_ERR_TIMEOUT and the CUDA context stays usable.  No fault, trap
+ * or unbounded spin is involved. */
+pisa_status pisa_selftest_timeout(uint64_t limit_ns, pisa_stream_t stream);
+
 /* Static description of a status code. */
 const char *pisa_status_string(pisa_status s);
 

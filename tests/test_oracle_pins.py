@@ -62,7 +62,9 @@ def test_worked_example(ex):
         np.testing.assert_allclose(cov, [_ev(c) for c in ex["cov"]], rtol=1e-14, atol=1e-14)
     N = st["kbar"].shape[0]
     ksel = O.num_selected(N, ex["density"])
-    sc = O.selection_scores(st["qbar"], st["kbar"], s)
+    lam = ex["cov_weight"]
+    cov = O.covariance_norms(k, v, b, st["kbar"], st["hbar"]) if lam else None
+    sc = O.selection_scores(st["qbar"], st["kbar"], s, cov, lam)
     idx = O.select_blocks(sc, ksel, ex["sink_idx"])
     assert idx.tolist() == ex["idx"]
     for mode in ("hyd", "0th"):
@@ -71,7 +73,8 @@ def test_worked_example(ex):
             continue
         o = O.piecewise_attention(q, k, v, b, idx, st, s, mode)
         np.testing.assert_allclose(o, _arr(ex[key]), rtol=1e-13, atol=1e-13)
-        r = O.pisa_attention_head(q, k, v, b, ex["density"], ex["sink_idx"], mode, scale=s)
+        r = O.pisa_attention_head(q, k, v, b, ex["density"], ex["sink_idx"], mode, scale=s,
+                                  cov_weight=lam)
         np.testing.assert_allclose(r["out"], _arr(ex[key]), rtol=1e-13, atol=1e-13)
 
 
