@@ -80,8 +80,11 @@ def dense_flops(wl):
 
 
 def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
-    """4d sum_i n_i sum_{S_i} n_j + 4d sum_i n_i |U_i| + [hyd] 2 L d^2, per head, summed."""
+    """4d sum_i n_i sum_{S_i} n_j + 4d sum_i n_i |U_i| + [hyd] 2 L d^2, per head, summed.
+    Mode 1st reads every key of every unselected block as well: 4d L^2 per head."""
     b, L, d = wl.block_size, wl.L, wl.d
+    if wl.mode == "1st":
+        return 4.0 * d * L * L * wl.B * wl.H
     N = -(-L // b)
     k_sel = idx.shape[-1]
     n_last = L - (N - 1) * b
@@ -130,6 +133,8 @@ def k3_executed_flops(wl, idx: torch.Tensor, heads: int = 2) -> float:
     `heads` heads and scaled to all heads."""
     b, d = wl.block_size, wl.d
     N = -(-wl.L // b)
+    if wl.mode == "1st":   # every block of every pair
+        return 4.0 * d * 128 * 64 * N * (-(-N // 2)) * wl.B * wl.H
     nch = -(-N // 64)
     tile = 4.0 * d * 128 * 64
     tot = 0.0

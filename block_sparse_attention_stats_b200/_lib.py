@@ -21,6 +21,7 @@ PISA_ERR_DEVICE = 6
 
 PISA_MODE_HYD = 0
 PISA_MODE_0TH = 1
+PISA_MODE_1ST = 2
 PISA_BF16 = 0
 PISA_F32 = 1
 PISA_SINK_NONE = -(2 ** 31)

@@ -16,7 +16,7 @@ import torch
 from . import _lib as L
 
 _DT = {torch.bfloat16: L.PISA_BF16, torch.float32: L.PISA_F32}
-_MODE = {"hyd": L.PISA_MODE_HYD, "0th": L.PISA_MODE_0TH}
+_MODE = {"hyd": L.PISA_MODE_HYD, "0th": L.PISA_MODE_0TH, "1st": L.PISA_MODE_1ST}
 
 
 class PisaError(RuntimeError):

@@ -104,8 +104,8 @@ __global__ void __launch_bounds__(192, 2)
                                   const __grid_constant__ CUtensorMap tm_hbar,
                                   const int32_t *__restrict__ idx,
                                   const int2 *__restrict__ pairs, int k_sel, int L, int N,
-                                  float scale, int hyd, int dense, void *__restrict__ out,
-                                  int out_f32) {
+                                  float scale, int hyd, int dense, int blockwise,
+                                  void *__restrict__ out, int out_f32) {
   using C = TcCfg<D>;
   using namespace sm100;
   extern __shared__ unsigned char smem_raw[];
@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(192, 2)
     for (int w0 = 0; w0 < nwords; w0 += 32) {
       const int w = w0 + lane;
       const uint32_t lo = w < nwords ? bm_lo[w] : 0u, hi = w < nwords ? bm_hi[w] : 0u;
-      uint32_t u = lo | hi;
+      // block-wise first order visits every block (Taylor weights where unselected)
+      uint32_t u = blockwise ? (w < nwords ? valid_bits(w, N) : 0u) : (lo | hi);
       const int cnt = __popc(u);
       int incl = cnt;
 #pragma unroll
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(192, 2)
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
     // centroid chunks that hold an unselected block for either half
-    if (!dense) {
+    if (!dense && !blockwise) {
       const int nch = (N + 63) / 64;
       for (int c0 = 0; c0 < nch; c0 += 32) {
         const int c = c0 + lane;
@@ -410,10 +411,13 @@ __global__ void __launch_bounds__(192, 2)
       const bool centroid = e < 0;
       uint64_t cmask = 0;
       bool active;
+      // block-wise first order: an unselected block enters through its own
+      // first-order Taylor expansion about its centroid
+      const bool taylor = blockwise && exists && !centroid && ((e >> half) & 1) == 0;
       if (!exists) {
         active = false;
       } else if (!centroid) {
-        active = ((e >> half) & 1) != 0;
+        active = ((e >> half) & 1) != 0 || taylor;
       } else {
         const int c = -e - 1;
         const uint32_t m0 = ~bm[2 * c] & valid_bits(2 * c, N);
@@ -425,6 +429,8 @@ __global__ void __launch_bounds__(192, 2)
       float tmax = -INFINITY;
       const uint32_t s_addr = lane_addr + C::kColS + 64 * b;
       uint32_t pk[32];
+      float taylor_ell = 0.f;
+      int taylor_nj = 0;
       if (active) {
         uint32_t r0[32], r1[32];
         tmem_ld_x32(s_addr, r0);
@@ -440,7 +446,23 @@ __global__ void __launch_bounds__(192, 2)
         uint64_t keep = ~0ull;
         if (centroid) keep = cmask;
         else if ((e >> 2) == N - 1 && n_last < 64) keep = (1ull << n_last) - 1ull;
-        if (keep != ~0ull) {
+        if (taylor) {
+          // alpha = exp(s q kbar_j) with s q kbar_j = mean of the exact logits of
+          // the block; weights alpha (1 + s q k_n - s q kbar_j); D gains alpha n_j
+          const int nj = popcount64(keep);
+          float acc8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc8[i] = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) acc8[i & 7] += ((keep >> i) & 1ull) ? sv[i] : 0.f;
+          const float sum = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
+                            ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+          const float mean = sum / (float)nj;
+          taylor_ell = mean;
+          taylor_nj = nj;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) sv[i] = ((keep >> i) & 1ull) ? sv[i] : 0.f;
+        } else if (keep != ~0ull) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) sv[i] = ((keep >> i) & 1ull) ? sv[i] : -INFINITY;
         }
@@ -456,6 +478,7 @@ __global__ void __launch_bounds__(192, 2)
           for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], sv[i + 56]);
           tmax = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         }
+        if (taylor) tmax = taylor_ell;
         const float m_t = tmax * sl2;                  // finite: the row has a key here
         const bool grow = m_t > m_run + 8.0f;          // lazy rescale threshold 2^8
         const bool need_o = grow && m_run != -INFINITY;
@@ -480,6 +503,16 @@ __global__ void __launch_bounds__(192, 2)
           l_run *= f;
           a_run *= f;
         }
+        if (taylor) {
+          const float alpha = ex2_approx(fmaf(taylor_ell, sl2, -m_run));
+          const float c1 = alpha * scale, c0 = alpha * (1.f - scale * taylor_ell);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const bool k0 = (keep >> (2 * i)) & 1ull, k1 = (keep >> (2 * i + 1)) & 1ull;
+            pk[i] = pack_bf16x2(k0 ? fmaf(sv[2 * i], c1, c0) : 0.f, k1 ? fmaf(sv[2 * i + 1], c1, c0) : 0.f);
+          }
+          l_run += alpha * (float)taylor_nj;
+        } else {
         const float neg = -m_run;
         const float2 sl2x2 = make_float2(sl2, sl2), neg2 = make_float2(neg, neg);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -507,6 +540,7 @@ __global__ void __launch_bounds__(192, 2)
         } else {
           l_run += ps;
         }
+        }  // exponential weights
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = 0u;

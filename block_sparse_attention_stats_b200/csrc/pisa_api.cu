@@ -243,8 +243,8 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
                                            const __nv_bfloat16 *vsum16,
                                            const __nv_bfloat16 *hbar16, const int32_t *idx,
                                            const int2 *pairs, int k_sel, int BH, int L,
-                                           float scale, int hyd, int dense, void *out,
-                                           int out_f32, cudaStream_t st) {
+                                           float scale, int hyd, int dense, int blockwise,
+                                           void *out, int out_f32, cudaStream_t st) {
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
   const int smem = TcCfg<D>::smem_bytes(N);
   if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
@@ -264,7 +264,7 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
   PISA_CUDA(cudaFuncSetAttribute(piecewise_attention_tc_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   piecewise_attention_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), TcCfg<D>::kThreads, smem, st>>>(
-      mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, scale, hyd, dense, out, out_f32);
+      mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, scale, hyd, dense, blockwise, out, out_f32);
   return check_launch();
 }
 
@@ -317,12 +317,13 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
     v16 = c;
   }
   const int hyd = mode == PISA_MODE_HYD;
+  const int blockwise = mode == PISA_MODE_1ST;
   const int of32 = dt == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel,
-                                        BH, L, scale, hyd, 0, out, of32, st);
+                                        BH, L, scale, hyd, 0, blockwise, out, of32, st);
   return launch_attention_kernel<64>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel, BH,
-                                     L, scale, hyd, 0, out, of32, st);
+                                     L, scale, hyd, 0, blockwise, out, of32, st);
 }
 
 }  // namespace pisa
@@ -454,7 +455,7 @@ pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, p
                                   void *workspace, size_t ws_bytes, pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, block_size));
   if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
-  if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH) return PISA_ERR_INVALID_ARG;
+  if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH && mode != PISA_MODE_1ST) return PISA_ERR_INVALID_ARG;
   const int N = ceil_div(L, 64);
   if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
@@ -476,7 +477,7 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
   if (opts) o = *opts;
   PISA_TRY(check_shape(B, H, L, d, block_size));
   if (o.dtype != PISA_BF16 && o.dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
-  if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH) return PISA_ERR_INVALID_ARG;
+  if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH && mode != PISA_MODE_1ST) return PISA_ERR_INVALID_ARG;
   if (!sink_valid(sink_idx)) return PISA_ERR_INVALID_ARG;
   if (!(o.scale >= 0.f) || !std::isfinite(o.scale) || !std::isfinite(o.cov_weight))
     return PISA_ERR_INVALID_ARG;
@@ -573,9 +574,9 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
   const int of32 = dtype == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr,
-                                        nullptr, 0, BH, L, s, 0, 1, out, of32, st);
+                                        nullptr, 0, BH, L, s, 0, 1, 0, out, of32, st);
   return launch_attention_kernel<64>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                     0, BH, L, s, 0, 1, out, of32, st);
+                                     0, BH, L, s, 0, 1, 0, out, of32, st);
 }
 
 pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v,

@@ -61,7 +61,13 @@ typedef enum {
 
 typedef enum {
   PISA_MODE_HYD = 0, /* zeroth-order tail + global first-order term ("_hyd") */
-  PISA_MODE_0TH = 1  /* zeroth-order tail only ("_0th") */
+  PISA_MODE_0TH = 1, /* zeroth-order tail only ("_0th") */
+  PISA_MODE_1ST = 2  /* block-wise first order: every unselected block j adds
+                        alpha_tj (s q_t H_j) with its own H_j (the gist.science
+                        summary, "Global First-Order Correction": the per-block
+                        alternative to Hbar; atlas.scime.ai "Surprising findings":
+                        the "first-order-only" ablation).  Work equals dense
+                        attention: every K/V block is read. */
 } pisa_mode;
 
 typedef enum { PISA_BF16 = 0, PISA_F32 = 1 } pisa_dtype;
@@ -138,6 +144,8 @@ pisa_status pisa_select(const float *qbar, const float *kbar, const float *cov,
  *   D_t = sum_{j in S_i} sum_n e^{s q_t k_{j,n}} + sum_{j in U_i} n_j alpha_tj
  *   N_t = sum_{j in S_i} sum_n e^{s q_t k_{j,n}} v_{j,n} + sum_{j in U_i} alpha_tj vsum_j
  *         + [hyd] (s q_t hbar) sum_{j in U_i} alpha_tj,     alpha_tj = e^{s q_t kbar_j}
+ *         + [1st] sum_{j in U_i} alpha_tj (s q_t H_j)  (computed per token as
+ *           sum_n alpha_tj (s q_t k_{j,n} - s q_t kbar_j) v_{j,n}; hbar unused)
  *   out_t = N_t / D_t
  * with S_i = idx row i (k_sel ascending, distinct indices < N) and U_i its
  * complement.  kbar, vsum, hbar as written by pisa_block_stats.  out

@@ -29,6 +29,9 @@ Sources (cited by page title and section):
   every query block; density, block_size arguments).
 * [SK] "Pisa Sparse Attention" (skillmd.com agent skill), "Implementation":
   the covariance weight 0.1 and the Frobenius norm of the covariance term.
+* [AT] atlas.scime.ai summary, "Surprising findings": the "first-order-only"
+  variant, and [GS] "Global First-Order Correction": a distinct first-order
+  term for every unselected block (memory-bound) -- mode "1st" below.
 
 Readings where the pages are silent (each one is listed in the design doc):
 
@@ -199,14 +202,16 @@ def piecewise_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, block_size:
       N_t = sum_{j in S_i} sum_n exp(s q_t k_{j,n}) v_{j,n}
             + sum_{j in U_i} alpha_{t,j} vsum_j
             + [mode hyd] (s q_t Hbar) sum_{j in U_i} alpha_{t,j}
+            + [mode 1st] sum_{j in U_i} alpha_{t,j} (s q_t H_j)
       alpha_{t,j} = exp(s q_t kbar_j)
+    Mode "1st" (block-wise first order) needs stats["H"], the per-block H_j.
     One per-row constant (the row maximum of all exponents) is factored out of
     N_t and D_t to keep exp() in range; it cancels in the quotient.
 
     Returns an array [L, d] with rows of the requested blocks filled (NaN elsewhere).
     """
-    if mode not in ("hyd", "0th"):
-        raise ValueError("mode must be 'hyd' or '0th'")
+    if mode not in ("hyd", "0th", "1st"):
+        raise ValueError("mode must be 'hyd', '0th' or '1st'")
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -236,6 +241,10 @@ def piecewise_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, block_size:
         Nt = p_exact @ v[ex] + alpha @ vsum[U]
         if mode == "hyd":
             Nt = Nt + (scale * (qi @ hbar)) * alpha.sum(axis=1)[:, None]
+        elif mode == "1st" and U.size:
+            # sum_j alpha_tj H_j as one product, then contract with s q_t
+            W = (alpha @ stats["H"][U].reshape(U.size, d * d)).reshape(-1, d, d)
+            Nt = Nt + scale * np.einsum("ta,tab->tb", qi, W)
         out[rows] = Nt / D[:, None]
     return out
 
@@ -269,7 +278,7 @@ def pisa_attention_head(q, k, v, block_size: int, density: float,
     q = np.asarray(q, dtype=np.float64)
     L, d = q.shape
     s = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    st = block_stats(q, k, v, block_size)
+    st = block_stats(q, k, v, block_size, keep_blockwise=(mode == "1st"))
     N = st["kbar"].shape[0]
     cov = None
     if cov_weight != 0.0:

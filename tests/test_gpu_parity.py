@@ -97,6 +97,16 @@ def test_ragged_and_degenerate(P, L, sink, mode, d):
     assert _run_case(P, wl) == 0
 
 
+@pytest.mark.parametrize("L,d,sink,cov", [(4608, 128, -1, 0.1), (1000, 128, None, 0.0),
+                                          (777, 64, 0, 0.0)])
+def test_blockwise_first_order(P, L, d, sink, cov):
+    """Mode 1st: every unselected block through its own first-order expansion
+    (linear values make the H_j large and distinct)."""
+    wl = WORKLOADS["flux"].with_(H=2, L=L, d=d, sink_idx=sink, cov_weight=cov, mode="1st",
+                                 cluster_kind="image" if L == 4608 else "block")
+    assert _run_case(P, wl, value_mode="linear") == 0
+
+
 def test_linear_values_first_order_visible(P):
     """V = K W + noise makes Hbar large, so the hyd term is exercised."""
     wl = WORKLOADS["flux"].with_(H=2, L=2048, cluster_kind="block", cov_weight=0.0,

@@ -53,7 +53,7 @@ with open(GOLDEN) as f:
 def test_worked_example(ex):
     q, k, v = (np.array(ex[n], dtype=np.float64) for n in ("q", "k", "v"))
     b, s = ex["block_size"], ex["scale"]
-    st = O.block_stats(q, k, v, b)
+    st = O.block_stats(q, k, v, b, keep_blockwise=True)
     for key in ("qbar", "kbar", "vsum", "hbar"):
         if key in ex:
             np.testing.assert_allclose(st[key], _arr(ex[key]), rtol=0, atol=1e-14)
@@ -67,7 +67,7 @@ def test_worked_example(ex):
     sc = O.selection_scores(st["qbar"], st["kbar"], s, cov, lam)
     idx = O.select_blocks(sc, ksel, ex["sink_idx"])
     assert idx.tolist() == ex["idx"]
-    for mode in ("hyd", "0th"):
+    for mode in ("hyd", "0th", "1st"):
         key = "o_" + mode
         if key not in ex:
             continue
@@ -223,6 +223,49 @@ def test_taylor_order_of_hybrid_and_zeroth():
         assert 3.4 < a["hyd"] / c["hyd"] < 4.6
         assert 1.7 < a["0th"] / c["0th"] < 2.3
     assert e3["hyd"] < 0.05 * e3["0th"]
+
+
+def test_blockwise_first_order_is_second_order_accurate():
+    """Keys k_{j,n} = kbar_j + eps delta_{j,n} with DIFFERENT deviations and
+    values per block (H_j all differ): the block-wise first-order tail is the
+    exact first-order expansion of every unselected block (error O(eps^2)),
+    while the hybrid (shared Hbar) and zeroth-order tails are O(eps)."""
+    b, N, d = 4, 8, 4
+    L = b * N
+    rng = np.random.default_rng(38)
+    kbar = rng.standard_normal((N, d))
+    delta = rng.standard_normal((N, b, d))
+    delta -= delta.mean(axis=1, keepdims=True)
+    q = rng.standard_normal((L, d))
+    v = rng.standard_normal((L, d))
+
+    def errs(eps):
+        k = (kbar[:, None, :] + eps * delta).reshape(L, d)
+        ref = _sdpa(q, k, v, 1 / math.sqrt(d))
+        return {m: np.abs(O.pisa_attention_head(q, k, v, b, 0.25, None, m)["out"] - ref).max()
+                for m in ("1st", "hyd", "0th")}
+
+    e1, e2, e3 = errs(0.02), errs(0.01), errs(0.005)
+    for a, c in ((e1, e2), (e2, e3)):
+        assert 3.4 < a["1st"] / c["1st"] < 4.6
+        assert 1.7 < a["hyd"] / c["hyd"] < 2.3
+    assert e3["1st"] < 0.05 * e3["hyd"]
+
+
+def test_blockwise_first_order_equals_hybrid_when_blocks_share_H():
+    """Same deviations and values in every block: H_j = Hbar, so the two
+    first-order variants coincide."""
+    b, N, d = 4, 6, 3
+    L = b * N
+    rng = np.random.default_rng(39)
+    delta = rng.standard_normal((b, d))
+    delta -= delta.mean(0)
+    k = (rng.standard_normal((N, 1, d)) + 0.3 * delta[None]).reshape(L, d)
+    v = np.tile(rng.standard_normal((b, d)), (N, 1))
+    q = rng.standard_normal((L, d))
+    h = O.pisa_attention_head(q, k, v, b, 0.34, -1, "hyd")["out"]
+    f = O.pisa_attention_head(q, k, v, b, 0.34, -1, "1st")["out"]
+    np.testing.assert_allclose(f, h, rtol=1e-12, atol=1e-12)
 
 
 # ----------------------------------------------------------------------------

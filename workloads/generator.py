@@ -170,7 +170,7 @@ class Workload:
     d: int
     block_size: int
     density: float
-    mode: str                      # "hyd" or "0th"
+    mode: str                      # "hyd", "0th" or "1st" (block-wise first order)
     sink_idx: Optional[int]        # None, 0 or -1
     dtype: str                     # "bf16" or "f32"
     cov_weight: float              # lambda of covariance-aware scoring (0 = off)
@@ -207,6 +207,10 @@ WORKLOADS = {
                          density=0.15, mode="0th", sink_idx=-1, dtype="bf16",
                          cov_weight=0.1, cluster_kind="image", seed=DEFAULT_SEED + 3,
                          densities=(0.05, 0.10, 0.15, 0.25, 1.0)),
+    # the same FLUX shape with the block-wise first-order tail ("first-order-only")
+    "flux_1st": Workload("flux_1st", B=1, H=24, L=4608, d=128, block_size=64, density=0.15,
+                         mode="1st", sink_idx=-1, dtype="bf16", cov_weight=0.1,
+                         cluster_kind="image", seed=DEFAULT_SEED + 2),
     # Wan2.1-14B 720p-ish latent video: 21 frames x 45 x 80
     "wan": Workload("wan", B=1, H=40, L=75600, d=128, block_size=64, density=0.125,
                     mode="hyd", sink_idx=None, dtype="bf16", cov_weight=0.0,
