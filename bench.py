@@ -451,6 +451,29 @@ def run_pisa(args, wl):
         dense = {"ms": dms, "tflops": dense_flops(wl) / (dms * 1e-3) / 1e12,
                  "kernel": "pisa_dense_attention (all blocks exact, same kernel family)"}
 
+    # ---- distributional-stability diagnostic over the step's own selection -------
+    diag = None
+    if not args.no_diagnostic:
+        qs = 8 if wl.L > 20000 else 1
+        lo, hi, nb = -8.0, 8.0, 64
+        P.pisa_tail_score_histogram(Q, K, idx, lo, hi, nb, wl.block_size, query_stride=qs)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        r = P.pisa_tail_score_histogram(Q, K, idx, lo, hi, nb, wl.block_size, query_stride=qs)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        hx, hy = r["hist_x"].cpu(), r["hist_y"].cpu()
+        n = max(r["n"], 1.0)
+        centre = 1 + nb // 2                      # first bin at or above 0
+        diag = {"query_stride": qs, "scores": int(r["n"]), "ms": e0.elapsed_time(e1),
+                "mean_x": r["mean_x"], "sd_x": math.sqrt(max(r["var_x"], 0.0)),
+                "frac_x_below_0": float(hx[:centre].sum()) / n,
+                "mean_y": r["mean_y"], "sd_y": math.sqrt(max(r["var_y"], 0.0)),
+                "frac_abs_y_above_1": float(hy[:centre - nb // 16].sum()
+                                            + hy[centre + nb // 16:].sum()) / n,
+                "range": [lo, hi], "nbins": nb}
+
     # ---- e2e: public API with pinned host buffers ------------------------------
     e2e = None
     if not args.no_e2e:
@@ -528,6 +551,7 @@ def run_pisa(args, wl):
                                    / (peaks.get("hbm_gbs", 6650.0) * 1e9)),
         },
         "dense_baseline": dense,
+        "tail_diagnostic": diag,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -561,6 +585,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-diagnostic", action="store_true",
+                    help="skip the histogram of the unselected blocks' scores")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (small cases for profiling only)")
     args = ap.parse_args()

@@ -16,5 +16,6 @@ from .api import (  # noqa: F401
     pisa_select,
     pisa_selftest_timeout,
     pisa_sparse_attention,
+    pisa_tail_score_histogram,
     pisa_workspace_bytes,
 )

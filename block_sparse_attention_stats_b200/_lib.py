@@ -56,6 +56,8 @@ SIGNATURES = {
     "pisa_block_stats_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                       _P, _P, _P, _P, _P, _P]),
     "pisa_selftest_timeout": (_I, [ctypes.c_uint64, _P]),
+    "pisa_tail_score_histogram": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _F, _F, _I,
+                                       _I, _P, _P, _P, _P]),
     "pisa_device_status": (_I, [_P]),
     "pisa_status_string": (ctypes.c_char_p, [_I]),
     "pisa_last_error": (ctypes.c_char_p, []),

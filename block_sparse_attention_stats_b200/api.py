@@ -224,6 +224,30 @@ def pisa_dense_attention(q, k, v, scale: Optional[float] = None,
     return out
 
 
+def pisa_tail_score_histogram(q, k, idx, lo: float = -8.0, hi: float = 8.0, nbins: int = 64,
+                              block_size: int = 64, scale: Optional[float] = None,
+                              query_stride: int = 1, stream=None):
+    """Histograms of the pre-softmax scores x = s q k of the unselected blocks and
+    of their deviation y = s q (k - kbar_j) from the block-centroid score; returns
+    dict(hist_x, hist_y [nbins + 2] int64 with under/overflow bins, n, mean_x,
+    var_x, mean_y, var_y, edges)."""
+    lib = L.load()
+    B, H, Ln, d = q.shape
+    hx = torch.empty(nbins + 2, dtype=torch.int64, device=q.device)
+    hy = torch.empty(nbins + 2, dtype=torch.int64, device=q.device)
+    mom = torch.empty(5, dtype=torch.float64, device=q.device)
+    _check("pisa_tail_score_histogram", lib.pisa_tail_score_histogram(
+        _ptr(q), _ptr(k), _DT[q.dtype], _ptr(idx), idx.shape[-1], B, H, Ln, d, block_size,
+        0.0 if scale is None else float(scale), float(lo), float(hi), int(nbins),
+        int(query_stride), _ptr(hx), _ptr(hy), _ptr(mom), _stream(stream)))
+    m = mom.cpu().tolist()
+    n = max(m[0], 1.0)
+    return dict(hist_x=hx, hist_y=hy, n=m[0], sum_x=m[1], sum_x2=m[2], sum_y=m[3], sum_y2=m[4],
+                mean_x=m[1] / n, var_x=m[2] / n - (m[1] / n) ** 2,
+                mean_y=m[3] / n, var_y=m[4] / n - (m[3] / n) ** 2,
+                edges=torch.linspace(lo, hi, nbins + 1))
+
+
 def pisa_selftest_timeout(limit_ns: int = 10_000_000, stream=None) -> None:
     """Run the bounded-wait self-test kernel (see include/pisa.h); the following
     pisa_device_status call raises PisaError with status PISA_ERR_TIMEOUT."""

@@ -16,6 +16,7 @@
 #include "k2_select.cuh"
 #include "k3_pack.cuh"
 #include "k3_attention_tc.cuh"
+#include "k5_tail_histogram.cuh"
 
 namespace pisa {
 
@@ -606,6 +607,45 @@ pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v
                              partial, st);
   return launch_stats<64>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
                           partial, st);
+}
+
+pisa_status pisa_tail_score_histogram(const void *q, const void *k, pisa_dtype dtype,
+                                      const int32_t *idx, int k_sel, int B, int H, int L, int d,
+                                      int block_size, float scale, float lo, float hi, int nbins,
+                                      int query_stride, unsigned long long *hist_x,
+                                      unsigned long long *hist_y, double *moments,
+                                      pisa_stream_t stream) {
+  PISA_TRY(check_shape(B, H, L, d, block_size));
+  if (dtype != PISA_BF16) return PISA_ERR_UNSUPPORTED;
+  const int N = ceil_div(L, 64);
+  if (k_sel < 1 || k_sel > N || nbins < 1 || nbins > 4096 || query_stride < 1)
+    return PISA_ERR_INVALID_ARG;
+  if (!std::isfinite(lo) || !std::isfinite(hi) || !(lo < hi) || !(scale >= 0.f) ||
+      !std::isfinite(scale))
+    return PISA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !idx || !hist_x || !hist_y || !moments)
+    return PISA_ERR_INVALID_ARG;
+  const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
+  cudaStream_t st = (cudaStream_t)stream;
+  PISA_CUDA(cudaMemsetAsync(hist_x, 0, sizeof(unsigned long long) * (nbins + 2), st));
+  PISA_CUDA(cudaMemsetAsync(hist_y, 0, sizeof(unsigned long long) * (nbins + 2), st));
+  PISA_CUDA(cudaMemsetAsync(moments, 0, sizeof(double) * 5, st));
+  const int smem = 3 * 64 * d * 2 + 8 * (nbins + 2) * 4 + ceil_div(N, 32) * 4;
+  if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
+  dim3 grid(ceil_div(N, query_stride), B * H);
+  const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k;
+  if (d == 128) {
+    PISA_CUDA(cudaFuncSetAttribute(tail_histogram_kernel<128>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    tail_histogram_kernel<128><<<grid, kHistThreads, smem, st>>>(
+        q16, k16, idx, k_sel, L, N, s, lo, hi, nbins, query_stride, hist_x, hist_y, moments);
+  } else {
+    PISA_CUDA(cudaFuncSetAttribute(tail_histogram_kernel<64>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    tail_histogram_kernel<64><<<grid, kHistThreads, smem, st>>>(
+        q16, k16, idx, k_sel, L, N, s, lo, hi, nbins, query_stride, hist_x, hist_y, moments);
+  }
+  return check_launch();
 }
 
 pisa_status pisa_selftest_timeout(uint64_t limit_ns, pisa_stream_t stream) {

@@ -158,6 +158,29 @@ pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v,
                                   pisa_mode mode, void *out, void *workspace,
                                   size_t ws_bytes, pisa_stream_t stream);
 
+/* ---- diagnostic ------------------------------------------------------------ */
+
+/* Distributional stability of the non-critical blocks (gist.science summary,
+ * section 2 "Key Insights" 1: their pre-softmax scores are bell-shaped and
+ * centred at or below zero, which is why their Taylor approximation is
+ * accurate).  For every token t of the query blocks i = 0, query_stride,
+ * 2 query_stride, ..., every unselected block j in U_i (idx row i gives S_i) and
+ * every key n of block j:
+ *   x = s q_t k_n               pre-softmax score
+ *   y = s q_t (k_n - kbar_j)    the variable of block j's Taylor expansion
+ * hist_x / hist_y (nbins + 2 counts each, device, zeroed here): [0] values
+ * below lo, [1 .. nbins] the equal bins of [lo, hi), [nbins + 1] values >= hi.
+ * moments (5 doubles, device, zeroed here): count, sum x, sum x^2, sum y,
+ * sum y^2.  bf16 q, k only; 1 <= nbins <= 4096.  Reads every key of every
+ * unselected block of the sampled query blocks (dense-size work when
+ * query_stride is 1). */
+pisa_status pisa_tail_score_histogram(const void *q, const void *k, pisa_dtype dtype,
+                                      const int32_t *idx, int k_sel, int B, int H, int L, int d,
+                                      int block_size, float scale, float lo, float hi, int nbins,
+                                      int query_stride, unsigned long long *hist_x,
+                                      unsigned long long *hist_y, double *moments,
+                                      pisa_stream_t stream);
+
 /* ---- the whole path ----------------------------------------------------- */
 
 /* The authors' `piecewise_sparse_attention_{hyd,0th}(q, k, v, density,

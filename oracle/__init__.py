@@ -16,4 +16,5 @@ from .pisa_oracle import (  # noqa: F401
     pisa_attention,
     selection_scores,
     select_blocks,
+    tail_score_histogram,
 )

@@ -310,3 +310,53 @@ def pisa_attention(Q, K, V, block_size: int, density: float, sink_idx: Optional[
                                     sink_idx, mode, scale, cov_weight)
             out[b, h] = r["out"]
     return out
+
+
+# ----------------------------------------------------------------------------
+# distributional-stability diagnostic ([GS] "Key Insights" 1)
+# ----------------------------------------------------------------------------
+
+def tail_score_histogram(q, k, block_size: int, selected: np.ndarray, scale: float,
+                         lo: float, hi: float, nbins: int,
+                         query_blocks: Optional[Iterable[int]] = None) -> Dict[str, np.ndarray]:
+    """Distribution of the pre-softmax scores of the unselected (non-critical)
+    blocks, and of their deviation from the block-centroid score.
+
+    For every token t of the requested query blocks i, every unselected block
+    j in U_i and every key n of block j:
+        x = s q_t k_n                     (pre-softmax score)
+        y = s q_t (k_n - kbar_j)          (the variable of the block's Taylor
+                                           expansion about its centroid)
+    Histograms over nbins equal bins of [lo, hi), with one underflow bin in
+    front and one overflow bin at the end (nbins + 2 counts each), plus the
+    count and the sums of x, x^2, y, y^2.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    L, d = q.shape
+    N, starts, counts = block_partition(L, block_size)
+    edges = np.linspace(lo, hi, nbins + 1)
+    hx = np.zeros(nbins + 2, dtype=np.int64)
+    hy = np.zeros(nbins + 2, dtype=np.int64)
+    mom = np.zeros(5)
+    blocks = range(N) if query_blocks is None else query_blocks
+
+    def add(h, vals):
+        h[0] += int((vals < lo).sum())
+        h[-1] += int((vals >= hi).sum())
+        inside = vals[(vals >= lo) & (vals < hi)]
+        h[1:-1] += np.histogram(inside, bins=edges)[0]
+
+    for i in blocks:
+        qi = q[starts[i]:starts[i] + counts[i]]
+        in_S = np.zeros(N, dtype=bool)
+        in_S[selected[i]] = True
+        for j in np.nonzero(~in_S)[0]:
+            kb = k[starts[j]:starts[j] + counts[j]]
+            x = scale * (qi @ kb.T)
+            y = scale * (qi @ (kb - kb.mean(axis=0)).T)
+            add(hx, x.ravel())
+            add(hy, y.ravel())
+            mom += [x.size, x.sum(), (x * x).sum(), y.sum(), (y * y).sum()]
+    return dict(hist_x=hx, hist_y=hy, n=mom[0], sum_x=mom[1], sum_x2=mom[2],
+                sum_y=mom[3], sum_y2=mom[4], edges=edges)

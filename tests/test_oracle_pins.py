@@ -424,3 +424,43 @@ def test_generator_is_deterministic_and_per_head():
         assert torch.equal(x, y)
     assert not torch.equal(a[0], c[0])
     assert a[0].dtype == torch.float32 and a[0].shape == (1024, 64)
+
+
+# ----------------------------------------------------------------------------
+# distributional-stability diagnostic
+# ----------------------------------------------------------------------------
+
+def test_tail_histogram_bruteforce_and_identities():
+    """Counts against a per-element loop with explicit bin arithmetic; the
+    deviations y sum to zero over each block (so their mean is 0); the total
+    count is (tokens) x (keys of unselected blocks)."""
+    L, b, d = 40, 8, 3
+    rng = np.random.default_rng(40)
+    q, k = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    s, lo, hi, nb = 0.7, -2.0, 2.0, 8
+    N = 5
+    sel = np.array([[0, 2], [1, 3], [2, 4], [0, 1], [3, 4]])
+    r = O.tail_score_histogram(q, k, b, sel, s, lo, hi, nb)
+    hx = np.zeros(nb + 2, dtype=np.int64)
+    hy = np.zeros(nb + 2, dtype=np.int64)
+    width = (hi - lo) / nb
+    n_tot = 0
+    for i in range(N):
+        for j in range(N):
+            if j in sel[i]:
+                continue
+            kb = k[j * b:(j + 1) * b]
+            cen = kb.mean(axis=0)
+            for t in range(i * b, (i + 1) * b):
+                for kn in kb:
+                    n_tot += 1
+                    for h, val in ((hx, s * q[t] @ kn), (hy, s * q[t] @ (kn - cen))):
+                        if val < lo:
+                            h[0] += 1
+                        elif val >= hi:
+                            h[-1] += 1
+                        else:
+                            h[1 + min(nb - 1, int((val - lo) // width))] += 1
+    assert (r["hist_x"] == hx).all() and (r["hist_y"] == hy).all()
+    assert r["n"] == n_tot == N * b * (N - 2) * b
+    assert abs(r["sum_y"]) < 1e-9
