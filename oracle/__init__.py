@@ -18,3 +18,4 @@ from .pisa_oracle import (  # noqa: F401
     select_blocks,
     tail_score_histogram,
 )
+from .pisa_backward import zeroth_order_backward, zeroth_order_forward  # noqa: F401
