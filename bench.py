@@ -79,6 +79,27 @@ def dense_flops(wl):
     return 4.0 * wl.B * wl.H * wl.L * wl.L * wl.d
 
 
+def bwd_flops(wl, k_sel):
+    """(algorithmic, executed) FLOPs of one zeroth-order backward.
+
+    Algorithmic: five products per (query row, key) pair of the augmented
+    softmax (recomputed logits q.k, dP = dout.value, dV += P dout, dK += dz q,
+    dQ += dz k), 2 d FLOPs each, over the exact keys of S_i and the centroids of
+    U_i.  Executed: the kernels' 64 x 64 tiles, nine products per tile pair
+    (the dq kernel forms logits and dP twice: once for Delta, once for dq), plus
+    the padding of the last block and of the 64-centroid chunks."""
+    N = -(-wl.L // wl.block_size)
+    C = -(-N // 64)
+    BH = wl.B * wl.H
+    # every query token sees k_sel exact blocks (counted as full blocks: a
+    # partial last block adds at most block_size keys per row too many) and
+    # N - k_sel centroids
+    pairs = wl.L * (k_sel * wl.block_size + (N - k_sel))
+    alg = BH * 10.0 * wl.d * pairs
+    execd = BH * 9.0 * 2 * 64 * 64 * wl.d * N * (k_sel + C)
+    return alg, execd
+
+
 def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
     """4d sum_i n_i sum_{S_i} n_j + 4d sum_i n_i |U_i| + [hyd] 2 L d^2, per head, summed.
     Mode 1st reads every key of every unselected block as well: 4d L^2 per head."""
@@ -474,6 +495,50 @@ def run_pisa(args, wl):
                                             + hy[centre + nb // 16:].sum()) / n,
                 "range": [lo, hi], "nbins": nb}
 
+    # ---- backward of the zeroth-order variant (training), same inputs -----------
+    bwd = None
+    if not args.no_backward and wl.dtype == "bf16":
+        G = torch.randn(Q.shape, generator=torch.Generator(device=dev).manual_seed(11),
+                        device=dev).to(Q.dtype)
+        lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+        P.pisa_sparse_attention_fwd(Q, K, V, stt["kbar"], stt["vsum"], stt["hbar"], idx, "0th",
+                                    wl.block_size, out=out, lse=lse, workspace=k3_ws)
+        bws = mk(lib.pisa_sparse_attention_bwd_workspace_bytes(wl.B, wl.H, wl.L, wl.d,
+                                                                wl.block_size))
+        grads = tuple(torch.empty_like(Q) for _ in range(3))
+
+        def bstep():
+            P.pisa_sparse_attention_bwd(Q, K, V, G, lse, stt["kbar"], stt["vsum"], idx,
+                                        wl.block_size, grads=grads, workspace=bws)
+
+        for _ in range(3):
+            bstep()
+        torch.cuda.synchronize()
+        reps = 3 if wl.L > 20000 else 10
+        bev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+        for r_ in range(reps):
+            if l2_flush is not None:
+                l2_flush.zero_()
+            bev[2 * r_].record(stream)
+            bstep()
+            bev[2 * r_ + 1].record(stream)
+        torch.cuda.synchronize()
+        P.pisa_device_status()
+        bms = sum(bev[2 * r_].elapsed_time(bev[2 * r_ + 1]) for r_ in range(reps)) / reps
+        f_alg_b, f_exec_b = bwd_flops(wl, idx.shape[-1])
+        pk = _peaks()[0]
+        p_sus_b = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        bwd = {"ms": bms, "mode": "0th", "launches": 5,
+               "kernels": "pack_centroids, selection_bitmap, bwd_dq (2 sweeps), "
+                          "bwd_kv<centroid>, bwd_kv<exact> (mma.sync)",
+               "roofline": {"bound": "tensor", "achieved": f_alg_b / (bms * 1e-3) / 1e12,
+                            "peak": p_sus_b, "unit": "TFLOP/s",
+                            "frac": f_alg_b / (bms * 1e-3) / 1e12 / p_sus_b,
+                            "algorithmic_tflop": f_alg_b / 1e12,
+                            "executed_tflop": f_exec_b / 1e12,
+                            "executed_frac": f_exec_b / (bms * 1e-3) / 1e12 / p_sus_b}}
+        del grads, G
+
     # ---- e2e: public API with pinned host buffers ------------------------------
     e2e = None
     if not args.no_e2e:
@@ -552,6 +617,7 @@ def run_pisa(args, wl):
         },
         "dense_baseline": dense,
         "tail_diagnostic": diag,
+        "backward_0th": bwd,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -585,6 +651,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the zeroth-order backward")
     ap.add_argument("--no-diagnostic", action="store_true",
                     help="skip the histogram of the unselected blocks' scores")
     ap.add_argument("--heads", type=int, default=0,

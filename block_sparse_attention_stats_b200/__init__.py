@@ -5,6 +5,9 @@ include/pisa.h); this package is its thin Python binding.
 """
 from .api import (  # noqa: F401
     PisaError,
+    piecewise_sparse_attention,
+    piecewise_sparse_attention_0th,
+    piecewise_sparse_attention_hyd,
     pisa_attention,
     pisa_attention_ex,
     pisa_block_stats,
@@ -16,6 +19,8 @@ from .api import (  # noqa: F401
     pisa_select,
     pisa_selftest_timeout,
     pisa_sparse_attention,
+    pisa_sparse_attention_bwd,
+    pisa_sparse_attention_fwd,
     pisa_tail_score_histogram,
     pisa_workspace_bytes,
 )

@@ -9,7 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import math
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -168,6 +168,84 @@ def pisa_sparse_attention(q, k, v, kbar, vsum, hbar, idx, mode: str = "hyd",
         k_sel, B, H, Ln, d, block_size, 0.0 if scale is None else float(scale), _MODE[mode],
         _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
     return out
+
+
+def pisa_sparse_attention_fwd(q, k, v, kbar, vsum, hbar, idx, mode: str = "0th",
+                              block_size: int = 64, scale: Optional[float] = None,
+                              out: Optional[torch.Tensor] = None,
+                              lse: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None, stream=None):
+    """pisa_sparse_attention that also returns lse [B, H, L] float32 (ln D_t)."""
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    k_sel = idx.shape[-1]
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, H, Ln, dtype=torch.float32, device=q.device) if lse is None else lse
+    need = lib.pisa_sparse_attention_workspace_bytes(B, H, Ln, d, block_size, _DT[q.dtype])
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check("pisa_sparse_attention_fwd", lib.pisa_sparse_attention_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(idx),
+        k_sel, B, H, Ln, d, block_size, 0.0 if scale is None else float(scale), _MODE[mode],
+        _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return out, lse
+
+
+def pisa_sparse_attention_bwd(q, k, v, dout, lse, kbar, vsum, idx, block_size: int = 64,
+                              scale: Optional[float] = None,
+                              grads: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+                              workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients (dq, dk, dv) of the zeroth-order forward, bf16 [B, H, L, d]."""
+    lib = L.load()
+    B, H, Ln, d = _qkv_dims(q, k, v)
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
+                                                  torch.empty_like(v))
+    need = lib.pisa_sparse_attention_bwd_workspace_bytes(B, H, Ln, d, block_size)
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check("pisa_sparse_attention_bwd", lib.pisa_sparse_attention_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(kbar), _ptr(vsum),
+        _ptr(idx), idx.shape[-1], B, H, Ln, d, block_size,
+        0.0 if scale is None else float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return dq, dk, dv
+
+
+class _PiecewiseAttention0th(torch.autograd.Function):
+    """Zeroth-order piecewise attention with its backward (every step in libpisa)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, density, block_size, sink_idx, scale):
+        q, k, v = (x.contiguous() for x in (q, k, v))
+        st = pisa_block_stats(q, k, v, block_size)
+        idx = pisa_select(st["qbar"], st["kbar"], density, sink_idx, scale=scale)
+        out, lse = pisa_sparse_attention_fwd(q, k, v, st["kbar"], st["vsum"], st["hbar"], idx,
+                                             "0th", block_size, scale)
+        ctx.save_for_backward(q, k, v, lse, st["kbar"], st["vsum"], idx)
+        ctx.block_size, ctx.scale = block_size, scale
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, lse, kbar, vsum, idx = ctx.saved_tensors
+        dq, dk, dv = pisa_sparse_attention_bwd(q, k, v, dout.contiguous(), lse, kbar, vsum, idx,
+                                               ctx.block_size, ctx.scale)
+        return dq, dk, dv, None, None, None, None
+
+
+def piecewise_sparse_attention_0th(q, k, v, density: float = 0.15, block_size: int = 64,
+                                   sink_idx: Optional[int] = None,
+                                   scale: Optional[float] = None) -> torch.Tensor:
+    """The authors' trainable zeroth-order variant: bf16 [B, H, L, d] in and out,
+    differentiable with respect to q, k and v (selection held fixed)."""
+    return _PiecewiseAttention0th.apply(q, k, v, density, block_size, sink_idx, scale)
+
+
+def piecewise_sparse_attention_hyd(q, k, v, density: float = 0.15, block_size: int = 64,
+                                   sink_idx: Optional[int] = None) -> torch.Tensor:
+    """The paper version (zeroth-order tail + global first-order term), forward only."""
+    return pisa_attention(q, k, v, density, block_size, sink_idx, "hyd")
+
+
+piecewise_sparse_attention = piecewise_sparse_attention_hyd
 
 
 # ---- the whole path --------------------------------------------------------------

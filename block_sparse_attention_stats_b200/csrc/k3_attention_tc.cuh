@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(192, 2)
                                   const int32_t *__restrict__ idx,
                                   const int2 *__restrict__ pairs, int k_sel, int L, int N,
                                   float scale, int hyd, int dense, int blockwise,
-                                  void *__restrict__ out, int out_f32) {
+                                  void *__restrict__ out, int out_f32,
+                                  float *__restrict__ lse) {
   using C = TcCfg<D>;
   using namespace sm100;
   extern __shared__ unsigned char smem_raw[];
@@ -562,6 +563,9 @@ __global__ void __launch_bounds__(192, 2)
         const float inv = 1.f / l_run;
         const float fa = hyd ? scale * a_run : 0.f;
         const size_t obase = ((size_t)bh * L + (size_t)(store ? grow_row : 0)) * D;
+        // natural log of D_t: the weights were 2^(s q k log2(e) - m_run), summed in l_run
+        if (lse != nullptr && store)
+          lse[(size_t)bh * L + grow_row] = (m_run + log2f(l_run)) * 0.6931471805599453f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32], qh[32];

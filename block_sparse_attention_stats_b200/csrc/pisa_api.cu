@@ -6,6 +6,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 #include <string>
@@ -17,6 +18,7 @@
 #include "k3_pack.cuh"
 #include "k3_attention_tc.cuh"
 #include "k5_tail_histogram.cuh"
+#include "k6_backward.cuh"
 
 namespace pisa {
 
@@ -245,7 +247,8 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
                                            const __nv_bfloat16 *hbar16, const int32_t *idx,
                                            const int2 *pairs, int k_sel, int BH, int L,
                                            float scale, int hyd, int dense, int blockwise,
-                                           void *out, int out_f32, cudaStream_t st) {
+                                           void *out, int out_f32, float *lse,
+                                           cudaStream_t st) {
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
   const int smem = TcCfg<D>::smem_bytes(N);
   if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
@@ -265,7 +268,8 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
   PISA_CUDA(cudaFuncSetAttribute(piecewise_attention_tc_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   piecewise_attention_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), TcCfg<D>::kThreads, smem, st>>>(
-      mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, scale, hyd, dense, blockwise, out, out_f32);
+      mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, scale, hyd, dense, blockwise, out, out_f32,
+      lse);
   return check_launch();
 }
 
@@ -278,7 +282,7 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
                                         pisa_dtype dt, const float *kbar, const float *vsum,
                                         const float *hbar, const int32_t *idx, int k_sel, int BH,
                                         int L, int d, float scale, pisa_mode mode, void *out,
-                                        unsigned char *ws, cudaStream_t st) {
+                                        float *lse, unsigned char *ws, cudaStream_t st) {
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
   const SparseLayout lay = sparse_layout(1, BH, L, d, dt);
   __nv_bfloat16 *kbar16 = (__nv_bfloat16 *)(ws + lay.kbar16);
@@ -322,9 +326,58 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   const int of32 = dt == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel,
-                                        BH, L, scale, hyd, 0, blockwise, out, of32, st);
+                                        BH, L, scale, hyd, 0, blockwise, out, of32, lse, st);
   return launch_attention_kernel<64>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel, BH,
-                                     L, scale, hyd, 0, blockwise, out, of32, st);
+                                     L, scale, hyd, 0, blockwise, out, of32, lse, st);
+}
+
+// ---- backward of the zeroth-order variant ------------------------------------
+struct BwdLayout {
+  size_t delta, kbar16, vbar16, bm, dkbar, dvbar, total;
+};
+static BwdLayout bwd_layout(int B, int H, int L, int d) {
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+  const size_t BH = (size_t)B * H;
+  BwdLayout p;
+  size_t o = 0;
+  p.delta = o; o += align_up(BH * L * 4, 256);
+  p.kbar16 = o; o += align_up(BH * Npad * d * 2, 256);
+  p.vbar16 = o; o += align_up(BH * Npad * d * 2, 256);
+  p.bm = o; o += align_up(BH * N * nwords * 4, 256);
+  p.dkbar = o; o += align_up(BH * Npad * d * 4, 256);
+  p.dvbar = o; o += align_up(BH * Npad * d * 4, 256);
+  p.total = o;
+  return p;
+}
+
+template <int D>
+static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                              const __nv_bfloat16 *v, const __nv_bfloat16 *dout, const float *lse,
+                              const int32_t *idx, int k_sel, int BH, int L, float scale,
+                              const BwdLayout &lay, unsigned char *ws, __nv_bfloat16 *dq,
+                              __nv_bfloat16 *dk, __nv_bfloat16 *dv, cudaStream_t st) {
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+  float *delta = (float *)(ws + lay.delta);
+  const __nv_bfloat16 *kb = (const __nv_bfloat16 *)(ws + lay.kbar16);
+  const __nv_bfloat16 *vb = (const __nv_bfloat16 *)(ws + lay.vbar16);
+  const uint32_t *bm = (const uint32_t *)(ws + lay.bm);
+  float *dkbar = (float *)(ws + lay.dkbar), *dvbar = (float *)(ws + lay.dvbar);
+  const int dq_smem = BwdDqCfg<D>::kSmem, kv_smem = BwdKvCfg<D>::kSmem;
+  PISA_CUDA(cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dq_smem));
+  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_kernel<D, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kv_smem));
+  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_kernel<D, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kv_smem));
+  bwd_dq_kernel<D><<<dim3(N, BH), kBwdThreads, dq_smem, st>>>(
+      q, k, v, dout, lse, kb, vb, idx, bm, k_sel, L, N, Npad, nwords, scale, delta, dq);
+  PISA_TRY(check_launch());
+  bwd_kv_kernel<D, true><<<dim3(Npad / 64, BH), kBwdThreads, kv_smem, st>>>(
+      q, k, v, dout, lse, delta, kb, vb, bm, L, N, Npad, nwords, scale, dkbar, dvbar, dk, dv);
+  PISA_TRY(check_launch());
+  bwd_kv_kernel<D, false><<<dim3(N, BH), kBwdThreads, kv_smem, st>>>(
+      q, k, v, dout, lse, delta, kb, vb, bm, L, N, Npad, nwords, scale, dkbar, dvbar, dk, dv);
+  return check_launch();
 }
 
 }  // namespace pisa
@@ -449,11 +502,13 @@ pisa_status pisa_select(const float *qbar, const float *kbar, const float *cov, 
                        sink_block(sink_idx, N), idx, (float *)workspace, (cudaStream_t)stream);
 }
 
-pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, pisa_dtype dtype,
-                                  const float *kbar, const float *vsum, const float *hbar,
-                                  const int32_t *idx, int k_sel, int B, int H, int L, int d,
-                                  int block_size, float scale, pisa_mode mode, void *out,
-                                  void *workspace, size_t ws_bytes, pisa_stream_t stream) {
+static pisa_status sparse_attention_checked(const void *q, const void *k, const void *v,
+                                            pisa_dtype dtype, const float *kbar,
+                                            const float *vsum, const float *hbar,
+                                            const int32_t *idx, int k_sel, int B, int H, int L,
+                                            int d, int block_size, float scale, pisa_mode mode,
+                                            void *out, float *lse, void *workspace,
+                                            size_t ws_bytes, pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, block_size));
   if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
   if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH && mode != PISA_MODE_1ST) return PISA_ERR_INVALID_ARG;
@@ -467,7 +522,78 @@ pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, p
   if (ws_bytes < sparse_ws(B, H, L, d, dtype)) return PISA_ERR_WORKSPACE;
   const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
   return run_sparse_attention(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B * H, L, d, s, mode,
-                              out, (unsigned char *)workspace, (cudaStream_t)stream);
+                              out, lse, (unsigned char *)workspace, (cudaStream_t)stream);
+}
+
+pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, pisa_dtype dtype,
+                                  const float *kbar, const float *vsum, const float *hbar,
+                                  const int32_t *idx, int k_sel, int B, int H, int L, int d,
+                                  int block_size, float scale, pisa_mode mode, void *out,
+                                  void *workspace, size_t ws_bytes, pisa_stream_t stream) {
+  return sparse_attention_checked(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B, H, L, d,
+                                  block_size, scale, mode, out, nullptr, workspace, ws_bytes,
+                                  stream);
+}
+
+pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *v,
+                                      pisa_dtype dtype, const float *kbar, const float *vsum,
+                                      const float *hbar, const int32_t *idx, int k_sel, int B,
+                                      int H, int L, int d, int block_size, float scale,
+                                      pisa_mode mode, void *out, float *lse, void *workspace,
+                                      size_t ws_bytes, pisa_stream_t stream) {
+  if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u)) return PISA_ERR_INVALID_ARG;
+  return sparse_attention_checked(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B, H, L, d,
+                                  block_size, scale, mode, out, lse, workspace, ws_bytes, stream);
+}
+
+size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size) {
+  if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
+  return bwd_layout(B, H, L, d).total;
+}
+
+pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *v,
+                                      const void *dout, const float *lse,
+                                      const float *kbar, const float *vsum, const int32_t *idx,
+                                      int k_sel, int B, int H, int L, int d, int block_size,
+                                      float scale, void *dq, void *dk, void *dv, void *workspace,
+                                      size_t ws_bytes, pisa_stream_t stream) {
+  PISA_TRY(check_shape(B, H, L, d, block_size));
+  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+  if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
+  const void *ins[] = {q, k, v, dout};
+  void *outs[] = {dq, dk, dv};
+  for (const void *p : ins)
+    if (!aligned16(p)) return PISA_ERR_INVALID_ARG;
+  for (void *p : outs) {
+    if (!aligned16(p)) return PISA_ERR_INVALID_ARG;
+    for (const void *i : ins)
+      if (p == i) return PISA_ERR_INVALID_ARG;
+  }
+  if (dq == dk || dq == dv || dk == dv) return PISA_ERR_INVALID_ARG;
+  if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(kbar) || !aligned16(vsum) ||
+      !idx || !aligned16(workspace))
+    return PISA_ERR_INVALID_ARG;
+  const BwdLayout lay = bwd_layout(B, H, L, d);
+  if (ws_bytes < lay.total) return PISA_ERR_WORKSPACE;
+  const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
+  const int BH = B * H;
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned char *ws = (unsigned char *)workspace;
+  bwd_pack_centroids_kernel<<<grid_1d((size_t)BH * Npad * d, 256), 256, 0, st>>>(
+      kbar, vsum, N, Npad, d, BH, L, (__nv_bfloat16 *)(ws + lay.kbar16),
+      (__nv_bfloat16 *)(ws + lay.vbar16));
+  PISA_TRY(check_launch());
+  selection_bitmap_kernel<<<dim3(N, BH), 64, nwords * sizeof(uint32_t), st>>>(
+      idx, N, k_sel, nwords, (uint32_t *)(ws + lay.bm));
+  PISA_TRY(check_launch());
+  const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
+                      *v16 = (const __nv_bfloat16 *)v, *g16 = (const __nv_bfloat16 *)dout;
+  if (d == 128)
+    return launch_bwd<128>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, s, lay, ws,
+                           (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, st);
+  return launch_bwd<64>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, s, lay, ws,
+                        (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, st);
 }
 
 pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void *out, int B,
@@ -522,7 +648,7 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
                       sink_block(sink_idx, N), idx, (float *)scratch, st);
   if (r == PISA_OK)
     r = run_sparse_attention(q, k, v, o.dtype, kbar, vsum, hbar, idx, k_sel, BH, L, d, s, mode,
-                             out, scratch, st);
+                             out, nullptr, scratch, st);
   if (owned) {
     cudaError_t e = cudaFreeAsync(ws, st);
     if (e != cudaSuccess && r == PISA_OK) {
@@ -575,9 +701,9 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
   const int of32 = dtype == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr,
-                                        nullptr, 0, BH, L, s, 0, 1, 0, out, of32, st);
+                                        nullptr, 0, BH, L, s, 0, 1, 0, out, of32, nullptr, st);
   return launch_attention_kernel<64>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                     0, BH, L, s, 0, 1, 0, out, of32, st);
+                                     0, BH, L, s, 0, 1, 0, out, of32, nullptr, st);
 }
 
 pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v,

@@ -158,6 +158,43 @@ pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v,
                                   pisa_mode mode, void *out, void *workspace,
                                   size_t ws_bytes, pisa_stream_t stream);
 
+/* pisa_sparse_attention that also writes lse [B,H,L] float32 (4-byte
+ * aligned): lse_t = ln D_t, the natural log of the denominator above (the
+ * same in modes hyd and 0th, which differ only in the numerator).  It is what
+ * pisa_sparse_attention_bwd needs from the forward. */
+pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *v,
+                                      pisa_dtype dtype, const float *kbar, const float *vsum,
+                                      const float *hbar, const int32_t *idx, int k_sel, int B,
+                                      int H, int L, int d, int block_size, float scale,
+                                      pisa_mode mode, void *out, float *lse, void *workspace,
+                                      size_t ws_bytes, pisa_stream_t stream);
+
+/* ---- training: gradients of the zeroth-order variant ------------------------ */
+
+/* Workspace bytes of pisa_sparse_attention_bwd (0 on invalid arguments). */
+size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size);
+
+/* Gradients of the zeroth-order forward (the authors' README, "Kernel
+ * variants": piecewise_sparse_attention_0th "supports training"; the forward
+ * is the equation above without the hyd term).  Given dout = dL/d out, writes
+ *   dq = dL/dq,  dk = dL/dk,  dv = dL/dv        bf16 [B,H,L,d]
+ * with the selection idx held fixed (a discrete step) and the statistics
+ * differentiated: kbar_j is the mean key and vsum_j the value sum of block j,
+ * so each tail term's gradient reaches every key and value of block j.
+ * q, k, v, dout: bf16 [B,H,L,d]; lse from pisa_sparse_attention_fwd on the
+ * same q, k, v, kbar, vsum, idx; kbar, vsum: float32 from pisa_block_stats.
+ * The forward output itself is not needed: the row term
+ * Delta_t = sum_m P_tm (dout_t . value_m) is formed from the recomputed
+ * probabilities, consistent with the ones the gradients use.  dq, dk, dv must
+ * not overlap any input or one another.  No atomics: bitwise reproducible.
+ * `workspace`: pisa_sparse_attention_bwd_workspace_bytes(...) bytes. */
+pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *v,
+                                      const void *dout, const float *lse,
+                                      const float *kbar, const float *vsum, const int32_t *idx,
+                                      int k_sel, int B, int H, int L, int d, int block_size,
+                                      float scale, void *dq, void *dk, void *dv, void *workspace,
+                                      size_t ws_bytes, pisa_stream_t stream);
+
 /* ---- diagnostic ------------------------------------------------------------ */
 
 /* Distributional stability of the non-critical blocks (gist.science summary,
