@@ -161,6 +161,21 @@ def k3_executed_flops(wl, idx: torch.Tensor, heads: int = 2) -> float:
     tot = 0.0
     idx_np = idx.reshape(-1, N, idx.shape[-1]).cpu().numpy()
     use = min(heads, idx_np.shape[0])
+    if b == 128:
+        # one CTA per query block: the 64-token tiles of its selected blocks
+        # (the last block may have one tile) and the centroid chunks it needs
+        ntile = -(-wl.L // 64)
+        tiles_of = np.array([min(2, ntile - 2 * j) for j in range(N)])
+        for h in range(use):
+            bits = np.zeros((N, N), dtype=bool)
+            np.put_along_axis(bits, idx_np[h].astype(np.int64), True, axis=1)
+            for i in range(N):
+                chunks = sum(int((~bits[i, c * 64:min(N, c * 64 + 64)]).any())
+                             for c in range(nch))
+                tot += (int(tiles_of[bits[i]].sum()) + chunks) * tile
+                if wl.mode == "hyd":
+                    tot += 2.0 * 128 * d * d
+        return tot * (wl.B * wl.H) / use
     for h in range(use):
         bits = np.zeros((N, N), dtype=bool)
         np.put_along_axis(bits, idx_np[h].astype(np.int64), True, axis=1)
@@ -446,7 +461,8 @@ def run_pisa(args, wl):
                       cov_weight=wl.cov_weight, workspace=sel_ws, out=idx)
         e[2].record(stream)
         P.pisa_sparse_attention(Q, K, V, stt["kbar"], stt["vsum"], stt["hbar"], idx,
-                                mode=wl.mode, out=out, workspace=k3_ws)
+                                mode=wl.mode, block_size=wl.block_size, out=out,
+                                workspace=k3_ws)
         e[3].record(stream)
     torch.cuda.synchronize()
     parts = {"block_stats": [e[0].elapsed_time(e[1]) for e in ev],
@@ -474,7 +490,7 @@ def run_pisa(args, wl):
 
     # ---- distributional-stability diagnostic over the step's own selection -------
     diag = None
-    if not args.no_diagnostic:
+    if not args.no_diagnostic and wl.block_size == 64:
         qs = 8 if wl.L > 20000 else 1
         lo, hi, nb = -8.0, 8.0, 64
         P.pisa_tail_score_histogram(Q, K, idx, lo, hi, nb, wl.block_size, query_stride=qs)
@@ -497,7 +513,7 @@ def run_pisa(args, wl):
 
     # ---- backward of the zeroth-order variant (training), same inputs -----------
     bwd = None
-    if not args.no_backward and wl.dtype == "bf16":
+    if not args.no_backward and wl.dtype == "bf16" and wl.block_size == 64:
         G = torch.randn(Q.shape, generator=torch.Generator(device=dev).manual_seed(11),
                         device=dev).to(Q.dtype)
         lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)

@@ -26,7 +26,7 @@
 namespace pisa {
 
 constexpr int kStatsThreads = 256;
-constexpr int kBlk = 64;  // tokens per block (block_size)
+constexpr int kBlk = 64;  // tokens per streamed tile; a block is 1 or 2 tiles (block_size 64 / 128)
 
 // Chunking of pass 1: at most two CTAs per SM over the whole problem (one wave).
 __host__ __device__ inline int stats_num_chunks(int BH, int N) {
@@ -97,7 +97,8 @@ __device__ __forceinline__ void ktv_mma(float (&acc)[StatsMmaCfg<D>::kMT][StatsM
 // tensor cores: C = 1^T X with an all-ones A operand; every row of C holds the
 // column sums.  Warp w handles n-tiles 6w .. 6w+5 of the 3D/8 tiles.
 template <int D>
-__device__ __forceinline__ void colsum_mma(uint32_t tiles, float *colsum, int warp, int lane) {
+__device__ __forceinline__ void colsum_mma(uint32_t tiles, float *colsum, int warp, int lane,
+                                           bool accumulate) {
   using C = StatsMmaCfg<D>;
   constexpr int kNT = 3 * D / 8;           // 8-column tiles over Q, K, V
   constexpr int kPerWarp = kNT / 8;        // 6 (D=128) or 3 (D=64)
@@ -130,8 +131,9 @@ __device__ __forceinline__ void colsum_mma(uint32_t tiles, float *colsum, int wa
     for (int i = 0; i < kPerWarp; ++i) {
       const int nt = warp * kPerWarp + i;
       const int which = nt / (D / 8), col = (nt % (D / 8)) * 8 + 2 * lane;
-      colsum[which * D + col] = acc[i][0];
-      colsum[which * D + col + 1] = acc[i][1];
+      colsum[which * D + col] = accumulate ? colsum[which * D + col] + acc[i][0] : acc[i][0];
+      colsum[which * D + col + 1] =
+          accumulate ? colsum[which * D + col + 1] + acc[i][1] : acc[i][1];
     }
   }
 }
@@ -139,9 +141,10 @@ __device__ __forceinline__ void colsum_mma(uint32_t tiles, float *colsum, int wa
 template <int D>
 __global__ void __launch_bounds__(kStatsThreads)
     stats_pass_bf16_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
-                           const __nv_bfloat16 *__restrict__ V, int L, int N, int nchunk,
+                           const __nv_bfloat16 *__restrict__ V, int L, int N, int sub, int nchunk,
                            float *__restrict__ qbar, float *__restrict__ kbar,
                            float *__restrict__ vsum, float *__restrict__ partial) {
+  // N blocks of sub x 64 tokens; the kernel streams 64-token tiles
   using C = StatsMmaCfg<D>;
   extern __shared__ __align__(128) unsigned char smem[];
   // [stage][Q,K,V] tiles, then column sums (3 x D floats)
@@ -151,6 +154,8 @@ __global__ void __launch_bounds__(kStatsThreads)
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int per = ceil_div(N, nchunk);
   const int j0 = chunk * per, j1 = min(N, j0 + per);
+  const int ntile = ceil_div(L, kBlk);
+  const int u0 = j0 * sub, u1 = min(ntile, j1 * sub);   // 64-token tiles of this chunk
   const size_t head = (size_t)bh * L * D;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int warp_m0 = (warp / C::kWarpsN) * C::kWarpRows;
@@ -164,53 +169,57 @@ __global__ void __launch_bounds__(kStatsThreads)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
 
-  auto issue = [&](int j, int stage) {
-    int valid = min(kBlk, L - j * kBlk);
-    size_t off = head + (size_t)j * kBlk * D;
+  auto issue = [&](int u, int stage) {
+    int valid = min(kBlk, L - u * kBlk);
+    size_t off = head + (size_t)u * kBlk * D;
     uint32_t st = sbase + stage * 3 * C::kTileBytes;
     stats_load_tile_bf16<D>(st, Q + off, valid);
     stats_load_tile_bf16<D>(st + C::kTileBytes, K + off, valid);
     stats_load_tile_bf16<D>(st + 2 * C::kTileBytes, V + off, valid);
   };
 
-  if (j0 < j1) issue(j0, 0);
+  if (u0 < u1) issue(u0, 0);
   cp_async_commit();
-  for (int j = j0; j < j1; ++j) {
-    const int stage = (j - j0) & 1;
-    if (j + 1 < j1) issue(j + 1, stage ^ 1);
+  for (int u = u0; u < u1; ++u) {
+    const int stage = (u - u0) & 1;
+    if (u + 1 < u1) issue(u + 1, stage ^ 1);
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
 
-    const int n_j = min(kBlk, L - j * kBlk);
-    // column sums of Q, K, V (zero-filled rows past L add nothing)
-    colsum_mma<D>(sbase + stage * 3 * C::kTileBytes, colsum, warp, lane);
+    const int j = u / sub, s = u - j * sub;
+    const bool last = s == sub - 1 || u == ntile - 1;   // block j ends with this tile
+    // column sums of Q, K, V (zero-filled rows past L add nothing), summed
+    // over the tiles of block j
+    colsum_mma<D>(sbase + stage * 3 * C::kTileBytes, colsum, warp, lane, s > 0);
     const uint32_t sK = sbase + stage * 3 * C::kTileBytes + C::kTileBytes;
     ktv_mma<D>(acc, sK, sK + C::kTileBytes, warp_m0, warp_n0, lane);
     __syncthreads();  // colsum visible
-
-    const float inv_n = 1.f / (float)n_j;
-    const size_t so = ((size_t)bh * N + j) * D;
-    for (int t = tid; t < 3 * D; t += kStatsThreads) {
-      const int which = t / D, col = t % D;
-      if (which == 0) qbar[so + col] = colsum[t] * inv_n;
-      else if (which == 1) kbar[so + col] = colsum[t] * inv_n;
-      else vsum[so + col] = colsum[t];
-    }
-    // acc -= kbar_j^T vsum_j
-    const int g = lane >> 2, tq = lane & 3;
-#pragma unroll
-    for (int mt = 0; mt < C::kMT; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < C::kNT; ++nt) {
-        const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
-        const float ka = colsum[D + a0] * inv_n, kb = colsum[D + a0 + 8] * inv_n;
-        const float v0 = colsum[2 * D + c0], v1 = colsum[2 * D + c0 + 1];
-        acc[mt][nt][0] -= ka * v0;
-        acc[mt][nt][1] -= ka * v1;
-        acc[mt][nt][2] -= kb * v0;
-        acc[mt][nt][3] -= kb * v1;
+    if (last) {
+      const int n_j = min(sub * kBlk, L - j * sub * kBlk);
+      const float inv_n = 1.f / (float)n_j;
+      const size_t so = ((size_t)bh * N + j) * D;
+      for (int t = tid; t < 3 * D; t += kStatsThreads) {
+        const int which = t / D, col = t % D;
+        if (which == 0) qbar[so + col] = colsum[t] * inv_n;
+        else if (which == 1) kbar[so + col] = colsum[t] * inv_n;
+        else vsum[so + col] = colsum[t];
       }
+      // acc -= kbar_j^T vsum_j
+      const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+      for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::kNT; ++nt) {
+          const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
+          const float ka = colsum[D + a0] * inv_n, kb = colsum[D + a0 + 8] * inv_n;
+          const float v0 = colsum[2 * D + c0], v1 = colsum[2 * D + c0 + 1];
+          acc[mt][nt][0] -= ka * v0;
+          acc[mt][nt][1] -= ka * v1;
+          acc[mt][nt][2] -= kb * v0;
+          acc[mt][nt][3] -= kb * v1;
+        }
+    }
     __syncthreads();  // stage and colsum free for reuse
   }
   cp_async_wait<0>();
@@ -235,7 +244,7 @@ __global__ void __launch_bounds__(kStatsThreads)
 template <int D>
 __global__ void __launch_bounds__(kStatsThreads)
     stats_pass_f32_kernel(const float *__restrict__ Q, const float *__restrict__ K,
-                          const float *__restrict__ V, int L, int N, int nchunk,
+                          const float *__restrict__ V, int L, int N, int sub, int nchunk,
                           float *__restrict__ qbar, float *__restrict__ kbar,
                           float *__restrict__ vsum, float *__restrict__ partial) {
   constexpr int kPer = D * D / kStatsThreads;
@@ -255,30 +264,41 @@ __global__ void __launch_bounds__(kStatsThreads)
   for (int r = 0; r < kPer; ++r) acc[r] = 0.f;
 
   for (int j = j0; j < j1; ++j) {
-    const int n_j = min(kBlk, L - j * kBlk);
-    const size_t off = head + (size_t)j * kBlk * D;
-    for (int e = tid; e < kBlk * D; e += kStatsThreads) {
-      const bool ok = e < n_j * D;
-      sQ[e] = ok ? Q[off + e] : 0.f;
-      sK[e] = ok ? K[off + e] : 0.f;
-      sV[e] = ok ? V[off + e] : 0.f;
-    }
-    __syncthreads();
-    for (int t = tid; t < 3 * D; t += kStatsThreads) {
-      const float *tile = (t < D) ? sQ : (t < 2 * D ? sK : sV);
-      const int col = t % D;
-      float s = 0.f;
-      for (int row = 0; row < kBlk; ++row) s += tile[row * D + col];
-      colsum[t] = s;
+    const int n_j = min(sub * kBlk, L - j * sub * kBlk);
+    for (int t = tid; t < 3 * D; t += kStatsThreads) colsum[t] = 0.f;
+    // the block's 64-token tiles: column sums and sum_n k_n^T v_n
+    for (int s0 = 0; s0 < n_j; s0 += kBlk) {
+      const int rows = min(kBlk, n_j - s0);
+      const size_t off = head + ((size_t)j * sub * kBlk + s0) * D;
+      __syncthreads();
+      for (int e = tid; e < kBlk * D; e += kStatsThreads) {
+        const bool ok = e < rows * D;
+        sQ[e] = ok ? Q[off + e] : 0.f;
+        sK[e] = ok ? K[off + e] : 0.f;
+        sV[e] = ok ? V[off + e] : 0.f;
+      }
+      __syncthreads();
+      for (int t = tid; t < 3 * D; t += kStatsThreads) {
+        const float *tile = (t < D) ? sQ : (t < 2 * D ? sK : sV);
+        const int col = t % D;
+        float sum = 0.f;
+        for (int row = 0; row < kBlk; ++row) sum += tile[row * D + col];
+        colsum[t] += sum;
+      }
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int e = tid + r * kStatsThreads, a = e / D, c = e % D;
+        float sum = 0.f;
+        for (int row = 0; row < kBlk; ++row) sum += sK[row * D + a] * sV[row * D + c];
+        acc[r] += sum;
+      }
     }
     __syncthreads();
     const float inv_n = 1.f / (float)n_j;
 #pragma unroll
     for (int r = 0; r < kPer; ++r) {
       const int e = tid + r * kStatsThreads, a = e / D, c = e % D;
-      float s = 0.f;
-      for (int row = 0; row < kBlk; ++row) s += sK[row * D + a] * sV[row * D + c];
-      acc[r] += s - (colsum[D + a] * inv_n) * colsum[2 * D + c];
+      acc[r] -= (colsum[D + a] * inv_n) * colsum[2 * D + c];
     }
     const size_t so = ((size_t)bh * N + j) * D;
     for (int t = tid; t < 3 * D; t += kStatsThreads) {
@@ -331,7 +351,7 @@ __device__ __forceinline__ float block_reduce_sum(float v, float *red) {
 template <int D>
 __global__ void __launch_bounds__(kStatsThreads)
     cov_pass_bf16_kernel(const __nv_bfloat16 *__restrict__ K, const __nv_bfloat16 *__restrict__ V,
-                         int L, int N, int nchunk, const float *__restrict__ kbar,
+                         int L, int N, int sub, int nchunk, const float *__restrict__ kbar,
                          const float *__restrict__ vsum, const float *__restrict__ hbar,
                          float *__restrict__ cov) {
   using C = StatsMmaCfg<D>;
@@ -341,6 +361,8 @@ __global__ void __launch_bounds__(kStatsThreads)
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int per = ceil_div(N, nchunk);
   const int j0 = chunk * per, j1 = min(N, j0 + per);
+  const int ntile = ceil_div(L, kBlk);
+  const int u0 = j0 * sub, u1 = min(ntile, j1 * sub);
   const size_t head = (size_t)bh * L * D;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int warp_m0 = (warp / C::kWarpsN) * C::kWarpRows;
@@ -361,48 +383,54 @@ __global__ void __launch_bounds__(kStatsThreads)
       hb[mt][nt][3] = Hb[(a0 + 8) * D + c0 + 1];
     }
 
-  auto issue = [&](int j, int stage) {
-    int valid = min(kBlk, L - j * kBlk);
-    size_t off = head + (size_t)j * kBlk * D;
+  auto issue = [&](int u, int stage) {
+    int valid = min(kBlk, L - u * kBlk);
+    size_t off = head + (size_t)u * kBlk * D;
     uint32_t st = sbase + stage * 2 * C::kTileBytes;
     stats_load_tile_bf16<D>(st, K + off, valid);
     stats_load_tile_bf16<D>(st + C::kTileBytes, V + off, valid);
   };
-  if (j0 < j1) issue(j0, 0);
+  float acc[C::kMT][C::kNT][4];
+  if (u0 < u1) issue(u0, 0);
   cp_async_commit();
-  for (int j = j0; j < j1; ++j) {
-    const int stage = (j - j0) & 1;
-    if (j + 1 < j1) issue(j + 1, stage ^ 1);
+  for (int u = u0; u < u1; ++u) {
+    const int stage = (u - u0) & 1;
+    if (u + 1 < u1) issue(u + 1, stage ^ 1);
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
-    float acc[C::kMT][C::kNT][4];
+    const int j = u / sub, s = u - j * sub;
+    const bool last = s == sub - 1 || u == ntile - 1;
+    if (s == 0) {
 #pragma unroll
-    for (int mt = 0; mt < C::kMT; ++mt)
+      for (int mt = 0; mt < C::kMT; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < C::kNT; ++nt)
+        for (int nt = 0; nt < C::kNT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+          for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    }
     const uint32_t sK = sbase + stage * 2 * C::kTileBytes;
     ktv_mma<D>(acc, sK, sK + C::kTileBytes, warp_m0, warp_n0, lane);
-    const float *kb = kbar + ((size_t)bh * N + j) * D;
-    const float *vs = vsum + ((size_t)bh * N + j) * D;
-    float ss = 0.f;
-#pragma unroll
-    for (int mt = 0; mt < C::kMT; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < C::kNT; ++nt) {
-        const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
-        const float ka = kb[a0], kc = kb[a0 + 8], v0 = vs[c0], v1 = vs[c0 + 1];
-        float e0 = acc[mt][nt][0] - ka * v0 - hb[mt][nt][0];
-        float e1 = acc[mt][nt][1] - ka * v1 - hb[mt][nt][1];
-        float e2 = acc[mt][nt][2] - kc * v0 - hb[mt][nt][2];
-        float e3 = acc[mt][nt][3] - kc * v1 - hb[mt][nt][3];
-        ss += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
-      }
     __syncthreads();  // tiles of this stage consumed
-    float tot = block_reduce_sum(ss, red);
-    if (tid == 0) cov[(size_t)bh * N + j] = sqrtf(tot);
+    if (last) {
+      const float *kb = kbar + ((size_t)bh * N + j) * D;
+      const float *vs = vsum + ((size_t)bh * N + j) * D;
+      float ss = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::kNT; ++nt) {
+          const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
+          const float ka = kb[a0], kc = kb[a0 + 8], v0 = vs[c0], v1 = vs[c0 + 1];
+          float e0 = acc[mt][nt][0] - ka * v0 - hb[mt][nt][0];
+          float e1 = acc[mt][nt][1] - ka * v1 - hb[mt][nt][1];
+          float e2 = acc[mt][nt][2] - kc * v0 - hb[mt][nt][2];
+          float e3 = acc[mt][nt][3] - kc * v1 - hb[mt][nt][3];
+          ss += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+        }
+      float tot = block_reduce_sum(ss, red);
+      if (tid == 0) cov[(size_t)bh * N + j] = sqrtf(tot);
+    }
   }
   cp_async_wait<0>();
 }
@@ -410,7 +438,7 @@ __global__ void __launch_bounds__(kStatsThreads)
 template <int D>
 __global__ void __launch_bounds__(kStatsThreads)
     cov_pass_f32_kernel(const float *__restrict__ K, const float *__restrict__ V, int L, int N,
-                        const float *__restrict__ kbar, const float *__restrict__ vsum,
+                        int sub, const float *__restrict__ kbar, const float *__restrict__ vsum,
                         const float *__restrict__ hbar, float *__restrict__ cov) {
   constexpr int kPer = D * D / kStatsThreads;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -418,14 +446,28 @@ __global__ void __launch_bounds__(kStatsThreads)
   float *sV = sK + kBlk * D;
   float *red = sV + kBlk * D;
   const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const int n_j = min(kBlk, L - j * kBlk);
-  const size_t off = (size_t)bh * L * D + (size_t)j * kBlk * D;
-  for (int e = tid; e < kBlk * D; e += kStatsThreads) {
-    const bool ok = e < n_j * D;
-    sK[e] = ok ? K[off + e] : 0.f;
-    sV[e] = ok ? V[off + e] : 0.f;
+  const int n_j = min(sub * kBlk, L - j * sub * kBlk);
+  float acc[kPer];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) acc[r] = 0.f;
+  for (int s0 = 0; s0 < n_j; s0 += kBlk) {
+    const int rows = min(kBlk, n_j - s0);
+    const size_t off = (size_t)bh * L * D + ((size_t)j * sub * kBlk + s0) * D;
+    __syncthreads();
+    for (int e = tid; e < kBlk * D; e += kStatsThreads) {
+      const bool ok = e < rows * D;
+      sK[e] = ok ? K[off + e] : 0.f;
+      sV[e] = ok ? V[off + e] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int e = tid + r * kStatsThreads, a = e / D, c = e % D;
+      float sum = 0.f;
+      for (int row = 0; row < kBlk; ++row) sum += sK[row * D + a] * sV[row * D + c];
+      acc[r] += sum;
+    }
   }
-  __syncthreads();
   const float *kb = kbar + ((size_t)bh * N + j) * D;
   const float *vs = vsum + ((size_t)bh * N + j) * D;
   const float *Hb = hbar + (size_t)bh * D * D;
@@ -433,9 +475,7 @@ __global__ void __launch_bounds__(kStatsThreads)
 #pragma unroll
   for (int r = 0; r < kPer; ++r) {
     const int e = tid + r * kStatsThreads, a = e / D, c = e % D;
-    float s = 0.f;
-    for (int row = 0; row < kBlk; ++row) s += sK[row * D + a] * sV[row * D + c];
-    const float h = s - kb[a] * vs[c] - Hb[e];
+    const float h = acc[r] - kb[a] * vs[c] - Hb[e];
     ss += h * h;
   }
   float tot = block_reduce_sum(ss, red);

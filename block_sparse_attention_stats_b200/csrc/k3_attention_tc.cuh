@@ -20,6 +20,11 @@
 // summed into a_t = sum_{U_i} alpha_tj.  In the paper ("hyd") mode a last MMA
 // forms Q Hbar and the epilogue adds s a_t (q_t Hbar) to the numerator.
 //
+// With 128-token blocks (block_size 128) a CTA is one query block: both
+// halves share S_i, every selected block contributes its two 64-token tiles,
+// and the centroids (one per 128-token block, n_j = 128) are masked by the
+// block-level selection.
+//
 // Roles (192 threads):
 //   warp 0      TMA producer: Q once, then the K/V (or kbar/vsum) tile of every
 //               list entry into a 2-stage ring, then Hbar;
@@ -81,9 +86,10 @@ template <int D> struct TcCfg {
   static constexpr int kBarHFull = kBarTeardown + 1;
   static_assert(kBarHFull < kNumBars, "barrier slots");
 
-  __host__ __device__ static int smem_bytes(int N) {
-    const int nwords = (N + 31) / 32;
-    return kOffDyn + (2 * nwords + N + (N + 63) / 64) * 4 + 1024;  // + alignment slack
+  // N 64-token tiles, Nc blocks (= centroids)
+  __host__ __device__ static int smem_bytes(int N, int Nc) {
+    const int nwords = (N + 31) / 32, cwords = (Nc + 31) / 32;
+    return kOffDyn + (2 * nwords + 2 * cwords + N + (Nc + 63) / 64) * 4 + 1024;  // + slack
   }
 };
 
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(192, 2)
                                   const __grid_constant__ CUtensorMap tm_hbar,
                                   const int32_t *__restrict__ idx,
                                   const int2 *__restrict__ pairs, int k_sel, int L, int N,
-                                  float scale, int hyd, int dense, int blockwise,
+                                  int bsub, int Nc, float scale, int hyd, int dense, int blockwise,
                                   void *__restrict__ out, int out_f32,
                                   float *__restrict__ lse) {
   using C = TcCfg<D>;
@@ -115,18 +121,30 @@ __global__ void __launch_bounds__(192, 2)
   unsigned char *smem = smem_raw + (sbase - raw);
   auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
   volatile int *misc = reinterpret_cast<volatile int *>(smem + C::kOffMisc);  // [0] tiles, [1] abort
-  const int nwords = (N + 31) / 32;
+  // bm_*: selected 64-token tiles per half; cbm_*: selected blocks (the
+  // centroid index space) per half.  With 64-token blocks the two coincide;
+  // with 128-token blocks both halves are one query block and share them.
+  const int nwords = (N + 31) / 32, cwords = (Nc + 31) / 32;
   uint32_t *bm_lo = reinterpret_cast<uint32_t *>(smem + C::kOffDyn);
-  uint32_t *bm_hi = bm_lo + nwords;
-  int *tiles = reinterpret_cast<int *>(bm_hi + nwords);
+  uint32_t *bm_hi = bsub == 1 ? bm_lo + nwords : bm_lo;
+  uint32_t *cbm_lo = bsub == 1 ? bm_lo : bm_lo + 2 * nwords;
+  uint32_t *cbm_hi = bsub == 1 ? bm_hi : cbm_lo;
+  int *tiles = reinterpret_cast<int *>(bm_lo + 2 * nwords + 2 * cwords);
 
   const int pair = blockIdx.x, bh = blockIdx.y;
-  // query blocks of the two halves (rows 0-63 and 64-127 of the tile)
+  // query blocks of the two halves (rows 0-63 and 64-127 of the tile), as
+  // 64-token tiles; the selection row of each half
   int qb0 = 2 * pair, qb1 = 2 * pair + 1 < N ? 2 * pair + 1 : -1;
-  if (pairs) {
+  int sr0 = qb0, sr1 = qb1;
+  if (bsub == 2) {
+    sr0 = pair;
+    sr1 = pair;
+  } else if (pairs) {
     const int2 pr = pairs[(size_t)bh * ((N + 1) / 2) + pair];
     qb0 = pr.x;
     qb1 = pr.y;
+    sr0 = qb0;
+    sr1 = qb1;
   }
   const bool has_hi = qb1 >= 0;
   // warp index through a shuffle so the compiler knows it is warp-uniform: the
@@ -169,21 +187,35 @@ __global__ void __launch_bounds__(192, 2)
     prefetch_tmap(&tm_vsum);
     prefetch_tmap(&tm_hbar);
   }
-  for (int w = tid; w < 2 * nwords; w += C::kThreads) bm_lo[w] = 0u;
+  for (int w = tid; w < 2 * nwords + 2 * cwords; w += C::kThreads) bm_lo[w] = 0u;
   __syncthreads();
   if (dense) {
     for (int w = tid; w < nwords; w += C::kThreads) {
       bm_lo[w] = valid_bits(w, N);
       bm_hi[w] = has_hi ? valid_bits(w, N) : 0u;
     }
-  } else {
-    const int32_t *r0 = idx + ((size_t)bh * N + qb0) * k_sel;
-    const int32_t *r1 = idx + ((size_t)bh * N + (has_hi ? qb1 : qb0)) * k_sel;
+  } else if (bsub == 1) {
+    const int32_t *r0 = idx + ((size_t)bh * Nc + sr0) * k_sel;
+    const int32_t *r1 = idx + ((size_t)bh * Nc + (has_hi ? sr1 : sr0)) * k_sel;
     for (int t = tid; t < (has_hi ? 2 : 1) * k_sel; t += C::kThreads) {
       const int j = t < k_sel ? r0[t] : r1[t - k_sel];
       uint32_t *bm = t < k_sel ? bm_lo : bm_hi;
       if (j >= 0 && j < N) atomicOr(&bm[j >> 5], 1u << (j & 31));
       else report_device_error(kDevErrRange);
+    }
+  } else {
+    // one selection row for the 128-token query block: block j covers the
+    // 64-token tiles 2j and 2j + 1 (the last block may have only the first)
+    const int32_t *r0 = idx + ((size_t)bh * Nc + sr0) * k_sel;
+    for (int t = tid; t < k_sel; t += C::kThreads) {
+      const int j = r0[t];
+      if (j >= 0 && j < Nc) {
+        atomicOr(&cbm_lo[j >> 5], 1u << (j & 31));
+        for (int u = bsub * j; u < bsub * j + bsub && u < N; ++u)
+          atomicOr(&bm_lo[u >> 5], 1u << (u & 31));
+      } else {
+        report_device_error(kDevErrRange);
+      }
     }
   }
   __syncthreads();
@@ -212,15 +244,15 @@ __global__ void __launch_bounds__(192, 2)
     }
     // centroid chunks that hold an unselected block for either half
     if (!dense && !blockwise) {
-      const int nch = (N + 63) / 64;
+      const int nch = (Nc + 63) / 64;
       for (int c0 = 0; c0 < nch; c0 += 32) {
         const int c = c0 + lane;
         bool need = false;
         if (c < nch) {
           for (int h = 0; h < (has_hi ? 2 : 1); ++h) {
-            const uint32_t *bm = h ? bm_hi : bm_lo;
-            const uint32_t m0 = ~bm[2 * c] & valid_bits(2 * c, N);
-            const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & valid_bits(2 * c + 1, N)) : 0u;
+            const uint32_t *cb = h ? cbm_hi : cbm_lo;
+            const uint32_t m0 = ~cb[2 * c] & valid_bits(2 * c, Nc);
+            const uint32_t m1 = (2 * c + 1 < cwords) ? (~cb[2 * c + 1] & valid_bits(2 * c + 1, Nc)) : 0u;
             need = need || ((m0 | m1) != 0u);
           }
         }
@@ -393,10 +425,12 @@ __global__ void __launch_bounds__(192, 2)
     const int row = sp * 32 + lane;          // query row in the tile = TMEM lane
     const int half = row >> 6;               // warp-uniform
     const bool exists = half == 0 || has_hi;
-    const uint32_t *bm = half ? bm_hi : bm_lo;
+    const uint32_t *cbm = half ? cbm_hi : cbm_lo;
     const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
     const float sl2 = scale * kLog2e;
-    const int n_last = L - (N - 1) * 64;
+    const int n_last = L - (N - 1) * 64;                 // tokens in the last 64-token tile
+    const float wblk = 64.f * (float)bsub;               // n_j of a full block
+    const int nc_last = L - (Nc - 1) * 64 * bsub;        // n_j of the last block
     float m_run = -INFINITY, l_run = 0.f, a_run = 0.f;
     bool ok = true;
     // waits and abort checks are made warp-uniform: TMEM access is warp-collective
@@ -421,8 +455,8 @@ __global__ void __launch_bounds__(192, 2)
         active = ((e >> half) & 1) != 0 || taylor;
       } else {
         const int c = -e - 1;
-        const uint32_t m0 = ~bm[2 * c] & valid_bits(2 * c, N);
-        const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & valid_bits(2 * c + 1, N)) : 0u;
+        const uint32_t m0 = ~cbm[2 * c] & valid_bits(2 * c, Nc);
+        const uint32_t m1 = (2 * c + 1 < cwords) ? (~cbm[2 * c + 1] & valid_bits(2 * c + 1, Nc)) : 0u;
         cmask = (uint64_t)m0 | ((uint64_t)m1 << 32);
         active = cmask != 0;
       }
@@ -528,16 +562,16 @@ __global__ void __launch_bounds__(192, 2)
         const float2 s2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
         const float ps = s2.x + s2.y;
         if (centroid) {
-          // weight n_j = 64 except for the last block, which holds n_last tokens
+          // weight n_j = 64 bsub except for the last block, which holds nc_last tokens
           float pl = 0.f;
-          if ((-e - 1) == (N - 1) / 64 && n_last < 64) {
-            const int col = (N - 1) % 64;
+          if ((-e - 1) == (Nc - 1) / 64 && nc_last < 64 * bsub) {
+            const int col = (Nc - 1) % 64;
 #pragma unroll
             for (int i = 0; i < 64; ++i)
               if (i == col) pl = ex2_approx(fmaf(sv[i], sl2, neg));
           }
           a_run += ps;
-          l_run += 64.f * ps - (64.f - (float)n_last) * pl;
+          l_run += wblk * ps - (wblk - (float)nc_last) * pl;
         } else {
           l_run += ps;
         }

@@ -58,7 +58,7 @@ static pisa_status check_shape(int B, int H, int L, int d, int block_size) {
   if (B < 1 || H < 1 || L < 1 || d < 1 || block_size < 1) return PISA_ERR_INVALID_ARG;
   if ((long long)B * H > 65535) return PISA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return PISA_ERR_UNSUPPORTED;
-  if (block_size != 64) return PISA_ERR_UNSUPPORTED;
+  if (block_size != 64 && block_size != 128) return PISA_ERR_UNSUPPORTED;
   if ((long long)L > (1LL << 24)) return PISA_ERR_UNSUPPORTED;
   return PISA_OK;
 }
@@ -73,8 +73,8 @@ static bool sink_valid(int sink_idx) {
 }
 
 // ---- scratch sizes --------------------------------------------------------
-static size_t stats_ws(int B, int H, int L, int d) {
-  const int N = ceil_div(L, 64), BH = B * H;
+static size_t stats_ws(int B, int H, int L, int d, int block_size) {
+  const int N = ceil_div(L, block_size), BH = B * H;
   return align_up((size_t)BH * stats_num_chunks(BH, N) * d * d * sizeof(float), 256);
 }
 static size_t select_ws(int B, int H, int N) {
@@ -108,9 +108,9 @@ struct PathLayout {
   size_t qbar, kbar, vsum, hbar, cov, idx, scratch, total;
 };
 
-static PathLayout path_layout(int B, int H, int L, int d, double density, pisa_dtype dt,
-                              int want_cov) {
-  const int N = ceil_div(L, 64);
+static PathLayout path_layout(int B, int H, int L, int d, int block_size, double density,
+                              pisa_dtype dt, int want_cov) {
+  const int N = ceil_div(L, block_size);
   const size_t BH = (size_t)B * H;
   const int k_sel = pisa_num_selected(N, density);
   PathLayout p;
@@ -123,7 +123,7 @@ static PathLayout path_layout(int B, int H, int L, int d, double density, pisa_d
   p.cov = o; o += want_cov ? align_up(BH * N * sizeof(float), 256) : 0;
   p.idx = o; o += align_up(BH * N * (size_t)(k_sel > 0 ? k_sel : 1) * sizeof(int32_t), 256);
   p.scratch = o;
-  size_t s = stats_ws(B, H, L, d);
+  size_t s = stats_ws(B, H, L, d, block_size);
   s = s > select_ws(B, H, N) ? s : select_ws(B, H, N);
   const size_t a = sparse_ws(B, H, L, d, dt);
   s = s > a ? s : a;
@@ -141,10 +141,10 @@ static unsigned grid_1d(size_t n, int threads) {
 // ---- launches ---------------------------------------------------------------
 template <int D>
 static pisa_status launch_stats(const void *q, const void *k, const void *v, pisa_dtype dt,
-                                int BH, int L, int want_cov, float *qbar, float *kbar,
+                                int BH, int L, int sub, int want_cov, float *qbar, float *kbar,
                                 float *vsum, float *hbar, float *cov, float *partial,
                                 cudaStream_t st) {
-  const int N = ceil_div(L, 64);
+  const int N = ceil_div(L, 64 * sub);   // blocks of sub x 64 tokens
   const int nchunk = stats_num_chunks(BH, N);
   dim3 grid(nchunk, BH);
   if (dt == PISA_BF16) {
@@ -152,15 +152,15 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
     PISA_CUDA(cudaFuncSetAttribute(stats_pass_bf16_kernel<D>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     stats_pass_bf16_kernel<D><<<grid, kStatsThreads, smem, st>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N,
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N, sub,
         nchunk, qbar, kbar, vsum, partial);
   } else {
     const int smem = 3 * kBlk * D * (int)sizeof(float) + 3 * D * (int)sizeof(float);
     PISA_CUDA(cudaFuncSetAttribute(stats_pass_f32_kernel<D>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     stats_pass_f32_kernel<D><<<grid, kStatsThreads, smem, st>>>(
-        (const float *)q, (const float *)k, (const float *)v, L, N, nchunk, qbar, kbar, vsum,
-        partial);
+        (const float *)q, (const float *)k, (const float *)v, L, N, sub, nchunk, qbar, kbar,
+        vsum, partial);
   }
   PISA_TRY(check_launch());
   hbar_reduce_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(partial, nchunk, D * D, N,
@@ -172,14 +172,14 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
       PISA_CUDA(cudaFuncSetAttribute(cov_pass_bf16_kernel<D>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
       cov_pass_bf16_kernel<D><<<grid, kStatsThreads, smem, st>>>(
-          (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N, nchunk, kbar, vsum, hbar,
-          cov);
+          (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N, sub, nchunk, kbar, vsum,
+          hbar, cov);
     } else {
       const int smem = 2 * kBlk * D * (int)sizeof(float) + 32 * (int)sizeof(float);
       PISA_CUDA(cudaFuncSetAttribute(cov_pass_f32_kernel<D>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
       cov_pass_f32_kernel<D><<<dim3(N, BH), kStatsThreads, smem, st>>>(
-          (const float *)k, (const float *)v, L, N, kbar, vsum, hbar, cov);
+          (const float *)k, (const float *)v, L, N, sub, kbar, vsum, hbar, cov);
     }
     PISA_TRY(check_launch());
   }
@@ -245,12 +245,13 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
                                            const __nv_bfloat16 *v, const __nv_bfloat16 *kbar16,
                                            const __nv_bfloat16 *vsum16,
                                            const __nv_bfloat16 *hbar16, const int32_t *idx,
-                                           const int2 *pairs, int k_sel, int BH, int L,
+                                           const int2 *pairs, int k_sel, int BH, int L, int bsub,
                                            float scale, int hyd, int dense, int blockwise,
                                            void *out, int out_f32, float *lse,
                                            cudaStream_t st) {
-  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64;
-  const int smem = TcCfg<D>::smem_bytes(N);
+  const int N = ceil_div(L, 64);
+  const int Nc = ceil_div(L, 64 * bsub), Ncpad = ceil_div(Nc, 64) * 64;
+  const int smem = TcCfg<D>::smem_bytes(N, Nc);
   if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv, mkb, mvs, mh;
   PISA_TRY(make_map(&mq, q, D, L, BH, 64));
@@ -261,15 +262,15 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
     mvs = mv;
     mh = mk;
   } else {
-    PISA_TRY(make_map(&mkb, kbar16, D, Npad, BH, 64));
-    PISA_TRY(make_map(&mvs, vsum16, D, Npad, BH, 64));
+    PISA_TRY(make_map(&mkb, kbar16, D, Ncpad, BH, 64));
+    PISA_TRY(make_map(&mvs, vsum16, D, Ncpad, BH, 64));
     PISA_TRY(make_map(&mh, hbar16, D, D, BH, D));
   }
   PISA_CUDA(cudaFuncSetAttribute(piecewise_attention_tc_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   piecewise_attention_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), TcCfg<D>::kThreads, smem, st>>>(
-      mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, scale, hyd, dense, blockwise, out, out_f32,
-      lse);
+      mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, bsub, Nc, scale, hyd, dense, blockwise,
+      out, out_f32, lse);
   return check_launch();
 }
 
@@ -281,9 +282,13 @@ static pisa_status to_bf16(const void *src, __nv_bfloat16 *dst, size_t n, cudaSt
 static pisa_status run_sparse_attention(const void *q, const void *k, const void *v,
                                         pisa_dtype dt, const float *kbar, const float *vsum,
                                         const float *hbar, const int32_t *idx, int k_sel, int BH,
-                                        int L, int d, float scale, pisa_mode mode, void *out,
-                                        float *lse, unsigned char *ws, cudaStream_t st) {
-  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+                                        int L, int d, int bsub, float scale, pisa_mode mode,
+                                        void *out, float *lse, unsigned char *ws,
+                                        cudaStream_t st) {
+  // N 64-token tiles; Nc blocks of bsub tiles (the selection's and the
+  // centroids' index space); with bsub = 1 they coincide
+  const int N = ceil_div(L, 64), nwords = ceil_div(N, 32);
+  const int Nc = ceil_div(L, 64 * bsub), Ncpad = ceil_div(Nc, 64) * 64;
   const SparseLayout lay = sparse_layout(1, BH, L, d, dt);
   __nv_bfloat16 *kbar16 = (__nv_bfloat16 *)(ws + lay.kbar16);
   __nv_bfloat16 *vsum16 = (__nv_bfloat16 *)(ws + lay.vsum16);
@@ -291,22 +296,26 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   uint32_t *bm = (uint32_t *)(ws + lay.bm);
   uint16_t *ov = (uint16_t *)(ws + lay.ov);
   int2 *pairs = (int2 *)(ws + lay.pairs);
-  pack_stats_kernel<<<grid_1d((size_t)BH * (Npad * d + d * d), 256), 256, 0, st>>>(
-      kbar, vsum, hbar, N, Npad, d, BH, kbar16, vsum16, hbar16);
+  pack_stats_kernel<<<grid_1d((size_t)BH * (Ncpad * d + d * d), 256), 256, 0, st>>>(
+      kbar, vsum, hbar, Nc, Ncpad, d, BH, kbar16, vsum16, hbar16);
   PISA_TRY(check_launch());
-  // schedule: pair query blocks whose exact sets overlap most
-  selection_bitmap_kernel<<<dim3(N, BH), 64, nwords * sizeof(uint32_t), st>>>(idx, N, k_sel,
-                                                                              nwords, bm);
-  PISA_TRY(check_launch());
-  pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, nwords, ov);
-  PISA_TRY(check_launch());
-  const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
-  const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
-  if (pair_smem > 48 * 1024)
-    PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   pair_smem));
-  pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
-  PISA_TRY(check_launch());
+  if (bsub == 1) {
+    // schedule: pair query blocks whose exact sets overlap most
+    selection_bitmap_kernel<<<dim3(N, BH), 64, nwords * sizeof(uint32_t), st>>>(idx, N, k_sel,
+                                                                                nwords, bm);
+    PISA_TRY(check_launch());
+    pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, nwords, ov);
+    PISA_TRY(check_launch());
+    const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
+    const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
+    if (pair_smem > 48 * 1024)
+      PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     pair_smem));
+    pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
+    PISA_TRY(check_launch());
+  } else {
+    pairs = nullptr;   // the two 64-row halves of one 128-token query block share S_i
+  }
   const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
                       *v16 = (const __nv_bfloat16 *)v;
   if (dt == PISA_F32) {
@@ -326,9 +335,9 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   const int of32 = dt == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel,
-                                        BH, L, scale, hyd, 0, blockwise, out, of32, lse, st);
+                                        BH, L, bsub, scale, hyd, 0, blockwise, out, of32, lse, st);
   return launch_attention_kernel<64>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel, BH,
-                                     L, scale, hyd, 0, blockwise, out, of32, lse, st);
+                                     L, bsub, scale, hyd, 0, blockwise, out, of32, lse, st);
 }
 
 // ---- backward of the zeroth-order variant ------------------------------------
@@ -443,7 +452,7 @@ int pisa_num_selected(int N, double density) {
 
 size_t pisa_block_stats_workspace_bytes(int B, int H, int L, int d, int block_size) {
   if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
-  return stats_ws(B, H, L, d);
+  return stats_ws(B, H, L, d, block_size);
 }
 
 size_t pisa_select_workspace_bytes(int B, int H, int N) {
@@ -460,8 +469,8 @@ size_t pisa_sparse_attention_workspace_bytes(int B, int H, int L, int d, int blo
 size_t pisa_workspace_bytes(int B, int H, int L, int d, int block_size, double density,
                             pisa_dtype dtype, int want_cov) {
   if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
-  if (pisa_num_selected(ceil_div(L, 64), density) < 1) return 0;
-  return path_layout(B, H, L, d, density, dtype, want_cov).total;
+  if (pisa_num_selected(ceil_div(L, block_size), density) < 1) return 0;
+  return path_layout(B, H, L, d, block_size, density, dtype, want_cov).total;
 }
 
 pisa_status pisa_block_stats(const void *q, const void *k, const void *v, pisa_dtype dtype,
@@ -474,13 +483,14 @@ pisa_status pisa_block_stats(const void *q, const void *k, const void *v, pisa_d
       !aligned16(vsum) || !aligned16(hbar) || !aligned16(workspace))
     return PISA_ERR_INVALID_ARG;
   if (want_cov && !aligned16(cov)) return PISA_ERR_INVALID_ARG;
-  if (ws_bytes < stats_ws(B, H, L, d)) return PISA_ERR_WORKSPACE;
+  if (ws_bytes < stats_ws(B, H, L, d, block_size)) return PISA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   float *partial = (float *)workspace;
+  const int sub = block_size / 64;
   if (d == 128)
-    return launch_stats<128>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
-                             partial, st);
-  return launch_stats<64>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
+    return launch_stats<128>(q, k, v, dtype, B * H, L, sub, want_cov, qbar, kbar, vsum, hbar,
+                             cov, partial, st);
+  return launch_stats<64>(q, k, v, dtype, B * H, L, sub, want_cov, qbar, kbar, vsum, hbar, cov,
                           partial, st);
 }
 
@@ -512,7 +522,8 @@ static pisa_status sparse_attention_checked(const void *q, const void *k, const 
   PISA_TRY(check_shape(B, H, L, d, block_size));
   if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
   if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH && mode != PISA_MODE_1ST) return PISA_ERR_INVALID_ARG;
-  const int N = ceil_div(L, 64);
+  if (mode == PISA_MODE_1ST && block_size != 64) return PISA_ERR_UNSUPPORTED;
+  const int N = ceil_div(L, block_size);
   if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kbar) ||
@@ -521,8 +532,9 @@ static pisa_status sparse_attention_checked(const void *q, const void *k, const 
   if (out == q || out == k || out == v) return PISA_ERR_INVALID_ARG;
   if (ws_bytes < sparse_ws(B, H, L, d, dtype)) return PISA_ERR_WORKSPACE;
   const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
-  return run_sparse_attention(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B * H, L, d, s, mode,
-                              out, lse, (unsigned char *)workspace, (cudaStream_t)stream);
+  return run_sparse_attention(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B * H, L, d,
+                              block_size / 64, s, mode, out, lse, (unsigned char *)workspace,
+                              (cudaStream_t)stream);
 }
 
 pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, pisa_dtype dtype,
@@ -547,7 +559,7 @@ pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *
 }
 
 size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size) {
-  if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
+  if (check_shape(B, H, L, d, block_size) != PISA_OK || block_size != 64) return 0;
   return bwd_layout(B, H, L, d).total;
 }
 
@@ -558,6 +570,7 @@ pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *
                                       float scale, void *dq, void *dk, void *dv, void *workspace,
                                       size_t ws_bytes, pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, block_size));
+  if (block_size != 64) return PISA_ERR_UNSUPPORTED;
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
   if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
@@ -608,7 +621,8 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
   if (!sink_valid(sink_idx)) return PISA_ERR_INVALID_ARG;
   if (!(o.scale >= 0.f) || !std::isfinite(o.scale) || !std::isfinite(o.cov_weight))
     return PISA_ERR_INVALID_ARG;
-  const int N = ceil_div(L, 64);
+  if (mode == PISA_MODE_1ST && block_size != 64) return PISA_ERR_UNSUPPORTED;
+  const int N = ceil_div(L, block_size);
   const int k_sel = pisa_num_selected(N, density);
   if (k_sel < 1) return PISA_ERR_INVALID_ARG;
   if ((long long)N * 4 > 200 * 1024) return PISA_ERR_UNSUPPORTED;
@@ -616,7 +630,7 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
     return PISA_ERR_INVALID_ARG;
   if (out == q || out == k || out == v) return PISA_ERR_INVALID_ARG;
   const int want_cov = o.cov_weight != 0.f;
-  const PathLayout p = path_layout(B, H, L, d, density, o.dtype, want_cov);
+  const PathLayout p = path_layout(B, H, L, d, block_size, density, o.dtype, want_cov);
   cudaStream_t st = (cudaStream_t)stream;
   unsigned char *ws = (unsigned char *)o.workspace;
   bool owned = false;
@@ -637,18 +651,19 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
   int32_t *idx = (int32_t *)(ws + p.idx);
   unsigned char *scratch = ws + p.scratch;
   pisa_status r;
+  const int sub = block_size / 64;
   if (d == 128)
-    r = launch_stats<128>(q, k, v, o.dtype, BH, L, want_cov, qbar, kbar, vsum, hbar, cov,
+    r = launch_stats<128>(q, k, v, o.dtype, BH, L, sub, want_cov, qbar, kbar, vsum, hbar, cov,
                           (float *)scratch, st);
   else
-    r = launch_stats<64>(q, k, v, o.dtype, BH, L, want_cov, qbar, kbar, vsum, hbar, cov,
+    r = launch_stats<64>(q, k, v, o.dtype, BH, L, sub, want_cov, qbar, kbar, vsum, hbar, cov,
                          (float *)scratch, st);
   if (r == PISA_OK)
     r = launch_select(qbar, kbar, cov, o.cov_weight, s, BH, N, d, k_sel,
                       sink_block(sink_idx, N), idx, (float *)scratch, st);
   if (r == PISA_OK)
-    r = run_sparse_attention(q, k, v, o.dtype, kbar, vsum, hbar, idx, k_sel, BH, L, d, s, mode,
-                             out, nullptr, scratch, st);
+    r = run_sparse_attention(q, k, v, o.dtype, kbar, vsum, hbar, idx, k_sel, BH, L, d, sub, s,
+                             mode, out, nullptr, scratch, st);
   if (owned) {
     cudaError_t e = cudaFreeAsync(ws, st);
     if (e != cudaSuccess && r == PISA_OK) {
@@ -701,9 +716,9 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
   const int of32 = dtype == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr,
-                                        nullptr, 0, BH, L, s, 0, 1, 0, out, of32, nullptr, st);
+                                        nullptr, 0, BH, L, 1, s, 0, 1, 0, out, of32, nullptr, st);
   return launch_attention_kernel<64>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                     0, BH, L, s, 0, 1, 0, out, of32, nullptr, st);
+                                     0, BH, L, 1, s, 0, 1, 0, out, of32, nullptr, st);
 }
 
 pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v,
@@ -717,7 +732,7 @@ pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v
       !aligned16(vsum) || !aligned16(hbar))
     return PISA_ERR_INVALID_ARG;
   if (want_cov && !aligned16(cov)) return PISA_ERR_INVALID_ARG;
-  const size_t need = stats_ws(B, H, L, d);
+  const size_t need = stats_ws(B, H, L, d, block_size);
   if (need > (size_t)PISA_NOALLOC_SCRATCH_BYTES) {
     t_last_error = "pisa_block_stats_noalloc: this shape needs " + std::to_string(need) +
                    " bytes of scratch; the static array holds " +
@@ -728,10 +743,11 @@ pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v
   PISA_TRY(noalloc_scratch(&scratch));
   cudaStream_t st = (cudaStream_t)stream;
   float *partial = (float *)scratch;
+  const int sub = block_size / 64;
   if (d == 128)
-    return launch_stats<128>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
-                             partial, st);
-  return launch_stats<64>(q, k, v, dtype, B * H, L, want_cov, qbar, kbar, vsum, hbar, cov,
+    return launch_stats<128>(q, k, v, dtype, B * H, L, sub, want_cov, qbar, kbar, vsum, hbar,
+                             cov, partial, st);
+  return launch_stats<64>(q, k, v, dtype, B * H, L, sub, want_cov, qbar, kbar, vsum, hbar, cov,
                           partial, st);
 }
 
@@ -742,6 +758,7 @@ pisa_status pisa_tail_score_histogram(const void *q, const void *k, pisa_dtype d
                                       unsigned long long *hist_y, double *moments,
                                       pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, block_size));
+  if (block_size != 64) return PISA_ERR_UNSUPPORTED;
   if (dtype != PISA_BF16) return PISA_ERR_UNSUPPORTED;
   const int N = ceil_div(L, 64);
   if (k_sel < 1 || k_sel > N || nbins < 1 || nbins > 4096 || query_stride < 1)

@@ -59,6 +59,8 @@ def test_workspace_sizes(lib):
     # unsupported shapes report 0
     assert lib.pisa_workspace_bytes(1, 1, 1024, 96, 64, 0.25, L.PISA_BF16, 0) == 0
     assert lib.pisa_workspace_bytes(1, 1, 1024, 128, 32, 0.25, L.PISA_BF16, 0) == 0
+    assert lib.pisa_workspace_bytes(1, 1, 1024, 128, 128, 0.25, L.PISA_BF16, 0) > 0
+    assert lib.pisa_sparse_attention_bwd_workspace_bytes(1, 1, 1024, 128, 128) == 0
 
 
 def _attn(lib, q=0x1000, k=0x2000, v=0x3000, out=0x4000, B=1, H=1, Ln=128, d=128, bs=64,
@@ -72,7 +74,9 @@ def test_argument_checks_fail_before_any_launch(lib):
     assert _attn(lib, q=0x1001) == L.PISA_ERR_INVALID_ARG          # misaligned
     assert _attn(lib, out=0x1000) == L.PISA_ERR_INVALID_ARG        # out aliases q
     assert _attn(lib, d=96) == L.PISA_ERR_UNSUPPORTED
-    assert _attn(lib, bs=128) == L.PISA_ERR_UNSUPPORTED
+    assert _attn(lib, bs=96) == L.PISA_ERR_UNSUPPORTED
+    # block_size 128 is supported, but not by the block-wise first-order mode
+    assert _attn(lib, bs=128, mode=L.PISA_MODE_1ST) == L.PISA_ERR_UNSUPPORTED
     assert _attn(lib, Ln=0) == L.PISA_ERR_INVALID_ARG
     assert _attn(lib, dens=0.0) == L.PISA_ERR_INVALID_ARG
     assert _attn(lib, dens=1.5) == L.PISA_ERR_INVALID_ARG

@@ -32,7 +32,7 @@ def sample_blocks(N: int, n: int, seed: int):
     return sorted(set([0, N - 1] + [int(x) for x in mid]))
 
 
-@pytest.mark.parametrize("name", ["wan", "hunyuan", "flux"])
+@pytest.mark.parametrize("name", ["wan", "hunyuan", "flux", "wan_b128"])
 def test_fullsize_sampled(P, name):
     wl = WORKLOADS[name]
     Q, K, V = generate_qkv(wl, "cuda")

@@ -97,6 +97,27 @@ def test_ragged_and_degenerate(P, L, sink, mode, d):
     assert _run_case(P, wl) == 0
 
 
+@pytest.mark.parametrize("L,d,sink,mode,cov", [
+    (4608, 128, -1, "hyd", 0.1),    # FLUX-like shape, 36 blocks of 128 tokens
+    (1000, 128, None, "hyd", 0.0),  # last block 104 tokens: its second tile is partial
+    (4673, 128, -1, "0th", 0.1),    # last block 65 tokens: its second tile holds 1 token
+    (900, 64, 0, "hyd", 0.1),       # last block 4 tokens in one tile; odd tile count
+    (129, 128, -1, "hyd", 0.0),     # N = 2 with a one-token sink block
+    (100, 64, None, "0th", 0.0),    # N = 1
+])
+def test_block_size_128(P, L, d, sink, mode, cov):
+    """128-token blocks: statistics, selection and attention at block level,
+    exact tiles of 64 tokens, centroids with n_j = 128."""
+    wl = WORKLOADS["flux"].with_(B=2, H=2, L=L, d=d, block_size=128, sink_idx=sink, mode=mode,
+                                 cov_weight=cov, cluster_kind="block", density=0.2)
+    assert _run_case(P, wl) == 0
+
+
+def test_block_size_128_f32(P):
+    """f32 inputs with 128-token blocks (the f32 statistics kernels)."""
+    assert _run_case(P, WORKLOADS["tiny"].with_(block_size=128, cov_weight=0.1)) == 0
+
+
 @pytest.mark.parametrize("L,d,sink,cov", [(4608, 128, -1, 0.1), (1000, 128, None, 0.0),
                                           (777, 64, 0, 0.0)])
 def test_blockwise_first_order(P, L, d, sink, cov):

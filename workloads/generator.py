@@ -215,6 +215,15 @@ WORKLOADS = {
     "wan": Workload("wan", B=1, H=40, L=75600, d=128, block_size=64, density=0.125,
                     mode="hyd", sink_idx=None, dtype="bf16", cov_weight=0.0,
                     cluster_kind="video", grid=(21, 45, 80), seed=DEFAULT_SEED + 4),
+    # the FLUX and Wan shapes with 128-token blocks (the upper end of the block
+    # range the pages give)
+    "flux_b128": Workload("flux_b128", B=1, H=24, L=4608, d=128, block_size=128,
+                          density=0.15, mode="hyd", sink_idx=-1, dtype="bf16", cov_weight=0.1,
+                          cluster_kind="image", seed=DEFAULT_SEED + 2),
+    "wan_b128": Workload("wan_b128", B=1, H=40, L=75600, d=128, block_size=128,
+                         density=0.125, mode="hyd", sink_idx=None, dtype="bf16",
+                         cov_weight=0.0, cluster_kind="video", grid=(21, 45, 80),
+                         seed=DEFAULT_SEED + 4),
     # HunyuanVideo-13B 720p: 33 x 45 x 80 video tokens + 256 text tokens last
     "hunyuan": Workload("hunyuan", B=1, H=24, L=33 * 45 * 80 + 256, d=128,
                         block_size=64, density=0.10, mode="hyd", sink_idx=-1,
