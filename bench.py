@@ -48,8 +48,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the fused attention kernel, from an ncu capture,
 # keyed by the sha1 of the kernel source it was taken on (see profiles/).
 K3_TRAFFIC = {
-    # tcgen05 kernel, Wan-like H=4 ncu capture (303.2 MB read+write) scaled by heads
-    "8de7c1645474": {"wan": 3.032e9},
+    # H=4 ncu captures (dram read + write per launch) scaled by 10 to the 40 heads:
+    # Wan-like 301.4 MB, Wan-like with 128-token blocks 297.3 MB
+    "a1edd5427a78": {"wan": 3.014e9, "wan_b128": 2.973e9},
 }
 
 
