@@ -138,8 +138,10 @@ __device__ __forceinline__ void colsum_mma(uint32_t tiles, float *colsum, int wa
   }
 }
 
+// Two CTAs per SM (registers capped at 128): one CTA's loads stay in flight
+// while the other computes, which the HBM-bound pass needs.
 template <int D>
-__global__ void __launch_bounds__(kStatsThreads)
+__global__ void __launch_bounds__(kStatsThreads, 2)
     stats_pass_bf16_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
                            const __nv_bfloat16 *__restrict__ V, int L, int N, int sub, int nchunk,
                            float *__restrict__ qbar, float *__restrict__ kbar,
