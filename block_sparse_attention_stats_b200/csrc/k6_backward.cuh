@@ -16,13 +16,14 @@
 //   dkbar_j   = s sum_t dz_tj q_t,  dvbar_j = sum_t P_tj dout_t   (t with j in U_i)
 // The selection is a discrete step and is held fixed.
 //
-// Kernels (bf16 operands, f32 accumulation, mma.sync m16n8k16, 4 warps of 16
-// rows; tiles of 64 rows x D in XOR-swizzled shared memory, cp.async double
-// buffering):
+// Kernels of this file: bf16 operands, f32 accumulation, mma.sync m16n8k16,
+// 4 warps of 16 rows; tiles of 64 rows x D in XOR-swizzled shared memory,
+// cp.async double buffering.
 //   bwd_pack_centroids_kernel bf16 kbar_j and vbar_j (rows >= N zero)
-//   bwd_dq_kernel             one CTA per query block, two sweeps over its exact
-//                             blocks and every 64-centroid chunk masked to U_i:
-//                             Delta_t = sum_m P_tm dP_tm, then dq
+//   bwd_dq_tc_kernel          (k7_bwd_dq_tc.cuh, tcgen05) one CTA per pair of
+//                             query blocks, two sweeps over their exact tiles and
+//                             the centroid chunks: Delta_t = sum_m P_tm dP_tm,
+//                             then dq
 //   bwd_kv_kernel<CENT=true>  one CTA per 64-centroid chunk, over every query
 //                             block that leaves one of them unselected
 //                             -> dkbar_j / n_j, dvbar_j / n_j (float32)
@@ -145,163 +146,6 @@ __device__ __forceinline__ void bwd_c_to_a(const float (&c)[2 * KT][4], uint32_t
 __device__ __forceinline__ uint64_t bwd_valid_bits64(int c, int N) {   // centroids 64c.. < N
   const int n = N - 64 * c;
   return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
-}
-
-// ---------------------------------------------------------------------------
-// dq: one CTA per query block
-// ---------------------------------------------------------------------------
-template <int D> struct BwdDqCfg {
-  static constexpr int kTile = 64 * D * 2;
-  static constexpr int kSmem = 6 * kTile;   // Q, dO, 2 x (K, V)
-};
-
-template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 2)
-    bwd_dq_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
-                  const __nv_bfloat16 *__restrict__ V, const __nv_bfloat16 *__restrict__ dO,
-                  const float *__restrict__ lse, const __nv_bfloat16 *__restrict__ kbar16,
-                  const __nv_bfloat16 *__restrict__ vbar16, const int32_t *__restrict__ idx,
-                  const uint32_t *__restrict__ bm, int k_sel, int L, int N, int Npad, int nwords,
-                  float scale, float *__restrict__ delta, __nv_bfloat16 *__restrict__ dQ) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kT = BwdDqCfg<D>::kTile;
-  const uint32_t sb = smem_u32(smem);
-  const uint32_t sQ = sb, sdO = sb + kT;
-  const int i = blockIdx.x, bh = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, tq = lane & 3;
-  const size_t head = (size_t)bh * L * D;
-  const int nq = min(64, L - 64 * i);
-  const int C = (N + 63) / 64;
-  const int T = k_sel + C;          // tiles per sweep: exact blocks, then centroid chunks
-  const int32_t *row = idx + ((size_t)bh * N + i) * k_sel;
-  const uint32_t *bmrow = bm + ((size_t)bh * N + i) * nwords;
-  const int n_last = L - 64 * (N - 1);
-
-  auto block_of = [&](int t) -> int {
-    int j = row[t];
-    if (j < 0 || j >= N) {
-      report_device_error(kDevErrRange);
-      j = 0;
-    }
-    return j;
-  };
-  // two sweeps over the same T tiles: u < T computes Delta, u >= T computes dq
-  auto issue = [&](int u, int stage) {
-    const int t = u < T ? u : u - T;
-    const uint32_t dK = sb + (2 + 2 * stage) * kT, dV = dK + kT;
-    if (t < k_sel) {
-      const int j = block_of(t);
-      const int nv = min(64, L - 64 * j);
-      bwd_load_tile<D>(dK, K + head + (size_t)j * 64 * D, nv, tid);
-      bwd_load_tile<D>(dV, V + head + (size_t)j * 64 * D, nv, tid);
-    } else {
-      const size_t cb = ((size_t)bh * Npad + 64 * (t - k_sel)) * D;
-      bwd_load_tile<D>(dK, kbar16 + cb, 64, tid);
-      bwd_load_tile<D>(dV, vbar16 + cb, 64, tid);
-    }
-  };
-  bwd_load_tile<D>(sQ, Q + head + (size_t)i * 64 * D, nq, tid);
-  bwd_load_tile<D>(sdO, dO + head + (size_t)i * 64 * D, nq, tid);
-  issue(0, 0);
-  cp_async_commit();
-
-  const int rA = warp * 16 + g, rB = rA + 8;
-  const size_t tA = (size_t)bh * L + 64 * i + rA, tB = tA + 8;
-  const bool vA = 64 * i + rA < L, vB = 64 * i + rB < L;
-  const float sl2 = scale * kLog2e;
-  const float lA = vA ? lse[tA] * kLog2e : INFINITY, lB = vB ? lse[tB] * kLog2e : INFINITY;
-  // Delta_t = sum_m P_tm dP_tm over the row's augmented keys, from this
-  // kernel's own P and dP (equal to dout_t . o_t in exact arithmetic, and
-  // consistent with the P used below, so sum_m dz_tm vanishes to f32 rounding)
-  float dA = 0.f, dB = 0.f;
-
-  float acc[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-    for (int x = 0; x < 4; ++x) acc[n][x] = 0.f;
-
-  for (int u = 0; u < 2 * T; ++u) {
-    if (u + 1 < 2 * T) issue(u + 1, (u + 1) & 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const bool second = u >= T;
-    const int t = second ? u - T : u;
-    if (u == T) {
-      // end of the first sweep: complete the row sums across the quad
-      dA += __shfl_xor_sync(0xffffffffu, dA, 1);
-      dA += __shfl_xor_sync(0xffffffffu, dA, 2);
-      dB += __shfl_xor_sync(0xffffffffu, dB, 1);
-      dB += __shfl_xor_sync(0xffffffffu, dB, 2);
-      if (tq == 0) {
-        if (vA) delta[tA] = dA;
-        if (vB) delta[tB] = dB;
-      }
-    }
-    const uint32_t sK = sb + (2 + 2 * (u & 1)) * kT, sV = sK + kT;
-    // column weights: exact keys 1 (0 past the sequence end); centroids n_j
-    // for the blocks this query block left unselected, else 0
-    uint64_t keep;
-    float w_full, w_last = 0.f;
-    int last_col = -1;
-    if (t < k_sel) {
-      const int j = block_of(t);
-      const int nv = min(64, L - 64 * j);
-      keep = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
-      w_full = 1.f;
-    } else {
-      const int c = t - k_sel;
-      const uint32_t w0 = bmrow[2 * c];
-      const uint32_t w1 = 2 * c + 1 < nwords ? bmrow[2 * c + 1] : 0u;
-      keep = ~((uint64_t)w0 | ((uint64_t)w1 << 32)) & bwd_valid_bits64(c, N);
-      w_full = 64.f;
-      if (c == (N - 1) / 64) {
-        last_col = (N - 1) % 64;
-        w_last = (float)n_last;
-      }
-    }
-    float s[8][4], dp[8][4];
-    bwd_gemm_abt<D, 8>(s, sQ, warp * 16, sK, 0, lane);
-    bwd_gemm_abt<D, 8>(dp, sdO, warp * 16, sV, 0, lane);
-#pragma unroll
-    for (int n = 0; n < 8; ++n)
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int col = n * 8 + 2 * tq + (x & 1);
-        const bool hi = x >= 2;
-        float w = ((keep >> col) & 1ull) ? w_full : 0.f;
-        if (col == last_col) w = ((keep >> col) & 1ull) ? w_last : 0.f;
-        const float p = w * sm100::ex2_approx(fmaf(s[n][x], sl2, -(hi ? lB : lA)));
-        if (second) {
-          s[n][x] = p * (dp[n][x] - (hi ? dB : dA));   // dz
-        } else if (hi) {
-          dB = fmaf(p, dp[n][x], dB);
-        } else {
-          dA = fmaf(p, dp[n][x], dA);
-        }
-      }
-    if (second) {
-      uint32_t a[4][4];
-      bwd_c_to_a<4>(s, a);
-      bwd_gemm_ab<D, 4>(acc, a, sK, 0, lane);
-    }
-    __syncthreads();
-  }
-  cp_async_wait<0>();
-
-  // dq = s * acc
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n) {
-    const int col = n * 8 + 2 * tq;
-    if (vA)
-      *reinterpret_cast<uint32_t *>(dQ + tA * D + col) =
-          pack_bf16x2(scale * acc[n][0], scale * acc[n][1]);
-    if (vB)
-      *reinterpret_cast<uint32_t *>(dQ + tB * D + col) =
-          pack_bf16x2(scale * acc[n][2], scale * acc[n][3]);
-  }
 }
 
 // ---------------------------------------------------------------------------

@@ -1,0 +1,470 @@
+// dq of the zeroth-order backward on the sm_100a tensor cores (tcgen05).
+//
+// Same work unit as the fused forward: one CTA = two paired query blocks
+// (128 query rows, M = 128 MMAs) over the union of their exact tiles, then the
+// 64-centroid chunks masked per half to the half's unselected blocks.  With
+// P_tm = w_m exp(s q_t.key_m - lse_t) (w = 1 for exact keys, n_j for
+// centroids), dP_tm = dout_t . value_m and Delta_t = sum_m P_tm dP_tm:
+//   dq_t = s sum_m P_tm (dP_tm - Delta_t) key_m
+// The kernel makes two sweeps over the tile list: the first forms Delta_t
+// from its own P and dP (so that sum_m dz_tm vanishes to f32 rounding), the
+// second accumulates dq in tensor memory.
+//
+// Roles (320 threads):
+//   warp 0      TMA producer: Q and dout once, then K and V (or kbar and vbar)
+//               of every tile of both sweeps into 2-stage rings;
+//   warp 1      TMEM allocation; one elected lane issues every tcgen05.mma:
+//               S_u = Q K^T and dP_u = dout V^T into TMEM buffer u & 1, and in
+//               the second sweep dQ += dS_u K_u with dS read from TMEM;
+//   warps 2-9   two warpgroups of 4 warps; warpgroup g takes the tiles with
+//               u & 1 == g (buffer g), one thread per query row (TMEM lane):
+//               P and dP from TMEM, Delta partial sums (first sweep) or dS
+//               written back as bf16 over S (second sweep); the two Delta
+//               partials are combined through shared memory between sweeps;
+//               the epilogue scales dQ by s and stores it (half the columns
+//               each).
+// TMEM columns: dQ [0, D); buffer b: S [D + 128 b, D + 128 b + 64), dP the next
+// 64.  Every mbarrier wait is bounded; on a timeout the CTA records the error,
+// stops issuing, drains its copies and MMAs, frees TMEM and exits.
+#pragma once
+
+#include "pisa_common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace pisa {
+
+template <int D> struct DqTcCfg {
+  static constexpr int kThreads = 320;
+  static constexpr int kStages = 2;
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kBoxQBytes = 128 * 128;     // one 64-column box of 128 rows
+  static constexpr int kBoxKBytes = 64 * 128;      // one 64-column box of 64 rows
+  static constexpr int kTileBytes = 64 * D * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kQBytes;
+  static constexpr int kOffK = 2 * kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kNumBars = 16;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kOffMisc = kOffTmemSlot + 16;
+  static constexpr int kOffDelta = kOffMisc + 16;               // [2][128] f32
+  static constexpr int kOffDyn = kOffDelta + 2 * 128 * 4;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColDQ = 0;
+  static constexpr uint32_t kColBuf = D;                        // + 128 b
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKFull = 1;                           // + slot
+  static constexpr int kBarKEmpty = kBarKFull + kStages;
+  static constexpr int kBarVFull = kBarKEmpty + kStages;
+  static constexpr int kBarVEmpty = kBarVFull + kStages;
+  static constexpr int kBarSFull = kBarVEmpty + kStages;        // + buffer
+  static constexpr int kBarPFull = kBarSFull + 2;               // + buffer
+  static constexpr int kBarDelta = kBarPFull + 2;
+  static constexpr int kBarFinal = kBarDelta + 1;
+  static constexpr int kBarTeardown = kBarFinal + 1;
+  static_assert(kBarTeardown < kNumBars, "barrier slots");
+
+  __host__ __device__ static int smem_bytes(int N) {
+    const int nwords = (N + 31) / 32;
+    return kOffDyn + (2 * nwords + N + (N + 63) / 64) * 4 + 1024;   // + alignment slack
+  }
+};
+
+__device__ __forceinline__ uint32_t dq_valid_bits(int w, int N) {
+  const int lo = w * 32;
+  if (lo + 32 <= N) return 0xffffffffu;
+  if (lo >= N) return 0u;
+  return (1u << (N - lo)) - 1u;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_kbar,
+                     const __grid_constant__ CUtensorMap tm_vbar,
+                     const int32_t *__restrict__ idx, const int2 *__restrict__ pairs, int k_sel,
+                     int L, int N, float scale, const float *__restrict__ lse,
+                     float *__restrict__ delta_out, __nv_bfloat16 *__restrict__ dq) {
+  using C = DqTcCfg<D>;
+  using namespace sm100;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  unsigned char *smem = smem_raw + (sbase - raw);
+  auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
+  volatile int *misc = reinterpret_cast<volatile int *>(smem + C::kOffMisc);  // [0] tiles, [1] abort
+  float *delta_sm = reinterpret_cast<float *>(smem + C::kOffDelta);
+  const int nwords = (N + 31) / 32;
+  uint32_t *bm_lo = reinterpret_cast<uint32_t *>(smem + C::kOffDyn);
+  uint32_t *bm_hi = bm_lo + nwords;
+  int *tiles = reinterpret_cast<int *>(bm_hi + nwords);
+
+  const int pair = blockIdx.x, bh = blockIdx.y;
+  int qb0 = 2 * pair, qb1 = 2 * pair + 1 < N ? 2 * pair + 1 : -1;
+  if (pairs) {
+    const int2 pr = pairs[(size_t)bh * ((N + 1) / 2) + pair];
+    qb0 = pr.x;
+    qb1 = pr.y;
+  }
+  const bool has_hi = qb1 >= 0;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
+
+  // ---- set-up ---------------------------------------------------------------
+  if (warp == 1) {
+    tmem_alloc(sbase + C::kOffTmemSlot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar(C::kBarQ), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(C::kBarKFull + s), 1);
+      mbar_init(bar(C::kBarKEmpty + s), 1);
+      mbar_init(bar(C::kBarVFull + s), 1);
+      mbar_init(bar(C::kBarVEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::kBarSFull + b), 1);
+      mbar_init(bar(C::kBarPFull + b), 128);
+    }
+    mbar_init(bar(C::kBarDelta), 256);
+    mbar_init(bar(C::kBarFinal), 1);
+    mbar_init(bar(C::kBarTeardown), 1);
+    fence_mbar_init();
+    misc[1] = 0;
+  }
+  if (tid == 32) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_kbar);
+    prefetch_tmap(&tm_vbar);
+  }
+  for (int w = tid; w < 2 * nwords; w += C::kThreads) bm_lo[w] = 0u;
+  __syncthreads();
+  {
+    const int32_t *r0 = idx + ((size_t)bh * N + qb0) * k_sel;
+    const int32_t *r1 = idx + ((size_t)bh * N + (has_hi ? qb1 : qb0)) * k_sel;
+    for (int t = tid; t < (has_hi ? 2 : 1) * k_sel; t += C::kThreads) {
+      const int j = t < k_sel ? r0[t] : r1[t - k_sel];
+      uint32_t *bm = t < k_sel ? bm_lo : bm_hi;
+      if (j >= 0 && j < N) atomicOr(&bm[j >> 5], 1u << (j & 31));
+      else report_device_error(kDevErrRange);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exact tiles: ascending union of both halves' sets, with per-half flags
+    int base = 0;
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t lo = w < nwords ? bm_lo[w] : 0u, hi = w < nwords ? bm_hi[w] : 0u;
+      uint32_t u = lo | hi;
+      const int cnt = __popc(u);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int pos = base + incl - cnt;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1u;
+        tiles[pos++] = ((w * 32 + bit) << 2) | ((lo >> bit) & 1u) | (((hi >> bit) & 1u) << 1);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    // centroid chunks that hold an unselected block for either half
+    const int nch = (N + 63) / 64;
+    for (int c0 = 0; c0 < nch; c0 += 32) {
+      const int c = c0 + lane;
+      bool need = false;
+      if (c < nch) {
+        for (int h = 0; h < (has_hi ? 2 : 1); ++h) {
+          const uint32_t *bm = h ? bm_hi : bm_lo;
+          const uint32_t m0 = ~bm[2 * c] & dq_valid_bits(2 * c, N);
+          const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & dq_valid_bits(2 * c + 1, N)) : 0u;
+          need = need || ((m0 | m1) != 0u);
+        }
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, need);
+      if (need) tiles[base + __popc(bal & ((1u << lane) - 1u))] = -(c + 1);
+      base += __popc(bal);
+    }
+    if (lane == 0) misc[0] = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + C::kOffTmemSlot);
+  const int T = misc[0];
+  const int U = 2 * T;                 // both sweeps
+
+  auto uwait = [&](uint32_t b_addr, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(b_addr, parity));
+  };
+  auto aborted = [&]() -> bool { return __any_sync(0xffffffffu, misc[1] != 0); };
+
+  if (warp == 0) {
+    // ======================= TMA producer =====================================
+    if (elect_one()) {
+      mbar_expect_tx(bar(C::kBarQ), 2 * C::kQBytes);
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b) {
+        const uint32_t dq_ = sbase + C::kOffQ + b * C::kBoxQBytes;
+        const uint32_t dd_ = sbase + C::kOffDO + b * C::kBoxQBytes;
+        tma_load_3d(dq_, &tm_q, bar(C::kBarQ), 64 * b, qb0 * 64, bh);
+        tma_load_3d(dq_ + 64 * 128, &tm_q, bar(C::kBarQ), 64 * b, has_hi ? qb1 * 64 : L, bh);
+        tma_load_3d(dd_, &tm_do, bar(C::kBarQ), 64 * b, qb0 * 64, bh);
+        tma_load_3d(dd_ + 64 * 128, &tm_do, bar(C::kBarQ), 64 * b, has_hi ? qb1 * 64 : L, bh);
+      }
+    }
+    __syncwarp();
+    int issued = 0;
+    bool ok = true;
+    for (int u = 0; u < U; ++u) {
+      if (aborted()) { ok = false; break; }
+      const int sl = u % C::kStages;
+      if (u >= C::kStages) {
+        if (!uwait(bar(C::kBarKEmpty + sl), ((u / C::kStages) - 1) & 1)) { ok = false; break; }
+        if (!uwait(bar(C::kBarVEmpty + sl), ((u / C::kStages) - 1) & 1)) { ok = false; break; }
+      }
+      const int e = tiles[u < T ? u : u - T];
+      const CUtensorMap *mk = e >= 0 ? &tm_k : &tm_kbar;
+      const CUtensorMap *mv = e >= 0 ? &tm_v : &tm_vbar;
+      const int row = e >= 0 ? (e >> 2) * 64 : (-e - 1) * 64;
+      const uint32_t dk = sbase + C::kOffK + sl * C::kTileBytes;
+      const uint32_t dv = sbase + C::kOffV + sl * C::kTileBytes;
+      if (elect_one()) {
+        mbar_expect_tx(bar(C::kBarKFull + sl), C::kTileBytes);
+        mbar_expect_tx(bar(C::kBarVFull + sl), C::kTileBytes);
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b) {
+          tma_load_3d(dk + b * C::kBoxKBytes, mk, bar(C::kBarKFull + sl), 64 * b, row, bh);
+          tma_load_3d(dv + b * C::kBoxKBytes, mv, bar(C::kBarVFull + sl), 64 * b, row, bh);
+        }
+      }
+      __syncwarp();
+      issued = u + 1;
+    }
+    if (!ok) {
+      misc[1] = 1;
+      // let the copies already in flight land before the CTA exits
+      uwait(bar(C::kBarQ), 0);
+      for (int u = issued - C::kStages; u < issued; ++u)
+        if (u >= 0) {
+          uwait(bar(C::kBarKFull + u % C::kStages), (u / C::kStages) & 1);
+          uwait(bar(C::kBarVFull + u % C::kStages), (u / C::kStages) & 1);
+        }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================================
+    constexpr uint32_t kIdQK = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t kIdDQ = idesc_bf16_f32(128, D, 0, 1);
+    bool ok = uwait(bar(C::kBarQ), 0);
+    tc_fence_after();
+    auto a_desc = [&](uint32_t off, int k) -> uint64_t {
+      return smem_desc_sw128(sbase + off + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
+    };
+    // the second-sweep product for tile w once its dS is in TMEM; in the first
+    // sweep only the wait (buffer w & 1 is free again afterwards)
+    auto finish = [&](int w) -> bool {
+      const int b = w & 1, sl = w % C::kStages;
+      if (!uwait(bar(C::kBarPFull + b), (w >> 1) & 1)) return false;
+      if (w >= T) {
+        tc_fence_after();
+        const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tmem + C::kColDQ, tmem + C::kColBuf + 128 * b + kk * 8,
+                   smem_desc_sw128(kst + kk * 2048, C::kBoxKBytes, 1024), kIdDQ,
+                   (w > T || kk > 0) ? 1u : 0u);
+          tc_commit(bar(C::kBarKEmpty + sl));
+        }
+        __syncwarp();
+      }
+      return true;
+    };
+    for (int u = 0; ok && u < U; ++u) {
+      if (aborted()) { ok = false; break; }
+      const int sl = u % C::kStages, b = u & 1;
+      if (!uwait(bar(C::kBarKFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
+      if (!uwait(bar(C::kBarVFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
+      const uint32_t vst = sbase + C::kOffV + sl * C::kTileBytes;
+      if (elect_one()) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + C::kColBuf + 128 * b, a_desc(C::kOffQ, k),
+                 smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024), kIdQK,
+                 k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + C::kColBuf + 128 * b + 64, a_desc(C::kOffDO, k),
+                 smem_desc_sw128(vst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024), kIdQK,
+                 k > 0 ? 1u : 0u);
+        tc_commit(bar(C::kBarSFull + b));
+        tc_commit(bar(C::kBarVEmpty + sl));
+        if (u < T) tc_commit(bar(C::kBarKEmpty + sl));
+      }
+      __syncwarp();
+      if (u >= 1 && !finish(u - 1)) { ok = false; break; }
+    }
+    if (ok && U >= 1) ok = finish(U - 1);
+    if (ok) {
+      if (elect_one()) tc_commit(bar(C::kBarFinal));
+      __syncwarp();
+    }
+    if (!ok) {
+      misc[1] = 1;
+      // every MMA issued so far must finish before TMEM is released
+      if (elect_one()) tc_commit(bar(C::kBarTeardown));
+      __syncwarp();
+      uwait(bar(C::kBarTeardown), 0);
+    }
+  } else {
+    // ======================= dS warpgroups =====================================
+    const int g = (warp - 2) >> 2;               // warpgroup: tiles with u & 1 == g
+    const int sp = warp & 3;                     // TMEM sub-partition of this warp
+    const int row = sp * 32 + lane;              // query row in the tile = TMEM lane
+    const int half = row >> 6;
+    const bool exists = half == 0 || has_hi;
+    const int grow = (half ? qb1 : qb0) * 64 + (row & 63);
+    const bool valid = exists && grow < L;
+    const uint32_t *bm = half ? bm_hi : bm_lo;
+    const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
+    const uint32_t s_addr = lane_addr + C::kColBuf + 128 * g, dp_addr = s_addr + 64;
+    const float sl2 = scale * kLog2e;
+    const float lse2 = valid ? lse[(size_t)bh * L + grow] * kLog2e : INFINITY;
+    const int n_last = L - (N - 1) * 64;
+    float dpart = 0.f, dfull = 0.f;
+    bool exchanged = false, ok = true;
+    auto warp_wait = [&](uint32_t b_addr, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(b_addr, parity));
+    };
+    // combine the two warpgroups' Delta partial sums (once, before the first
+    // second-sweep tile of this warpgroup, or after its loop)
+    auto exchange = [&]() -> bool {
+      delta_sm[g * 128 + row] = dpart;
+      mbar_arrive(bar(C::kBarDelta));
+      if (!warp_wait(bar(C::kBarDelta), 0)) return false;
+      dfull = delta_sm[row] + delta_sm[128 + row];
+      if (g == 0 && valid) delta_out[(size_t)bh * L + grow] = dfull;
+      exchanged = true;
+      return true;
+    };
+    for (int u = g; u < U; u += 2) {
+      if (__any_sync(0xffffffffu, misc[1] != 0)) { ok = false; break; }
+      const bool second = u >= T;
+      if (second && !exchanged && !exchange()) { ok = false; break; }
+      if (!warp_wait(bar(C::kBarSFull + g), (u >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const int e = tiles[second ? u - T : u];
+      const bool centroid = e < 0;
+      uint64_t keep = 0ull;
+      float w_full = 1.f, w_last = 0.f;
+      int last_col = -1;
+      if (!exists) {
+        keep = 0ull;
+      } else if (!centroid) {
+        if ((e >> half) & 1) {
+          keep = ((e >> 2) == N - 1 && n_last < 64) ? ((1ull << n_last) - 1ull) : ~0ull;
+        }
+      } else {
+        const int c = -e - 1;
+        const uint32_t m0 = ~bm[2 * c] & dq_valid_bits(2 * c, N);
+        const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & dq_valid_bits(2 * c + 1, N)) : 0u;
+        keep = (uint64_t)m0 | ((uint64_t)m1 << 32);
+        w_full = 64.f;
+        if (c == (N - 1) / 64 && n_last < 64) {
+          last_col = (N - 1) % 64;
+          w_last = (float)n_last;
+        }
+      }
+      const bool active = __any_sync(0xffffffffu, keep != 0ull);
+      if (active) {
+        // 32 columns at a time; dS of columns 32h .. 32h+31 goes, packed, into
+        // TMEM columns 16h .. 16h+15 of the S buffer (already read)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t rs[32], rd[32], pk[16];
+          tmem_ld_x32(s_addr + 32 * h, rs);
+          tmem_ld_x32(dp_addr + 32 * h, rd);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float pz[2] = {0.f, 0.f};
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const int col = 32 * h + i + x;
+              const bool on = (keep >> col) & 1ull;
+              const float w = col == last_col ? w_last : w_full;
+              const float p = on ? w * ex2_approx(fmaf(__uint_as_float(rs[i + x]), sl2, -lse2))
+                                 : 0.f;
+              const float dp = __uint_as_float(rd[i + x]);
+              if (second) pz[x] = p * (dp - dfull);
+              else dpart = fmaf(p, dp, dpart);
+            }
+            pk[i / 2] = pack_bf16x2(pz[0], pz[1]);
+          }
+          if (second) tmem_st_x16(s_addr + 16 * h, pk);
+        }
+        if (second) tmem_wait_st();
+      } else if (second) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        tmem_st_x32(s_addr, pk);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarPFull + g));
+    }
+    if (ok && !exchanged) ok = exchange();
+    // ---- epilogue: dq = s dQ, this warpgroup's half of the columns ----------
+    if (ok && !__any_sync(0xffffffffu, misc[1] != 0)) {
+      if (!warp_wait(bar(C::kBarFinal), 0)) {
+        ok = false;
+      } else {
+        tc_fence_after();
+        const size_t obase = ((size_t)bh * L + (size_t)(valid ? grow : 0)) * D;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          const int col0 = g * (D / 2) + 32 * c;
+          uint32_t r[32];
+          tmem_ld_x32(lane_addr + C::kColDQ + col0, r);
+          tmem_wait_ld();
+          if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(dq + obase + col0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(
+                  pack_bf16x2(scale * __uint_as_float(r[8 * i]), scale * __uint_as_float(r[8 * i + 1])),
+                  pack_bf16x2(scale * __uint_as_float(r[8 * i + 2]), scale * __uint_as_float(r[8 * i + 3])),
+                  pack_bf16x2(scale * __uint_as_float(r[8 * i + 4]), scale * __uint_as_float(r[8 * i + 5])),
+                  pack_bf16x2(scale * __uint_as_float(r[8 * i + 6]), scale * __uint_as_float(r[8 * i + 7])));
+          }
+        }
+      }
+    }
+    if (!ok) misc[1] = 1;
+  }
+
+  // ---- teardown -----------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace pisa

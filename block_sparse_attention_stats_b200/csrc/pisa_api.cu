@@ -19,6 +19,7 @@
 #include "k3_attention_tc.cuh"
 #include "k5_tail_histogram.cuh"
 #include "k6_backward.cuh"
+#include "k7_bwd_dq_tc.cuh"
 
 namespace pisa {
 
@@ -342,7 +343,7 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
 
 // ---- backward of the zeroth-order variant ------------------------------------
 struct BwdLayout {
-  size_t delta, kbar16, vbar16, bm, dkbar, dvbar, total;
+  size_t delta, kbar16, vbar16, bm, ov, pairs, dkbar, dvbar, total;
 };
 static BwdLayout bwd_layout(int B, int H, int L, int d) {
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
@@ -353,6 +354,8 @@ static BwdLayout bwd_layout(int B, int H, int L, int d) {
   p.kbar16 = o; o += align_up(BH * Npad * d * 2, 256);
   p.vbar16 = o; o += align_up(BH * Npad * d * 2, 256);
   p.bm = o; o += align_up(BH * N * nwords * 4, 256);
+  p.ov = o; o += align_up(BH * N * kPairWindow * 2, 256);
+  p.pairs = o; o += align_up(BH * ((N + 1) / 2) * 8, 256);
   p.dkbar = o; o += align_up(BH * Npad * d * 4, 256);
   p.dvbar = o; o += align_up(BH * Npad * d * 4, 256);
   p.total = o;
@@ -369,18 +372,39 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   float *delta = (float *)(ws + lay.delta);
   const __nv_bfloat16 *kb = (const __nv_bfloat16 *)(ws + lay.kbar16);
   const __nv_bfloat16 *vb = (const __nv_bfloat16 *)(ws + lay.vbar16);
-  const uint32_t *bm = (const uint32_t *)(ws + lay.bm);
+  uint32_t *bm = (uint32_t *)(ws + lay.bm);
   float *dkbar = (float *)(ws + lay.dkbar), *dvbar = (float *)(ws + lay.dvbar);
-  const int dq_smem = BwdDqCfg<D>::kSmem, kv_smem = BwdKvCfg<D>::kSmem;
-  PISA_CUDA(cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // dq on the tensor cores: query blocks paired like the forward's
+  uint16_t *ov = (uint16_t *)(ws + lay.ov);
+  int2 *pairs = (int2 *)(ws + lay.pairs);
+  pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, nwords, ov);
+  PISA_TRY(check_launch());
+  const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
+  const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
+  if (pair_smem > 48 * 1024)
+    PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   pair_smem));
+  pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
+  PISA_TRY(check_launch());
+  const int dq_smem = DqTcCfg<D>::smem_bytes(N);
+  if (dq_smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
+  CUtensorMap mq, mdo, mk, mv, mkb, mvb;
+  PISA_TRY(make_map(&mq, q, D, L, BH, 64));
+  PISA_TRY(make_map(&mdo, dout, D, L, BH, 64));
+  PISA_TRY(make_map(&mk, k, D, L, BH, 64));
+  PISA_TRY(make_map(&mv, v, D, L, BH, 64));
+  PISA_TRY(make_map(&mkb, kb, D, Npad, BH, 64));
+  PISA_TRY(make_map(&mvb, vb, D, Npad, BH, 64));
+  PISA_CUDA(cudaFuncSetAttribute(bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dq_smem));
+  bwd_dq_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), DqTcCfg<D>::kThreads, dq_smem, st>>>(
+      mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, scale, lse, delta, dq);
+  PISA_TRY(check_launch());
+  const int kv_smem = BwdKvCfg<D>::kSmem;
   PISA_CUDA(cudaFuncSetAttribute(bwd_kv_kernel<D, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kv_smem));
   PISA_CUDA(cudaFuncSetAttribute(bwd_kv_kernel<D, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kv_smem));
-  bwd_dq_kernel<D><<<dim3(N, BH), kBwdThreads, dq_smem, st>>>(
-      q, k, v, dout, lse, kb, vb, idx, bm, k_sel, L, N, Npad, nwords, scale, delta, dq);
-  PISA_TRY(check_launch());
   bwd_kv_kernel<D, true><<<dim3(Npad / 64, BH), kBwdThreads, kv_smem, st>>>(
       q, k, v, dout, lse, delta, kb, vb, bm, L, N, Npad, nwords, scale, dkbar, dvbar, dk, dv);
   PISA_TRY(check_launch());
