@@ -10,21 +10,22 @@
 // from its own P and dP (so that sum_m dz_tm vanishes to f32 rounding), the
 // second accumulates dq in tensor memory.
 //
-// Roles (320 threads):
+// Roles (352 threads):
 //   warp 0      TMA producer: Q and dout once, then K and V (or kbar and vbar)
 //               of every tile of both sweeps into 2-stage rings;
-//   warp 1      TMEM allocation; one elected lane issues every tcgen05.mma:
-//               S_u = Q K^T and dP_u = dout V^T into TMEM buffer u & 1, and in
-//               the second sweep dQ += dS_u K_u with dS read from TMEM;
+//   warp 1      TMEM allocation; issues S_u = Q K^T into TMEM buffer u & 1;
+//   warp 10     issues dP_u = dout V^T into the same buffer and, in the second
+//               sweep, dQ += dS_u K_u with dS read from TMEM (one warp's issue
+//               rate would otherwise bound the kernel);
 //   warps 2-9   two warpgroups of 4 warps; warpgroup g takes the tiles with
 //               u & 1 == g (buffer g), one thread per query row (TMEM lane):
 //               P and dP from TMEM, Delta partial sums (first sweep) or dS
-//               written back as bf16 over S (second sweep); the two Delta
+//               written to a dS buffer as bf16 (second sweep); the two Delta
 //               partials are combined through shared memory between sweeps;
 //               the epilogue scales dQ by s and stores it (half the columns
 //               each).
 // TMEM columns: dQ [0, D); buffer b: S [D + 128 b, D + 128 b + 64), dP the next
-// 64.  Every mbarrier wait is bounded; on a timeout the CTA records the error,
+// 64; dS buffers (packed bf16) [D + 256 + 32 c, D + 256 + 32 c + 32).  Every mbarrier wait is bounded; on a timeout the CTA records the error,
 // stops issuing, drains its copies and MMAs, frees TMEM and exits.
 #pragma once
 
@@ -34,7 +35,7 @@
 namespace pisa {
 
 template <int D> struct DqTcCfg {
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;
   static constexpr int kStages = 2;
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kBoxQBytes = 128 * 128;     // one 64-column box of 128 rows
@@ -45,7 +46,7 @@ template <int D> struct DqTcCfg {
   static constexpr int kOffK = 2 * kQBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 20;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffMisc = kOffTmemSlot + 16;
   static constexpr int kOffDelta = kOffMisc + 16;               // [2][128] f32
@@ -53,6 +54,7 @@ template <int D> struct DqTcCfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColDQ = 0;
   static constexpr uint32_t kColBuf = D;                        // + 128 b
+  static constexpr uint32_t kColDS = D + 256;                   // + 32 b: packed bf16 dS
   static constexpr int kBarQ = 0;
   static constexpr int kBarKFull = 1;                           // + slot
   static constexpr int kBarKEmpty = kBarKFull + kStages;
@@ -60,7 +62,8 @@ template <int D> struct DqTcCfg {
   static constexpr int kBarVEmpty = kBarVFull + kStages;
   static constexpr int kBarSFull = kBarVEmpty + kStages;        // + buffer
   static constexpr int kBarPFull = kBarSFull + 2;               // + buffer
-  static constexpr int kBarDelta = kBarPFull + 2;
+  static constexpr int kBarDsFree = kBarPFull + 2;             // + dS buffer
+  static constexpr int kBarDelta = kBarDsFree + 2;
   static constexpr int kBarFinal = kBarDelta + 1;
   static constexpr int kBarTeardown = kBarFinal + 1;
   static_assert(kBarTeardown < kNumBars, "barrier slots");
@@ -79,7 +82,7 @@ __device__ __forceinline__ uint32_t dq_valid_bits(int w, int N) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_do,
                      const __grid_constant__ CUtensorMap tm_k,
@@ -128,12 +131,13 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(C::kBarVEmpty + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::kBarSFull + b), 1);
+      mbar_init(bar(C::kBarSFull + b), 2);       // S from warp 1, dP from warp 10
       mbar_init(bar(C::kBarPFull + b), 128);
+      mbar_init(bar(C::kBarDsFree + b), 1);
     }
     mbar_init(bar(C::kBarDelta), 256);
     mbar_init(bar(C::kBarFinal), 1);
-    mbar_init(bar(C::kBarTeardown), 1);
+    mbar_init(bar(C::kBarTeardown), 2);
     fence_mbar_init();
     misc[1] = 0;
   }
@@ -263,30 +267,38 @@ __global__ void __launch_bounds__(320, 1)
           uwait(bar(C::kBarVFull + u % C::kStages), (u / C::kStages) & 1);
         }
     }
-  } else if (warp == 1) {
-    // ======================= MMA issuer =======================================
+  } else if (warp == 1 || warp == 10) {
+    // ======================= MMA issuers ======================================
+    // One warp issues tcgen05.mma at a bounded rate, so the products are
+    // split: warp 1 issues S_u = Q K_u^T; warp 10 issues dP_u = dout V_u^T and,
+    // in the second sweep, dQ += dS_u K_u.  Buffer u & 1 is rewritten by S_u
+    // once the dS warpgroup has read tile u - 2 from it (PFull); dS lives in
+    // its own pair of buffers, released by the dQ products (DsFree).
     constexpr uint32_t kIdQK = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t kIdDQ = idesc_bf16_f32(128, D, 0, 1);
+    const bool s_warp = warp == 1;
     bool ok = uwait(bar(C::kBarQ), 0);
     tc_fence_after();
     auto a_desc = [&](uint32_t off, int k) -> uint64_t {
       return smem_desc_sw128(sbase + off + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
     };
-    // the second-sweep product for tile w once its dS is in TMEM; in the first
-    // sweep only the wait (buffer w & 1 is free again afterwards)
+    // warp 10: the second-sweep product for tile w once its dS is in TMEM (in
+    // the first sweep only the wait for the dS warpgroup)
     auto finish = [&](int w) -> bool {
       const int b = w & 1, sl = w % C::kStages;
       if (!uwait(bar(C::kBarPFull + b), (w >> 1) & 1)) return false;
       if (w >= T) {
         tc_fence_after();
+        const int db = (w - T) & 1;
         const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + C::kColDQ, tmem + C::kColBuf + 128 * b + kk * 8,
+            mma_ts(tmem + C::kColDQ, tmem + C::kColDS + 32 * db + kk * 8,
                    smem_desc_sw128(kst + kk * 2048, C::kBoxKBytes, 1024), kIdDQ,
                    (w > T || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::kBarKEmpty + sl));
+          tc_commit(bar(C::kBarDsFree + db));
         }
         __syncwarp();
       }
@@ -295,41 +307,49 @@ __global__ void __launch_bounds__(320, 1)
     for (int u = 0; ok && u < U; ++u) {
       if (aborted()) { ok = false; break; }
       const int sl = u % C::kStages, b = u & 1;
-      if (!uwait(bar(C::kBarKFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
-      if (!uwait(bar(C::kBarVFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
-      const uint32_t vst = sbase + C::kOffV + sl * C::kTileBytes;
-      if (elect_one()) {
+      if (s_warp) {
+        if (u >= 2 && !uwait(bar(C::kBarPFull + b), ((u - 2) >> 1) & 1)) { ok = false; break; }
+        if (!uwait(bar(C::kBarKFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + C::kColBuf + 128 * b, a_desc(C::kOffQ, k),
-                 smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024), kIdQK,
-                 k > 0 ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k)
+            mma_ss(tmem + C::kColBuf + 128 * b, a_desc(C::kOffQ, k),
+                   smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024),
+                   kIdQK, k > 0 ? 1u : 0u);
+          tc_commit(bar(C::kBarSFull + b));
+          if (u < T) tc_commit(bar(C::kBarKEmpty + sl));
+        }
+        __syncwarp();
+      } else {
+        if (!uwait(bar(C::kBarVFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t vst = sbase + C::kOffV + sl * C::kTileBytes;
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + C::kColBuf + 128 * b + 64, a_desc(C::kOffDO, k),
-                 smem_desc_sw128(vst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024), kIdQK,
-                 k > 0 ? 1u : 0u);
-        tc_commit(bar(C::kBarSFull + b));
-        tc_commit(bar(C::kBarVEmpty + sl));
-        if (u < T) tc_commit(bar(C::kBarKEmpty + sl));
+          for (int k = 0; k < D / 16; ++k)
+            mma_ss(tmem + C::kColBuf + 128 * b + 64, a_desc(C::kOffDO, k),
+                   smem_desc_sw128(vst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024),
+                   kIdQK, k > 0 ? 1u : 0u);
+          tc_commit(bar(C::kBarSFull + b));
+          tc_commit(bar(C::kBarVEmpty + sl));
+        }
+        __syncwarp();
+        if (u >= 1 && !finish(u - 1)) { ok = false; break; }
       }
-      __syncwarp();
-      if (u >= 1 && !finish(u - 1)) { ok = false; break; }
     }
-    if (ok && U >= 1) ok = finish(U - 1);
-    if (ok) {
+    if (!s_warp && ok && U >= 1) ok = finish(U - 1);
+    if (!s_warp && ok) {
+      // dQ is complete once warp 10's last product is (every dS waited on S)
       if (elect_one()) tc_commit(bar(C::kBarFinal));
       __syncwarp();
     }
-    if (!ok) {
-      misc[1] = 1;
-      // every MMA issued so far must finish before TMEM is released
-      if (elect_one()) tc_commit(bar(C::kBarTeardown));
-      __syncwarp();
-      uwait(bar(C::kBarTeardown), 0);
-    }
+    if (!ok) misc[1] = 1;
+    // before TMEM is released, every product either warp issued must finish
+    if (elect_one()) tc_commit(bar(C::kBarTeardown));
+    __syncwarp();
+    uwait(bar(C::kBarTeardown), 0);
   } else {
     // ======================= dS warpgroups =====================================
     const int g = (warp - 2) >> 2;               // warpgroup: tiles with u & 1 == g
@@ -369,6 +389,14 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const int e = tiles[second ? u - T : u];
       const bool centroid = e < 0;
+      // dS of second-sweep tile u goes to dS buffer (u - T) & 1, free once the
+      // dQ product of tile u - 2 has completed
+      const int r2 = u - T;
+      const uint32_t ds_addr = lane_addr + C::kColDS + 32 * (r2 & 1);
+      if (second && r2 >= 2 && !warp_wait(bar(C::kBarDsFree + (r2 & 1)), ((r2 - 2) >> 1) & 1)) {
+        ok = false;
+        break;
+      }
       uint64_t keep = 0ull;
       float w_full = 1.f, w_last = 0.f;
       int last_col = -1;
@@ -391,14 +419,17 @@ __global__ void __launch_bounds__(320, 1)
       }
       const bool active = __any_sync(0xffffffffu, keep != 0ull);
       if (active) {
-        // 32 columns at a time; dS of columns 32h .. 32h+31 goes, packed, into
-        // TMEM columns 16h .. 16h+15 of the S buffer (already read)
+        // all 64 S and 64 dP columns in one TMEM round trip; dS of columns
+        // 32h .. 32h+31 goes, packed, into dS-buffer columns 16h .. 16h+15
+        uint32_t r[4][32];   // S columns 0-31, 32-63, dP columns 0-31, 32-63
+        tmem_ld_x32(s_addr, r[0]);
+        tmem_ld_x32(s_addr + 32, r[1]);
+        tmem_ld_x32(dp_addr, r[2]);
+        tmem_ld_x32(dp_addr + 32, r[3]);
+        tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          uint32_t rs[32], rd[32], pk[16];
-          tmem_ld_x32(s_addr + 32 * h, rs);
-          tmem_ld_x32(dp_addr + 32 * h, rd);
-          tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             float pz[2] = {0.f, 0.f};
@@ -407,22 +438,22 @@ __global__ void __launch_bounds__(320, 1)
               const int col = 32 * h + i + x;
               const bool on = (keep >> col) & 1ull;
               const float w = col == last_col ? w_last : w_full;
-              const float p = on ? w * ex2_approx(fmaf(__uint_as_float(rs[i + x]), sl2, -lse2))
+              const float p = on ? w * ex2_approx(fmaf(__uint_as_float(r[h][i + x]), sl2, -lse2))
                                  : 0.f;
-              const float dp = __uint_as_float(rd[i + x]);
+              const float dp = __uint_as_float(r[2 + h][i + x]);
               if (second) pz[x] = p * (dp - dfull);
               else dpart = fmaf(p, dp, dpart);
             }
             pk[i / 2] = pack_bf16x2(pz[0], pz[1]);
           }
-          if (second) tmem_st_x16(s_addr + 16 * h, pk);
+          if (second) tmem_st_x16(ds_addr + 16 * h, pk);
         }
         if (second) tmem_wait_st();
       } else if (second) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = 0u;
-        tmem_st_x32(s_addr, pk);
+        tmem_st_x32(ds_addr, pk);
         tmem_wait_st();
       }
       tc_fence_before();
