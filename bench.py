@@ -521,7 +521,7 @@ def run_pisa(args, wl):
         P.pisa_sparse_attention_fwd(Q, K, V, stt["kbar"], stt["vsum"], stt["hbar"], idx, "0th",
                                     wl.block_size, out=out, lse=lse, workspace=k3_ws)
         bws = mk(lib.pisa_sparse_attention_bwd_workspace_bytes(wl.B, wl.H, wl.L, wl.d,
-                                                                wl.block_size))
+                                                                wl.block_size, idx.shape[-1]))
         grads = tuple(torch.empty_like(Q) for _ in range(3))
 
         def bstep():

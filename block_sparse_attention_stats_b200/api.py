@@ -199,7 +199,7 @@ def pisa_sparse_attention_bwd(q, k, v, dout, lse, kbar, vsum, idx, block_size: i
     B, H, Ln, d = _qkv_dims(q, k, v)
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
                                                   torch.empty_like(v))
-    need = lib.pisa_sparse_attention_bwd_workspace_bytes(B, H, Ln, d, block_size)
+    need = lib.pisa_sparse_attention_bwd_workspace_bytes(B, H, Ln, d, block_size, idx.shape[-1])
     ws = workspace if workspace is not None else _workspace(need, q.device)
     _check("pisa_sparse_attention_bwd", lib.pisa_sparse_attention_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(kbar), _ptr(vsum),

@@ -27,8 +27,11 @@
 //   bwd_kv_kernel<CENT=true>  one CTA per 64-centroid chunk, over every query
 //                             block that leaves one of them unselected
 //                             -> dkbar_j / n_j, dvbar_j / n_j (float32)
-//   bwd_kv_kernel<CENT=false> one CTA per key block j, over the query blocks
-//                             that selected it -> dk, dv, plus the centroid terms
+//   bwd_kv_tc_kernel          (k8_bwd_kv_tc.cuh, tcgen05) one CTA per pair of key
+//                             blocks, over the query blocks that selected either
+//                             -> dk, dv, plus the centroid terms
+//   bwd_kv_kernel<CENT=false> the same on mma.sync, one CTA per key block (kept
+//                             as the reference formulation; not launched)
 // No atomics: every output element is written by one CTA, so the results are
 // reproducible bit for bit.
 #pragma once
@@ -167,7 +170,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
                   const float *__restrict__ lse, const float *__restrict__ delta,
                   const __nv_bfloat16 *__restrict__ kbar16,
                   const __nv_bfloat16 *__restrict__ vbar16, const uint32_t *__restrict__ bm,
-                  int L, int N, int Npad, int nwords, float scale, float *__restrict__ dkbar,
+                  int L, int Lpad, int N, int Npad, int nwords, float scale,
+                  float *__restrict__ dkbar,
                   float *__restrict__ dvbar, __nv_bfloat16 *__restrict__ dK,
                   __nv_bfloat16 *__restrict__ dV) {
   using Cfg = BwdKvCfg<D>;
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
     bwd_load_tile<D>(dq, Q + head + (size_t)i * 64 * D, nq, tid);
     bwd_load_tile<D>(ddo, dO + head + (size_t)i * 64 * D, nq, tid);
     const int r = tid & 63;
-    const float *src = (tid < 64 ? lse : delta) + (size_t)bh * L + 64 * i;
+    const float *src = (tid < 64 ? lse : delta) + (size_t)bh * Lpad + 64 * i;
     const bool ok = r < nq;
     cp_async_4(smem_u32(vec + (stage * 2 + (tid >> 6)) * 64 + r), src + (ok ? r : 0), ok ? 4 : 0);
   };

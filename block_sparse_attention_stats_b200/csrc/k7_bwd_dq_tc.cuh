@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(352, 1)
                      const __grid_constant__ CUtensorMap tm_vbar,
                      const int32_t *__restrict__ idx, const int2 *__restrict__ pairs, int k_sel,
                      int L, int N, float scale, const float *__restrict__ lse,
-                     float *__restrict__ delta_out, __nv_bfloat16 *__restrict__ dq) {
+                     float *__restrict__ delta_out, int Lpad, __nv_bfloat16 *__restrict__ dq) {
   using C = DqTcCfg<D>;
   using namespace sm100;
   extern __shared__ unsigned char smem_raw[];
@@ -377,7 +377,8 @@ __global__ void __launch_bounds__(352, 1)
       mbar_arrive(bar(C::kBarDelta));
       if (!warp_wait(bar(C::kBarDelta), 0)) return false;
       dfull = delta_sm[row] + delta_sm[128 + row];
-      if (g == 0 && valid) delta_out[(size_t)bh * L + grow] = dfull;
+      // Delta into the padded [BH, Lpad] array (0 for rows past L)
+      if (g == 0 && exists) delta_out[(size_t)bh * Lpad + grow] = valid ? dfull : 0.f;
       exchanged = true;
       return true;
     };

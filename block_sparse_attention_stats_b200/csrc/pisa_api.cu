@@ -20,6 +20,7 @@
 #include "k5_tail_histogram.cuh"
 #include "k6_backward.cuh"
 #include "k7_bwd_dq_tc.cuh"
+#include "k8_bwd_kv_tc.cuh"
 
 namespace pisa {
 
@@ -343,23 +344,54 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
 
 // ---- backward of the zeroth-order variant ------------------------------------
 struct BwdLayout {
-  size_t delta, kbar16, vbar16, bm, ov, pairs, dkbar, dvbar, total;
+  size_t lse_pad, delta, kbar16, vbar16, bm, ov, pairs, dkbar, dvbar, counts, offsets, entries,
+      total;
+  long long cap;   // list entries per head
 };
-static BwdLayout bwd_layout(int B, int H, int L, int d) {
+static BwdLayout bwd_layout(int B, int H, int L, int d, int k_sel) {
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+  const int Lpad = N * 64, P = (N + 1) / 2;
   const size_t BH = (size_t)B * H;
   BwdLayout p;
   size_t o = 0;
-  p.delta = o; o += align_up(BH * L * 4, 256);
+  p.lse_pad = o; o += align_up(BH * Lpad * 4, 256);
+  p.delta = o; o += align_up(BH * Lpad * 4, 256);
   p.kbar16 = o; o += align_up(BH * Npad * d * 2, 256);
   p.vbar16 = o; o += align_up(BH * Npad * d * 2, 256);
   p.bm = o; o += align_up(BH * N * nwords * 4, 256);
   p.ov = o; o += align_up(BH * N * kPairWindow * 2, 256);
-  p.pairs = o; o += align_up(BH * ((N + 1) / 2) * 8, 256);
+  p.pairs = o; o += align_up(BH * P * 8, 256);
   p.dkbar = o; o += align_up(BH * Npad * d * 4, 256);
   p.dvbar = o; o += align_up(BH * Npad * d * 4, 256);
+  p.counts = o; o += align_up(BH * P * 4, 256);
+  p.offsets = o; o += align_up(BH * P * 8, 256);
+  // the lists of a head hold each selected (query block, key block) pair at most once
+  p.cap = (long long)N * k_sel;
+  p.entries = o; o += align_up(BH * (size_t)p.cap * 4, 256);
   p.total = o;
   return p;
+}
+
+// f32 [rows, cols] map with 64-element boxes of one row (per-row vectors)
+static pisa_status make_map_f32_rows(CUtensorMap *m, const void *base, uint64_t cols,
+                                     uint64_t rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) {
+    t_last_error = "cuTensorMapEncodeTiled is not available from the driver";
+    return PISA_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
+    return PISA_ERR_CUDA;
+  }
+  return PISA_OK;
 }
 
 template <int D>
@@ -369,11 +401,18 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                               const BwdLayout &lay, unsigned char *ws, __nv_bfloat16 *dq,
                               __nv_bfloat16 *dk, __nv_bfloat16 *dv, cudaStream_t st) {
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+  const int Lpad = N * 64, P = (N + 1) / 2;
+  float *lse_pad = (float *)(ws + lay.lse_pad);
   float *delta = (float *)(ws + lay.delta);
   const __nv_bfloat16 *kb = (const __nv_bfloat16 *)(ws + lay.kbar16);
   const __nv_bfloat16 *vb = (const __nv_bfloat16 *)(ws + lay.vbar16);
   uint32_t *bm = (uint32_t *)(ws + lay.bm);
   float *dkbar = (float *)(ws + lay.dkbar), *dvbar = (float *)(ws + lay.dvbar);
+  int *counts = (int *)(ws + lay.counts);
+  long long *offsets = (long long *)(ws + lay.offsets);
+  int *entries = (int *)(ws + lay.entries);
+  pad_lse_kernel<<<grid_1d((size_t)BH * Lpad, 256), 256, 0, st>>>(lse, L, Lpad, BH, lse_pad);
+  PISA_TRY(check_launch());
   // dq on the tensor cores: query blocks paired like the forward's
   uint16_t *ov = (uint16_t *)(ws + lay.ov);
   int2 *pairs = (int2 *)(ws + lay.pairs);
@@ -388,28 +427,43 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   PISA_TRY(check_launch());
   const int dq_smem = DqTcCfg<D>::smem_bytes(N);
   if (dq_smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
-  CUtensorMap mq, mdo, mk, mv, mkb, mvb;
+  CUtensorMap mq, mdo, mk, mv, mkb, mvb, mlse, mdel;
   PISA_TRY(make_map(&mq, q, D, L, BH, 64));
   PISA_TRY(make_map(&mdo, dout, D, L, BH, 64));
   PISA_TRY(make_map(&mk, k, D, L, BH, 64));
   PISA_TRY(make_map(&mv, v, D, L, BH, 64));
   PISA_TRY(make_map(&mkb, kb, D, Npad, BH, 64));
   PISA_TRY(make_map(&mvb, vb, D, Npad, BH, 64));
+  PISA_TRY(make_map_f32_rows(&mlse, lse_pad, Lpad, BH));
+  PISA_TRY(make_map_f32_rows(&mdel, delta, Lpad, BH));
   PISA_CUDA(cudaFuncSetAttribute(bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dq_smem));
-  bwd_dq_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), DqTcCfg<D>::kThreads, dq_smem, st>>>(
-      mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, scale, lse, delta, dq);
+  bwd_dq_tc_kernel<D><<<dim3(P, BH), DqTcCfg<D>::kThreads, dq_smem, st>>>(
+      mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, scale, lse, delta, Lpad, dq);
   PISA_TRY(check_launch());
+  // centroid gradients (mma.sync), then the exact keys' dk, dv on the tensor
+  // cores over the query-block lists of each key-block pair
   const int kv_smem = BwdKvCfg<D>::kSmem;
   PISA_CUDA(cudaFuncSetAttribute(bwd_kv_kernel<D, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kv_smem));
-  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_kernel<D, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kv_smem));
   bwd_kv_kernel<D, true><<<dim3(Npad / 64, BH), kBwdThreads, kv_smem, st>>>(
-      q, k, v, dout, lse, delta, kb, vb, bm, L, N, Npad, nwords, scale, dkbar, dvbar, dk, dv);
+      q, k, v, dout, lse_pad, delta, kb, vb, bm, L, Lpad, N, Npad, nwords, scale, dkbar, dvbar,
+      dk, dv);
   PISA_TRY(check_launch());
-  bwd_kv_kernel<D, false><<<dim3(N, BH), kBwdThreads, kv_smem, st>>>(
-      q, k, v, dout, lse, delta, kb, vb, bm, L, N, Npad, nwords, scale, dkbar, dvbar, dk, dv);
+  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, nwords, P, 0, counts, offsets, lay.cap,
+                                            entries);
+  PISA_TRY(check_launch());
+  kvlist_scan_kernel<<<BH, 1024, 0, st>>>(counts, P, offsets);
+  PISA_TRY(check_launch());
+  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, nwords, P, 1, counts, offsets, lay.cap,
+                                            entries);
+  PISA_TRY(check_launch());
+  const int kvtc_smem = KvTcCfg<D>::kSmem;
+  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kvtc_smem));
+  bwd_kv_tc_kernel<D><<<dim3(P, BH), KvTcCfg<D>::kThreads, kvtc_smem, st>>>(
+      mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, L, N, scale, dkbar, dvbar,
+      Npad, dk, dv);
   return check_launch();
 }
 
@@ -582,9 +636,11 @@ pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *
                                   block_size, scale, mode, out, lse, workspace, ws_bytes, stream);
 }
 
-size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size) {
+size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size,
+                                                 int k_sel) {
   if (check_shape(B, H, L, d, block_size) != PISA_OK || block_size != 64) return 0;
-  return bwd_layout(B, H, L, d).total;
+  if (k_sel < 1 || k_sel > ceil_div(L, 64)) return 0;
+  return bwd_layout(B, H, L, d, k_sel).total;
 }
 
 pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *v,
@@ -611,7 +667,7 @@ pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *
   if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(kbar) || !aligned16(vsum) ||
       !idx || !aligned16(workspace))
     return PISA_ERR_INVALID_ARG;
-  const BwdLayout lay = bwd_layout(B, H, L, d);
+  const BwdLayout lay = bwd_layout(B, H, L, d, k_sel);
   if (ws_bytes < lay.total) return PISA_ERR_WORKSPACE;
   const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
   const int BH = B * H;

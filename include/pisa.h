@@ -173,8 +173,10 @@ pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *
 
 /* ---- training: gradients of the zeroth-order variant ------------------------ */
 
-/* Workspace bytes of pisa_sparse_attention_bwd (0 on invalid arguments). */
-size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size);
+/* Workspace bytes of pisa_sparse_attention_bwd for k_sel selected blocks per
+ * query block (0 on invalid arguments). */
+size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size,
+                                                 int k_sel);
 
 /* Gradients of the zeroth-order forward (the authors' README, "Kernel
  * variants": piecewise_sparse_attention_0th "supports training"; the forward
