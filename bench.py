@@ -80,25 +80,45 @@ def dense_flops(wl):
     return 4.0 * wl.B * wl.H * wl.L * wl.L * wl.d
 
 
-def bwd_flops(wl, k_sel):
+def bwd_flops(wl, idx: torch.Tensor, heads: int = 2):
     """(algorithmic, executed) FLOPs of one zeroth-order backward.
 
     Algorithmic: five products per (query row, key) pair of the augmented
     softmax (recomputed logits q.k, dP = dout.value, dV += P dout, dK += dz q,
     dQ += dz k), 2 d FLOPs each, over the exact keys of S_i and the centroids of
-    U_i.  Executed: the kernels' 64 x 64 tiles, nine products per tile pair
-    (the dq kernel forms logits and dP twice: once for Delta, once for dq), plus
-    the padding of the last block and of the 64-centroid chunks."""
-    N = -(-wl.L // wl.block_size)
+    U_i.  Executed, replayed on `heads` heads and scaled: the dq kernel's
+    128 x 64 tiles over each query pair's union of exact tiles plus its centroid
+    chunks, five products each (logits and dP in both sweeps, dQ in the second);
+    the dk/dv kernel's 128 x 64 tiles over each key pair's union of query
+    blocks, four products each; the centroid kernel's 64 x 64 tiles over every
+    (chunk, query block) it visits, four products each."""
+    b, d = wl.block_size, wl.d
+    N = -(-wl.L // b)
     C = -(-N // 64)
     BH = wl.B * wl.H
-    # every query token sees k_sel exact blocks (counted as full blocks: a
-    # partial last block adds at most block_size keys per row too many) and
-    # N - k_sel centroids
-    pairs = wl.L * (k_sel * wl.block_size + (N - k_sel))
-    alg = BH * 10.0 * wl.d * pairs
-    execd = BH * 9.0 * 2 * 64 * 64 * wl.d * N * (k_sel + C)
-    return alg, execd
+    k_sel = idx.shape[-1]
+    pairs_alg = wl.L * (k_sel * b + (N - k_sel))
+    alg = BH * 10.0 * d * pairs_alg
+    idx_np = idx.reshape(-1, N, k_sel).cpu().numpy()
+    use = min(heads, idx_np.shape[0])
+    unit = 2.0 * 64 * 64 * d
+    tot = 0.0
+    for h in range(use):
+        bits = np.zeros((N, N), dtype=bool)
+        np.put_along_axis(bits, idx_np[h].astype(np.int64), True, axis=1)
+        for (i, j) in _pairs_like_kernel(bits):
+            sel = bits[i] | (bits[j] if j >= 0 else False)
+            chunks = sum(int((~bits[i, c * 64:min(N, c * 64 + 64)]).any() or
+                             (j >= 0 and (~bits[j, c * 64:min(N, c * 64 + 64)]).any()))
+                         for c in range(C))
+            tot += 5 * 2 * unit * (int(sel.sum()) + chunks)
+        for p in range(-(-N // 2)):
+            cols = bits[:, 2 * p] | (bits[:, 2 * p + 1] if 2 * p + 1 < N else False)
+            tot += 4 * 2 * unit * int(cols.sum())
+        for c in range(C):
+            need = (~bits[:, c * 64:min(N, c * 64 + 64)]).any(axis=1)
+            tot += 4 * unit * int(need.sum())
+    return alg, tot * BH / use
 
 
 def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
@@ -542,12 +562,13 @@ def run_pisa(args, wl):
         torch.cuda.synchronize()
         P.pisa_device_status()
         bms = sum(bev[2 * r_].elapsed_time(bev[2 * r_ + 1]) for r_ in range(reps)) / reps
-        f_alg_b, f_exec_b = bwd_flops(wl, idx.shape[-1])
+        f_alg_b, f_exec_b = bwd_flops(wl, idx)
         pk = _peaks()[0]
         p_sus_b = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-        bwd = {"ms": bms, "mode": "0th", "launches": 5,
-               "kernels": "pack_centroids, selection_bitmap, bwd_dq (2 sweeps), "
-                          "bwd_kv<centroid>, bwd_kv<exact> (mma.sync)",
+        bwd = {"ms": bms, "mode": "0th", "launches": 11,
+               "kernels": "dq: bwd_dq_tc (tcgen05, two sweeps); dk/dv of exact keys: "
+                          "bwd_kv_tc (tcgen05); centroid gradients: bwd_centroid (mma.sync); "
+                          "packing, bitmap, pairing, padding, list kernels",
                "roofline": {"bound": "tensor", "achieved": f_alg_b / (bms * 1e-3) / 1e12,
                             "peak": p_sus_b, "unit": "TFLOP/s",
                             "frac": f_alg_b / (bms * 1e-3) / 1e12 / p_sus_b,

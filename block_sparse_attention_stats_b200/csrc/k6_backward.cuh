@@ -24,14 +24,12 @@
 //                             query blocks, two sweeps over their exact tiles and
 //                             the centroid chunks: Delta_t = sum_m P_tm dP_tm,
 //                             then dq
-//   bwd_kv_kernel<CENT=true>  one CTA per 64-centroid chunk, over every query
+//   bwd_centroid_kernel       one CTA per 64-centroid chunk, over every query
 //                             block that leaves one of them unselected
 //                             -> dkbar_j / n_j, dvbar_j / n_j (float32)
 //   bwd_kv_tc_kernel          (k8_bwd_kv_tc.cuh, tcgen05) one CTA per pair of key
 //                             blocks, over the query blocks that selected either
 //                             -> dk, dv, plus the centroid terms
-//   bwd_kv_kernel<CENT=false> the same on mma.sync, one CTA per key block (kept
-//                             as the reference formulation; not launched)
 // No atomics: every output element is written by one CTA, so the results are
 // reproducible bit for bit.
 #pragma once
@@ -152,10 +150,9 @@ __device__ __forceinline__ uint64_t bwd_valid_bits64(int c, int N) {   // centro
 }
 
 // ---------------------------------------------------------------------------
-// dk, dv (CENT = false: one CTA per key block) and the centroid gradients
-// (CENT = true: one CTA per chunk of 64 centroids)
+// centroid gradients: one CTA per chunk of 64 centroids
 // ---------------------------------------------------------------------------
-template <int D> struct BwdKvCfg {
+template <int D> struct BwdCentCfg {
   static constexpr int kTile = 64 * D * 2;
   static constexpr int kOffVec = 6 * kTile;                 // lse, delta: 2 stages x 2 x 64 f32
   static constexpr int kOffList = kOffVec + 2 * 2 * 64 * 4;  // query-block list
@@ -163,18 +160,20 @@ template <int D> struct BwdKvCfg {
   static constexpr int kSmem = kOffWarp + 4 * 4;
 };
 
-template <int D, bool CENT>
+// The chunk's kbar_j / vbar_j tiles stay in shared memory; the CTA visits
+// every query block that leaves one of the chunk's centroids unselected
+// (lists built 1024 query blocks at a time).  lse and delta are the padded
+// [BH, Lpad] arrays (rows past L: lse +inf, delta 0).
+template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 2)
-    bwd_kv_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
-                  const __nv_bfloat16 *__restrict__ V, const __nv_bfloat16 *__restrict__ dO,
-                  const float *__restrict__ lse, const float *__restrict__ delta,
-                  const __nv_bfloat16 *__restrict__ kbar16,
-                  const __nv_bfloat16 *__restrict__ vbar16, const uint32_t *__restrict__ bm,
-                  int L, int Lpad, int N, int Npad, int nwords, float scale,
-                  float *__restrict__ dkbar,
-                  float *__restrict__ dvbar, __nv_bfloat16 *__restrict__ dK,
-                  __nv_bfloat16 *__restrict__ dV) {
-  using Cfg = BwdKvCfg<D>;
+    bwd_centroid_kernel(const __nv_bfloat16 *__restrict__ Q,
+                        const __nv_bfloat16 *__restrict__ dO, const float *__restrict__ lse,
+                        const float *__restrict__ delta, const __nv_bfloat16 *__restrict__ kbar16,
+                        const __nv_bfloat16 *__restrict__ vbar16,
+                        const uint32_t *__restrict__ bm, int L, int Lpad, int N, int Npad,
+                        int nwords, float scale, float *__restrict__ dkbar,
+                        float *__restrict__ dvbar) {
+  using Cfg = BwdCentCfg<D>;
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int kT = Cfg::kTile;
   const uint32_t sb = smem_u32(smem);
@@ -189,34 +188,21 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
   const int n_last = L - 64 * (N - 1);
   const float sl2 = scale * kLog2e;
 
-  // the fixed key-side tile
-  if (CENT) {
-    const size_t cb = ((size_t)bh * Npad + 64 * jb) * D;
-    bwd_load_tile<D>(sK, kbar16 + cb, 64, tid);
-    bwd_load_tile<D>(sV, vbar16 + cb, 64, tid);
-  } else {
-    const int nv = min(64, L - 64 * jb);
-    bwd_load_tile<D>(sK, K + head + (size_t)jb * 64 * D, nv, tid);
-    bwd_load_tile<D>(sV, V + head + (size_t)jb * 64 * D, nv, tid);
-  }
-  const int kA = warp * 16 + g, kB = kA + 8;       // this thread's key-side rows
-  // exact keys: weight 1 (0 past the sequence end); centroids: n_j when unselected
-  const float fixA = CENT ? (64 * jb + kA == N - 1 ? (float)n_last : 64.f)
-                          : (64 * jb + kA < L ? 1.f : 0.f);
-  const float fixB = CENT ? (64 * jb + kB == N - 1 ? (float)n_last : 64.f)
-                          : (64 * jb + kB < L ? 1.f : 0.f);
-  const uint64_t cvalid = CENT ? bwd_valid_bits64(jb, N) : 0ull;
+  const size_t cb = ((size_t)bh * Npad + 64 * jb) * D;
+  bwd_load_tile<D>(sK, kbar16 + cb, 64, tid);
+  bwd_load_tile<D>(sV, vbar16 + cb, 64, tid);
+  const int kA = warp * 16 + g, kB = kA + 8;       // this thread's centroid rows
+  const float fixA = 64 * jb + kA == N - 1 ? (float)n_last : 64.f;   // n_j
+  const float fixB = 64 * jb + kB == N - 1 ? (float)n_last : 64.f;
+  const uint64_t cvalid = bwd_valid_bits64(jb, N);
 
   auto selected_word = [&](int i, int w) -> uint32_t {
     return w < nwords ? bm[((size_t)bh * N + i) * nwords + w] : 0u;
   };
-  auto wants = [&](int i) -> bool {
-    if (CENT) {
-      const uint64_t sel = (uint64_t)selected_word(i, 2 * jb) |
-                           ((uint64_t)selected_word(i, 2 * jb + 1) << 32);
-      return (~sel & cvalid) != 0ull;
-    }
-    return (selected_word(i, jb >> 5) >> (jb & 31)) & 1u;
+  auto unselected = [&](int i) -> uint64_t {
+    const uint64_t sel = (uint64_t)selected_word(i, 2 * jb) |
+                         ((uint64_t)selected_word(i, 2 * jb + 1) << 32);
+    return ~sel & cvalid;
   };
   auto issue = [&](int i, int stage) {
     const uint32_t dq = sb + (2 + 2 * stage) * kT, ddo = dq + kT;
@@ -225,8 +211,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
     bwd_load_tile<D>(ddo, dO + head + (size_t)i * 64 * D, nq, tid);
     const int r = tid & 63;
     const float *src = (tid < 64 ? lse : delta) + (size_t)bh * Lpad + 64 * i;
-    const bool ok = r < nq;
-    cp_async_4(smem_u32(vec + (stage * 2 + (tid >> 6)) * 64 + r), src + (ok ? r : 0), ok ? 4 : 0);
+    cp_async_4(smem_u32(vec + (stage * 2 + (tid >> 6)) * 64 + r), src + r, 4);
   };
 
   float accK[D / 8][4], accV[D / 8][4];
@@ -244,7 +229,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int i = base + tid * 8 + r;
-      if (i < N && wants(i)) m |= 1u << r;
+      if (i < N && unselected(i) != 0ull) m |= 1u << r;
     }
     const int c = __popc(m);
     int x = c;
@@ -275,15 +260,9 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
       const int i = list[e];
       const uint32_t sQ = sb + (2 + 2 * st) * kT, sdO = sQ + kT;
       const float *ls = vec + (st * 2) * 64, *dl = vec + (st * 2 + 1) * 64;
-      float wA = fixA, wB = fixB;
-      if (CENT) {
-        const uint64_t sel = (uint64_t)selected_word(i, 2 * jb) |
-                             ((uint64_t)selected_word(i, 2 * jb + 1) << 32);
-        const uint64_t use = ~sel & cvalid;
-        if (!((use >> kA) & 1ull)) wA = 0.f;
-        if (!((use >> kB) & 1ull)) wB = 0.f;
-      }
-      const int nq = min(64, L - 64 * i);
+      const uint64_t use = unselected(i);
+      const float wA = ((use >> kA) & 1ull) ? fixA : 0.f;
+      const float wB = ((use >> kB) & 1ull) ? fixB : 0.f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float s[4][4], dp[4][4];
@@ -294,8 +273,10 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
 #pragma unroll
           for (int xx = 0; xx < 4; ++xx) {
             const int col = 32 * h + n * 8 + 2 * tq + (xx & 1);   // query row in block i
-            const float w = col < nq ? (xx >= 2 ? wB : wA) : 0.f;
-            const float p = w * sm100::ex2_approx(fmaf(s[n][xx], sl2, -ls[col] * kLog2e));
+            const float w = xx >= 2 ? wB : wA;
+            // padded query rows carry lse = +inf, so their probability is 0
+            const float p =
+                w != 0.f ? w * sm100::ex2_approx(fmaf(s[n][xx], sl2, -ls[col] * kLog2e)) : 0.f;
             s[n][xx] = p * (dp[n][xx] - dl[col]);   // dz
             dp[n][xx] = p;
           }
@@ -311,41 +292,21 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
   cp_async_commit();
   cp_async_wait<0>();
 
-  // ---- epilogue ---------------------------------------------------------------
+  // ---- epilogue: dkbar_j / n_j and dvbar_j / n_j (float32) -------------------
 #pragma unroll
   for (int hrow = 0; hrow < 2; ++hrow) {
-    const int kr = hrow ? kB : kA;
-    if (CENT) {
-      const int j = 64 * jb + kr;
-      if (j >= N) continue;
-      const float inv_n = 1.f / (j == N - 1 ? (float)n_last : 64.f);
-      float *pk = dkbar + ((size_t)bh * Npad + j) * D;
-      float *pv = dvbar + ((size_t)bh * Npad + j) * D;
+    const int j = 64 * jb + (hrow ? kB : kA);
+    if (j >= N) continue;
+    const float inv_n = 1.f / (j == N - 1 ? (float)n_last : 64.f);
+    float *pk = dkbar + ((size_t)bh * Npad + j) * D;
+    float *pv = dvbar + ((size_t)bh * Npad + j) * D;
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        const int col = n * 8 + 2 * tq;
-        *reinterpret_cast<float2 *>(pk + col) =
-            make_float2(scale * accK[n][2 * hrow] * inv_n, scale * accK[n][2 * hrow + 1] * inv_n);
-        *reinterpret_cast<float2 *>(pv + col) =
-            make_float2(accV[n][2 * hrow] * inv_n, accV[n][2 * hrow + 1] * inv_n);
-      }
-    } else {
-      const int tok = 64 * jb + kr;
-      if (tok >= L) continue;
-      const float *ck = dkbar + ((size_t)bh * Npad + jb) * D;
-      const float *cv = dvbar + ((size_t)bh * Npad + jb) * D;
-      __nv_bfloat16 *pk = dK + head + (size_t)tok * D;
-      __nv_bfloat16 *pv = dV + head + (size_t)tok * D;
-#pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        const int col = n * 8 + 2 * tq;
-        const float2 a = *reinterpret_cast<const float2 *>(ck + col);
-        const float2 b = *reinterpret_cast<const float2 *>(cv + col);
-        *reinterpret_cast<uint32_t *>(pk + col) =
-            pack_bf16x2(fmaf(scale, accK[n][2 * hrow], a.x), fmaf(scale, accK[n][2 * hrow + 1], a.y));
-        *reinterpret_cast<uint32_t *>(pv + col) =
-            pack_bf16x2(accV[n][2 * hrow] + b.x, accV[n][2 * hrow + 1] + b.y);
-      }
+    for (int n = 0; n < D / 8; ++n) {
+      const int col = n * 8 + 2 * tq;
+      *reinterpret_cast<float2 *>(pk + col) =
+          make_float2(scale * accK[n][2 * hrow] * inv_n, scale * accK[n][2 * hrow + 1] * inv_n);
+      *reinterpret_cast<float2 *>(pv + col) =
+          make_float2(accV[n][2 * hrow] * inv_n, accV[n][2 * hrow + 1] * inv_n);
     }
   }
 }

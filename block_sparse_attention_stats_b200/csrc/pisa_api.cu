@@ -443,12 +443,11 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   PISA_TRY(check_launch());
   // centroid gradients (mma.sync), then the exact keys' dk, dv on the tensor
   // cores over the query-block lists of each key-block pair
-  const int kv_smem = BwdKvCfg<D>::kSmem;
-  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_kernel<D, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kv_smem));
-  bwd_kv_kernel<D, true><<<dim3(Npad / 64, BH), kBwdThreads, kv_smem, st>>>(
-      q, k, v, dout, lse_pad, delta, kb, vb, bm, L, Lpad, N, Npad, nwords, scale, dkbar, dvbar,
-      dk, dv);
+  const int cent_smem = BwdCentCfg<D>::kSmem;
+  PISA_CUDA(cudaFuncSetAttribute(bwd_centroid_kernel<D>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, cent_smem));
+  bwd_centroid_kernel<D><<<dim3(Npad / 64, BH), kBwdThreads, cent_smem, st>>>(
+      q, dout, lse_pad, delta, kb, vb, bm, L, Lpad, N, Npad, nwords, scale, dkbar, dvbar);
   PISA_TRY(check_launch());
   kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, nwords, P, 0, counts, offsets, lay.cap,
                                             entries);
