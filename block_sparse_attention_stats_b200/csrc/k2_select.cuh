@@ -30,7 +30,7 @@ constexpr int kScoreTile = 128;
 constexpr int kScoreK = 16;
 constexpr int kScorePad = 4;
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
     scores_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar,
                   const float *__restrict__ cov, float cov_weight, float scale, int N, int D,
                   float *__restrict__ scores) {
@@ -47,21 +47,33 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
 
-  for (int e0 = 0; e0 < D; e0 += kScoreK) {
-    // 128 rows x 16 dims of each operand: two float4 per thread per operand
+  // 128 rows x 16 dims of each operand per chunk, two float4 per thread per
+  // operand; the next chunk is fetched into registers while this one is used
+  float4 pa[2], pb[2];
+  auto fetch = [&](int e0) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int t = tid + 256 * h;
       const int row = t >> 2, e4 = (t & 3) * 4;
       const int gi = i0 + row, gj = j0 + row;
-      const float4 a = gi < N ? *reinterpret_cast<const float4 *>(qb + (size_t)gi * D + e0 + e4)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 b = gj < N ? *reinterpret_cast<const float4 *>(kb + (size_t)gj * D + e0 + e4)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      pa[h] = gi < N ? *reinterpret_cast<const float4 *>(qb + (size_t)gi * D + e0 + e4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      pb[h] = gj < N ? *reinterpret_cast<const float4 *>(kb + (size_t)gj * D + e0 + e4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  fetch(0);
+  for (int e0 = 0; e0 < D; e0 += kScoreK) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int t = tid + 256 * h;
+      const int row = t >> 2, e4 = (t & 3) * 4;
+      const float4 a = pa[h], b = pb[h];
       As[e4 + 0][row] = a.x; As[e4 + 1][row] = a.y; As[e4 + 2][row] = a.z; As[e4 + 3][row] = a.w;
       Bs[e4 + 0][row] = b.x; Bs[e4 + 1][row] = b.y; Bs[e4 + 2][row] = b.z; Bs[e4 + 3][row] = b.w;
     }
     __syncthreads();
+    if (e0 + kScoreK < D) fetch(e0 + kScoreK);
 #pragma unroll
     for (int e = 0; e < kScoreK; ++e) {
       const float4 a0 = *reinterpret_cast<const float4 *>(&As[e][ty * 8]);
@@ -129,16 +141,26 @@ __global__ void __launch_bounds__(kTopkThreads)
 #pragma unroll
       for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0u;
       __syncwarp();
-      for (int j0 = 0; j0 < N; j0 += 32) {
-        const int j = j0 + lane;
-        const uint32_t key = j < N ? float_key(sc[j]) : 0u;
-        const bool part = j < N && j != sink && (key & mask) == prefix;
-        const unsigned act = __ballot_sync(0xffffffffu, part);
-        if (part) {
-          // aggregate lanes that hit the same bin into one shared-memory atomic
-          const unsigned digit = (key >> shift) & 255u;
-          const unsigned peers = __match_any_sync(act, digit);
-          if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+      for (int j0 = 0; j0 < N; j0 += 128) {
+        // four loads in flight per lane, then the four histogram updates
+        uint32_t kv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + 32 * u + lane;
+          kv[u] = j < N ? float_key(sc[j]) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + 32 * u + lane;
+          const uint32_t key = kv[u];
+          const bool part = j < N && j != sink && (key & mask) == prefix;
+          const unsigned act = __ballot_sync(0xffffffffu, part);
+          if (part) {
+            // aggregate lanes that hit the same bin into one shared-memory atomic
+            const unsigned digit = (key >> shift) & 255u;
+            const unsigned peers = __match_any_sync(act, digit);
+            if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+          }
         }
       }
       __syncwarp();
