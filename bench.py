@@ -140,12 +140,12 @@ def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
     return exact + tail + first
 
 
-PAIR_WINDOW = 16
+PAIR_WINDOW = 64
 
 
 def _pairs_like_kernel(bits: np.ndarray):
     """The fused kernel's query-block pairing (greedy, largest overlap of exact
-    sets within the next 16 blocks, nearer on ties), replayed on the host only to
+    sets within the next 64 blocks, nearer on ties), replayed on the host only to
     count the tensor-core tiles it issues."""
     N = bits.shape[0]
     used = np.zeros(N, dtype=bool)

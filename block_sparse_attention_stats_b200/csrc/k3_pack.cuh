@@ -51,9 +51,11 @@ __global__ void f32_to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 
 // the still-unpaired block among i+1 .. i+kPairWindow whose exact set shares
 // the most blocks with S_i (ties: the nearer one); when all of those are taken,
 // with the next unpaired block.  Only the schedule changes: every row still
-// sees exactly its own S_i and U_i.
+// sees exactly its own S_i and U_i.  On the Wan-like inputs the union of a
+// pair's exact sets averages 1.45 k_sel with adjacent pairs, 1.25 with a
+// window of 16 and 1.20 with 64.
 // ---------------------------------------------------------------------------
-constexpr int kPairWindow = 16;
+constexpr int kPairWindow = 64;
 
 // bm[bh][i][w]: bit j of word w set iff block 32w + j is in S_i.
 __global__ void selection_bitmap_kernel(const int32_t *__restrict__ idx, int N, int k_sel,
@@ -76,15 +78,17 @@ __global__ void pair_overlap_kernel(const uint32_t *__restrict__ bm, int N, int 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * (blockDim.x >> 5) + warp;
   const int bh = blockIdx.y;
-  if (i >= N || lane >= kPairWindow) return;
-  const int j = i + 1 + lane;
-  int cnt = 0;
-  if (j < N) {
-    const uint32_t *a = bm + ((size_t)bh * N + i) * nwords;
-    const uint32_t *b = bm + ((size_t)bh * N + j) * nwords;
-    for (int w = 0; w < nwords; ++w) cnt += __popc(a[w] & b[w]);
+  if (i >= N) return;
+  const uint32_t *a = bm + ((size_t)bh * N + i) * nwords;
+  for (int dd = lane; dd < kPairWindow; dd += 32) {
+    const int j = i + 1 + dd;
+    int cnt = 0;
+    if (j < N) {
+      const uint32_t *b = bm + ((size_t)bh * N + j) * nwords;
+      for (int w = 0; w < nwords; ++w) cnt += __popc(a[w] & b[w]);
+    }
+    ov[((size_t)bh * N + i) * kPairWindow + dd] = (uint16_t)cnt;
   }
-  ov[((size_t)bh * N + i) * kPairWindow + lane] = (uint16_t)cnt;
 }
 
 // One warp per head; pairs[bh][p] = (i0, i1), i1 = -1 for an unpaired block.
@@ -114,11 +118,14 @@ __global__ void pairing_kernel(const uint16_t *__restrict__ ov, int N, int stage
   int np = 0;
   for (int i = 0; i < N; ++i) {
     if (used[i]) continue;  // uniform: every lane reads the same byte
-    const int j = i + 1 + lane;
-    const bool cand = lane < kPairWindow && j < N && !used[j];
-    // key: overlap high, then nearer partner first
-    const int key = cand ? ((int)o[(size_t)i * kPairWindow + lane] << 8) | (255 - lane) : -1;
-    int best = key;
+    // key: overlap high, then nearer partner first; lane l looks at distances
+    // l + 1 and l + 33
+    int best = -1;
+    for (int dd = lane; dd < kPairWindow; dd += 32) {
+      const int j = i + 1 + dd;
+      if (j < N && !used[j])
+        best = max(best, ((int)o[(size_t)i * kPairWindow + dd] << 8) | (255 - dd));
+    }
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, s));
     int partner = -1;
