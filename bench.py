@@ -627,7 +627,11 @@ def run_pisa(args, wl):
     achieved = f_alg / (t_k3 * 1e-3) / 1e12
     src = _k3_source_hash()
     traffic = K3_TRAFFIC.get(src, {}).get(wl.name)
-    launches_per_step = 2 + (1 if want_cov else 0) + 2 + 2 + (3 if wl.dtype == "f32" else 0)
+    # statistics: pass 1 + hbar reduction (+ covariance pass); selection: scores +
+    # top-k; fused step: statistics packing (+ bitmap, overlaps, pairing with
+    # 64-token blocks) (+ three f32 -> bf16 copies) + the fused kernel
+    launches_per_step = (2 + (1 if want_cov else 0) + 2
+                         + (5 if wl.block_size == 64 else 2) + (3 if wl.dtype == "f32" else 0))
     line = {
         "metric": METRIC,
         "value": weak_scaling_value(world, dense_flops(wl), t_step),
