@@ -135,7 +135,13 @@ template <int D> struct KvTcCfg {
   static_assert(kBarTeardown < kNumBars, "barrier slots");
 };
 
-template <int D>
+// CENT = false: exact keys, as above.  CENT = true: the rows are 128
+// consecutive block centroids (kbar_j, vbar_j = vsum_j / n_j from the packed
+// centroid arrays) instead of keys; every query block is visited, a centroid
+// row takes weight n_j where the query block left block j unselected (0
+// elsewhere), and the epilogue writes dkbar_j / n_j and dvbar_j / n_j (float32)
+// for the exact pass's chain terms.
+template <int D, bool CENT>
 __global__ void __launch_bounds__(320, 1)
     bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_do,
@@ -144,8 +150,9 @@ __global__ void __launch_bounds__(320, 1)
                      const __grid_constant__ CUtensorMap tm_lse,
                      const __grid_constant__ CUtensorMap tm_delta,
                      const int *__restrict__ counts, const long long *__restrict__ offsets,
-                     long long cap, const int *__restrict__ entries, int L, int N, float scale,
-                     const float *__restrict__ dkbar, const float *__restrict__ dvbar, int Npad,
+                     long long cap, const int *__restrict__ entries,
+                     const uint32_t *__restrict__ bm, int nwords, int L, int N, float scale,
+                     float *__restrict__ dkbar, float *__restrict__ dvbar, int Npad,
                      __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV) {
   using C = KvTcCfg<D>;
   using namespace sm100;
@@ -159,9 +166,12 @@ __global__ void __launch_bounds__(320, 1)
 
   const int p = blockIdx.x, bh = blockIdx.y;
   const int P = (N + 1) / 2;
-  const int j0 = 2 * p, j1 = 2 * p + 1 < N ? 2 * p + 1 : -1;
-  const int T = counts[(size_t)bh * P + p];
-  const int *list = entries + bh * cap + offsets[(size_t)bh * P + p];
+  // row chunks (64 rows each) of this CTA: key blocks, or 64-centroid chunks
+  const int nchunk = CENT ? Npad / 64 : N;
+  const int j0 = 2 * p, j1 = 2 * p + 1 < nchunk ? 2 * p + 1 : -1;
+  const int T = CENT ? N : counts[(size_t)bh * P + p];
+  const int *list = CENT ? nullptr : entries + bh * cap + offsets[(size_t)bh * P + p];
+  const int row_end = CENT ? Npad : L;   // first row past the K / V (or centroid) rows
   const int tid = threadIdx.x, lane = tid & 31;
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
 
@@ -214,9 +224,9 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t dk = sbase + C::kOffK + b * C::kBoxPairBytes;
           const uint32_t dv = sbase + C::kOffV + b * C::kBoxPairBytes;
           tma_load_3d(dk, &tm_k, bar(C::kBarKV), 64 * b, j0 * 64, bh);
-          tma_load_3d(dk + 64 * 128, &tm_k, bar(C::kBarKV), 64 * b, j1 >= 0 ? j1 * 64 : L, bh);
+          tma_load_3d(dk + 64 * 128, &tm_k, bar(C::kBarKV), 64 * b, j1 >= 0 ? j1 * 64 : row_end, bh);
           tma_load_3d(dv, &tm_v, bar(C::kBarKV), 64 * b, j0 * 64, bh);
-          tma_load_3d(dv + 64 * 128, &tm_v, bar(C::kBarKV), 64 * b, j1 >= 0 ? j1 * 64 : L, bh);
+          tma_load_3d(dv + 64 * 128, &tm_v, bar(C::kBarKV), 64 * b, j1 >= 0 ? j1 * 64 : row_end, bh);
         }
       }
       __syncwarp();
@@ -227,7 +237,7 @@ __global__ void __launch_bounds__(320, 1)
           ok = false;
           break;
         }
-        const int i = list[u] >> 2;
+        const int i = CENT ? u : list[u] >> 2;
         if (elect_one()) {
           const uint32_t full = bar(C::kBarQFull + sl);
           mbar_expect_tx(full, 2 * C::kTileBytes + C::kVecBytes);
@@ -327,8 +337,9 @@ __global__ void __launch_bounds__(320, 1)
     const int row = sp * 32 + lane;              // key row in the tile = TMEM lane
     const int half = row >> 6;
     const int jb = half ? j1 : j0;
-    const int key = jb * 64 + (row & 63);
-    const bool kvalid = jb >= 0 && key < L;
+    const int key = jb * 64 + (row & 63);          // key token, or centroid index
+    const bool kvalid = jb >= 0 && key < (CENT ? N : L);
+    const float wn = (CENT && key == N - 1) ? (float)(L - 64 * (N - 1)) : 64.f;   // n_j
     const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
     const uint32_t s_addr = lane_addr + C::kColBuf + 128 * g, dp_addr = s_addr + 64;
     const float sl2 = scale * kLog2e;
@@ -338,11 +349,15 @@ __global__ void __launch_bounds__(320, 1)
     };
     for (int u = g; u < T; u += 2) {
       if (__any_sync(0xffffffffu, misc[1] != 0)) { ok = false; break; }
+      // centroid rows: was block `key` left unselected by query block u?
+      const uint32_t selw =
+          (CENT && kvalid) ? bm[((size_t)bh * N + u) * nwords + (key >> 5)] : 0u;
       if (!warp_wait(bar(C::kBarSFull + g), (u >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const int sl = u % C::kStages;
-      const int f = list[u] & 3;
-      const bool on = kvalid && ((f >> half) & 1);
+      const bool on = CENT ? (kvalid && !((selw >> (key & 31)) & 1u))
+                           : (kvalid && (((list[u] & 3) >> half) & 1));
+      const float wrow = CENT ? wn : 1.f;
       const float *ls = vec + sl * (C::kVecBytes / 4);     // lse of the 64 query rows
       const float *dl = ls + 64;                            // Delta of the 64 query rows
       uint32_t pp[32], pd[32];
@@ -363,8 +378,8 @@ __global__ void __launch_bounds__(320, 1)
             float pv[4], zv[4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-              const float pr = on ? ex2_approx(fmaf(__uint_as_float(r[h][i + x]), sl2,
-                                                    -lv[x] * kLog2e))
+              const float pr = on ? wrow * ex2_approx(fmaf(__uint_as_float(r[h][i + x]), sl2,
+                                                           -lv[x] * kLog2e))
                                   : 0.f;
               pv[x] = pr;
               zv[x] = pr * (__uint_as_float(r[2 + h][i + x]) - dv4[x]);
@@ -393,7 +408,35 @@ __global__ void __launch_bounds__(320, 1)
       if (!warp_wait(bar(C::kBarFinal), 0)) ok = false;
       else tc_fence_after();
     }
-    if (ok && !__any_sync(0xffffffffu, misc[1] != 0)) {
+    if (CENT && ok && !__any_sync(0xffffffffu, misc[1] != 0)) {
+      // dkbar_j / n_j = s dK / n_j, dvbar_j / n_j = dV / n_j
+      const float inv_n = 1.f / wn;
+      float *pk = dkbar + ((size_t)bh * Npad + (kvalid ? key : 0)) * D;
+      float *pv = dvbar + ((size_t)bh * Npad + (kvalid ? key : 0)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        const int col0 = g * (D / 2) + 32 * c;
+        uint32_t rk[32], rv[32];
+        tmem_ld_x32(lane_addr + C::kColDK + col0, rk);
+        tmem_ld_x32(lane_addr + C::kColDV + col0, rv);
+        tmem_wait_ld();
+        if (kvalid) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            reinterpret_cast<float4 *>(pk + col0)[i] =
+                make_float4(scale * inv_n * __uint_as_float(rk[4 * i]),
+                            scale * inv_n * __uint_as_float(rk[4 * i + 1]),
+                            scale * inv_n * __uint_as_float(rk[4 * i + 2]),
+                            scale * inv_n * __uint_as_float(rk[4 * i + 3]));
+            reinterpret_cast<float4 *>(pv + col0)[i] =
+                make_float4(inv_n * __uint_as_float(rv[4 * i]), inv_n * __uint_as_float(rv[4 * i + 1]),
+                            inv_n * __uint_as_float(rv[4 * i + 2]),
+                            inv_n * __uint_as_float(rv[4 * i + 3]));
+          }
+        }
+      }
+    }
+    if (!CENT && ok && !__any_sync(0xffffffffu, misc[1] != 0)) {
       const float *ck = dkbar + ((size_t)bh * Npad + (jb >= 0 ? jb : 0)) * D;
       const float *cv = dvbar + ((size_t)bh * Npad + (jb >= 0 ? jb : 0)) * D;
       const size_t obase = ((size_t)bh * L + (size_t)(kvalid ? key : 0)) * D;

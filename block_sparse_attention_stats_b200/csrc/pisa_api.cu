@@ -441,13 +441,17 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   bwd_dq_tc_kernel<D><<<dim3(P, BH), DqTcCfg<D>::kThreads, dq_smem, st>>>(
       mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, scale, lse, delta, Lpad, dq);
   PISA_TRY(check_launch());
-  // centroid gradients (mma.sync), then the exact keys' dk, dv on the tensor
-  // cores over the query-block lists of each key-block pair
-  const int cent_smem = BwdCentCfg<D>::kSmem;
-  PISA_CUDA(cudaFuncSetAttribute(bwd_centroid_kernel<D>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, cent_smem));
-  bwd_centroid_kernel<D><<<dim3(Npad / 64, BH), kBwdThreads, cent_smem, st>>>(
-      q, dout, lse_pad, delta, kb, vb, bm, L, Lpad, N, Npad, nwords, scale, dkbar, dvbar);
+  // centroid gradients, then the exact keys' dk, dv, both on the tensor cores
+  // (the exact pass over the query-block lists of each key-block pair)
+  const int kvtc_smem = KvTcCfg<D>::kSmem;
+  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_tc_kernel<D, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kvtc_smem));
+  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_tc_kernel<D, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kvtc_smem));
+  bwd_kv_tc_kernel<D, true><<<dim3(Npad / 128 + (Npad % 128 ? 1 : 0), BH), KvTcCfg<D>::kThreads,
+                              kvtc_smem, st>>>(
+      mq, mdo, mkb, mvb, mlse, mdel, nullptr, nullptr, 0, nullptr, bm, nwords, L, N, scale,
+      dkbar, dvbar, Npad, nullptr, nullptr);
   PISA_TRY(check_launch());
   kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, nwords, P, 0, counts, offsets, lay.cap,
                                             entries);
@@ -457,12 +461,9 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, nwords, P, 1, counts, offsets, lay.cap,
                                             entries);
   PISA_TRY(check_launch());
-  const int kvtc_smem = KvTcCfg<D>::kSmem;
-  PISA_CUDA(cudaFuncSetAttribute(bwd_kv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kvtc_smem));
-  bwd_kv_tc_kernel<D><<<dim3(P, BH), KvTcCfg<D>::kThreads, kvtc_smem, st>>>(
-      mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, L, N, scale, dkbar, dvbar,
-      Npad, dk, dv);
+  bwd_kv_tc_kernel<D, false><<<dim3(P, BH), KvTcCfg<D>::kThreads, kvtc_smem, st>>>(
+      mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, bm, nwords, L, N, scale,
+      dkbar, dvbar, Npad, dk, dv);
   return check_launch();
 }
 
