@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # keyed by the sha1 of the kernel source it was taken on (see profiles/).
 K3_TRAFFIC = {
     # H=4 ncu captures (dram read + write per launch) scaled by 10 to the 40 heads:
-    # Wan-like 301.4 MB, Wan-like with 128-token blocks 297.3 MB
-    "a1edd5427a78": {"wan": 3.014e9, "wan_b128": 2.973e9},
+    # Wan-like 300.7 MB, Wan-like with 128-token blocks 296.8 MB
+    "7974a8f98dec": {"wan": 3.007e9, "wan_b128": 2.968e9},
 }
 
 
