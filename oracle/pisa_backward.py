@@ -23,7 +23,7 @@ Sources (cited by page title and section):
   Transformers" (authors' README mirror), "Kernel variants": the _0th variant
   (zeroth-order tail only) is the one that supports backward for training.
 
-Readings (listed in the design doc): the gradient is that of the function the _0th
+Readings: the gradient is that of the function the _0th
 forward computes, selection held constant; lse_t = ln D_t (natural log, D_t
 as written, without any factored-out constant).
 """

@@ -33,7 +33,7 @@ Sources (cited by page title and section):
   variant, and [GS] "Global First-Order Correction": a distinct first-order
   term for every unselected block (memory-bound) -- mode "1st" below.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
 
 * softmax scale s = 1/sqrt(d) multiplies every q.k product (exact logits, the
   centroid logits, the selection scores and the first-order term s q Hbar);
