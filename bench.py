@@ -456,6 +456,29 @@ def run_pisa(args, wl):
     step_ms = [evs[2 * s].elapsed_time(evs[2 * s + 1]) for s in range(args.steps)]
     t_step = sum(step_ms) / len(step_ms)
 
+    # ---- the same step replayed from a CUDA graph (launch gaps removed) -------
+    graph = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            step()
+        torch.cuda.synchronize()
+        greps = max(3, min(args.steps, 10))
+        gev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * greps)]
+        for r_ in range(greps):
+            if l2_flush is not None:
+                l2_flush.zero_()
+            gev[2 * r_].record(stream)
+            g.replay()
+            gev[2 * r_ + 1].record(stream)
+        torch.cuda.synchronize()
+        graph = {"ms_per_step": sum(gev[2 * r_].elapsed_time(gev[2 * r_ + 1])
+                                    for r_ in range(greps)) / greps,
+                 "replays": greps}
+        del g
+
     # ---- per-kernel breakdown (same kernels, step by step through the C ABI) --
     lib = _lib.load()
     mk = lambda n: torch.empty(max(256, int(n)), dtype=torch.uint8, device=dev)
@@ -690,6 +713,7 @@ def run_pisa(args, wl):
                                    / (peaks.get("hbm_gbs", 6650.0) * 1e9)),
         },
         "dense_baseline": dense,
+        "graph_replay": graph,
         "tail_diagnostic": diag,
         "backward_0th": bwd,
         "gpu_launches": launches_per_step * args.steps,
@@ -727,6 +751,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip timing the step replayed from a CUDA graph")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip timing the zeroth-order backward")
     ap.add_argument("--no-diagnostic", action="store_true",
