@@ -697,6 +697,21 @@ def run_pisa(args, wl):
         "dtype": "bf16" if wl.dtype == "bf16" else "f32-in/bf16-mma",
         "data": "synthetic", "config": _config(wl),
         "kernels_ms": part_ms,
+        "ms_per_step_median": statistics.median(step_ms),
+        "kernels_roofline": {
+            # statistics: HBM-bound (reads Q, K, V once, K and V again with the
+            # covariance pass); selection: on chip (the N x N fp32 score
+            # contraction and the radix top-k)
+            "block_stats": {"bound": "hbm", "bytes": stats_bytes(wl),
+                            "achieved_gbs": stats_bytes(wl) / (part_ms["block_stats"] * 1e-3) / 1e9,
+                            "peak_gbs": peaks.get("hbm_gbs", 6650.0),
+                            "frac": stats_bytes(wl) / (part_ms["block_stats"] * 1e-3) / 1e9
+                            / peaks.get("hbm_gbs", 6650.0)},
+            "select": {"bound": "on-chip (fp32 score contraction, top-k)",
+                       "score_gflop": 2.0 * wl.B * wl.H * N * N * wl.d / 1e9,
+                       "score_tflops": 2.0 * wl.B * wl.H * N * N * wl.d
+                       / (part_ms["select"] * 1e-3) / 1e12},
+        },
         "roofline": {
             "kernel": "piecewise_attention (fused exact + centroid tail + first-order)",
             "bound": "tensor", "achieved": achieved, "peak": p_sus,
