@@ -65,6 +65,20 @@ static pisa_status check_shape(int B, int H, int L, int d, int block_size) {
   return PISA_OK;
 }
 
+// Shared memory of the fused kernel grows with the number of blocks (selection
+// bitmaps and the tile list); shapes beyond the 227 KB a CTA can hold are
+// refused before anything is launched.
+static bool fused_fits(int d, int L, int block_size) {
+  const int N = ceil_div(L, 64), Nc = ceil_div(L, block_size);
+  const int smem = d == 128 ? TcCfg<128>::smem_bytes(N, Nc) : TcCfg<64>::smem_bytes(N, Nc);
+  return smem <= 227 * 1024;
+}
+static bool bwd_fits(int d, int L) {
+  const int N = ceil_div(L, 64);
+  const int smem = d == 128 ? DqTcCfg<128>::smem_bytes(N) : DqTcCfg<64>::smem_bytes(N);
+  return smem <= 227 * 1024;
+}
+
 static int sink_block(int sink_idx, int N) {
   if (sink_idx == PISA_SINK_NONE) return -1;
   return sink_idx == 0 ? 0 : N - 1;
@@ -601,6 +615,7 @@ static pisa_status sparse_attention_checked(const void *q, const void *k, const 
   if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
   if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH && mode != PISA_MODE_1ST) return PISA_ERR_INVALID_ARG;
   if (mode == PISA_MODE_1ST && block_size != 64) return PISA_ERR_UNSUPPORTED;
+  if (!fused_fits(d, L, block_size)) return PISA_ERR_UNSUPPORTED;
   const int N = ceil_div(L, block_size);
   if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
@@ -651,6 +666,7 @@ pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *
                                       size_t ws_bytes, pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, block_size));
   if (block_size != 64) return PISA_ERR_UNSUPPORTED;
+  if (!bwd_fits(d, L)) return PISA_ERR_UNSUPPORTED;
   const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
   if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
@@ -702,6 +718,7 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
   if (!(o.scale >= 0.f) || !std::isfinite(o.scale) || !std::isfinite(o.cov_weight))
     return PISA_ERR_INVALID_ARG;
   if (mode == PISA_MODE_1ST && block_size != 64) return PISA_ERR_UNSUPPORTED;
+  if (!fused_fits(d, L, block_size)) return PISA_ERR_UNSUPPORTED;
   const int N = ceil_div(L, block_size);
   const int k_sel = pisa_num_selected(N, density);
   if (k_sel < 1) return PISA_ERR_INVALID_ARG;
@@ -771,6 +788,7 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
                                  void *workspace, size_t ws_bytes, pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, 64));
   if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
+  if (!fused_fits(d, L, 64)) return PISA_ERR_UNSUPPORTED;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return PISA_ERR_INVALID_ARG;
@@ -850,11 +868,11 @@ pisa_status pisa_tail_score_histogram(const void *q, const void *k, pisa_dtype d
     return PISA_ERR_INVALID_ARG;
   const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
   cudaStream_t st = (cudaStream_t)stream;
+  const int smem = 3 * 64 * d * 2 + 8 * (nbins + 2) * 4 + ceil_div(N, 32) * 4;
+  if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
   PISA_CUDA(cudaMemsetAsync(hist_x, 0, sizeof(unsigned long long) * (nbins + 2), st));
   PISA_CUDA(cudaMemsetAsync(hist_y, 0, sizeof(unsigned long long) * (nbins + 2), st));
   PISA_CUDA(cudaMemsetAsync(moments, 0, sizeof(double) * 5, st));
-  const int smem = 3 * 64 * d * 2 + 8 * (nbins + 2) * 4 + ceil_div(N, 32) * 4;
-  if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
   dim3 grid(ceil_div(N, query_stride), B * H);
   const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k;
   if (d == 128) {

@@ -77,6 +77,12 @@ def test_argument_checks_fail_before_any_launch(lib):
     assert _attn(lib, out=0x1000) == L.PISA_ERR_INVALID_ARG        # out aliases q
     assert _attn(lib, d=96) == L.PISA_ERR_UNSUPPORTED
     assert _attn(lib, bs=96) == L.PISA_ERR_UNSUPPORTED
+    # size limits, refused before any launch: more than 65535 (batch, head) pairs,
+    # more than 2^24 tokens, a selection row that no longer fits on chip
+    assert _attn(lib, B=2, H=40000) == L.PISA_ERR_UNSUPPORTED
+    assert _attn(lib, Ln=(1 << 24) + 1) == L.PISA_ERR_UNSUPPORTED
+    assert _attn(lib, Ln=64 * 60000) == L.PISA_ERR_UNSUPPORTED
+    assert _attn(lib, Ln=64 * 40000, dens=0.01) == L.PISA_ERR_UNSUPPORTED   # fused kernel
     # block_size 128 is supported, but not by the block-wise first-order mode
     assert _attn(lib, bs=128, mode=L.PISA_MODE_1ST) == L.PISA_ERR_UNSUPPORTED
     assert _attn(lib, Ln=0) == L.PISA_ERR_INVALID_ARG
