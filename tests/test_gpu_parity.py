@@ -206,3 +206,25 @@ def test_pisa_attention_default_entry_point(P):
     b = P.pisa_attention_ex(Q, K, V, wl.density, 64, wl.sink_idx, "hyd", workspace=ws)
     P.pisa_device_status()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("block_size,mode", [(64, "hyd"), (64, "0th"), (128, "hyd")])
+def test_identical_keys_per_block_give_dense_attention(P, block_size, mode):
+    """When every key of a block is the same vector, each block's centroid is its
+    keys and H_j = 0, so the zeroth-order tail is exact and the method equals dense
+    softmax attention at any density (including the partial last block, whose
+    weight n_j must be its true size).  Compared with the oracle's dense
+    attention, which shares no arithmetic with the tail path."""
+    L, d = 1000, 128
+    wl = WORKLOADS["flux"].with_(H=2, L=L, d=d, block_size=block_size, density=0.15,
+                                 sink_idx=-1, mode=mode, cov_weight=0.0, cluster_kind="block")
+    Q, K, V = generate_qkv(wl, "cpu")
+    for s0 in range(0, L, block_size):
+        K[:, :, s0:s0 + block_size] = K[:, :, s0:s0 + 1]
+    q, k, v = (x.cuda() for x in (Q, K, V))
+    out = P.pisa_attention_ex(q, k, v, wl.density, block_size, wl.sink_idx, mode)
+    P.pisa_device_status()
+    for h in range(wl.H):
+        ref = O.dense_attention(to64(Q[0, h]), to64(K[0, h]), to64(V[0, h]), wl.scale)
+        ma, rf = output_errors(to64(out[0, h]), ref)
+        assert ma <= MAX_ABS_TOL and rf <= REL_FRO_TOL, (h, ma, rf)
