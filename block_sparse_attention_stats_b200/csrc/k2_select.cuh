@@ -8,7 +8,12 @@
 //
 //   score_ij = scale * (qbar_i . kbar_j) + lambda * M_j      (float32)
 //
-// Pass 1 (scores_kernel): a float32 FMA GEMM per head, 64 x 64 output tiles,
+// Fused path (select_fused_kernel, short sequences, N <= 512): a group of query
+// blocks computes its score rows into shared memory and selects from there
+// (FLUX shape: 0.028 ms against 0.032 ms; at N = 1182 it is 1.9x slower than the
+// two-pass path, which streams each k-bar tile once per 128 x 128 score tile).
+// Two-pass path otherwise:
+// Pass 1 (scores_kernel): a float32 FMA GEMM per head, 128 x 128 output tiles,
 // each score summed over the head dimension in ascending order.
 // Pass 2 (topk_kernel): one warp per query block.  Scores become 32-bit keys
 // whose unsigned order is the float order; an MSB-first radix select (4 x 8
@@ -103,7 +108,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const int gj = j0 + tx * 8 + c;
-      if (gj < N) out[gj] = scale * acc[r][c] + cw[c];
+      if (gj < N) out[gj] = fmaf(scale, acc[r][c], cw[c]);
     }
   }
 }
@@ -117,18 +122,11 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 
 constexpr int kTopkThreads = 256;  // 8 warps, one query block per warp
 
-// One warp selects the exact set of one query block.  The row's scores stay
-// in global memory (L2) and are re-read on every pass.
-__global__ void __launch_bounds__(kTopkThreads)
-    topk_kernel(const float *__restrict__ scores, int N, int k_sel, int sink, size_t rows,
-                int32_t *__restrict__ idx) {
-  __shared__ unsigned hist_all[kTopkThreads / 32][256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t row = (size_t)blockIdx.x * (kTopkThreads / 32) + warp;
-  if (row >= rows) return;
-  unsigned *hist = hist_all[warp];
-  const float *sc = scores + row * N;
-  int32_t *out = idx + row * k_sel;
+// One warp selects the exact set of one query block from its scores `sc`
+// (global memory, re-read from L2 on every pass, or shared memory); `hist` is
+// the warp's 256-entry histogram.
+__device__ __forceinline__ void topk_row(const float *sc, int N, int k_sel, int sink,
+                                         unsigned *hist, int32_t *__restrict__ out, int lane) {
   const int need = k_sel - (sink >= 0 ? 1 : 0);
   const int candidates = N - (sink >= 0 ? 1 : 0);
   const bool take_all = need >= candidates;
@@ -227,6 +225,107 @@ __global__ void __launch_bounds__(kTopkThreads)
     out_base += __popc(sel_bal);
   }
   if (lane == 0 && out_base != k_sel) report_device_error(kDevErrRange);
+}
+
+// One warp per query block over the N x N score matrix in global memory.
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_kernel(const float *__restrict__ scores, int N, int k_sel, int sink, size_t rows,
+                int32_t *__restrict__ idx) {
+  __shared__ unsigned hist_all[kTopkThreads / 32][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * (kTopkThreads / 32) + warp;
+  if (row >= rows) return;
+  topk_row(scores + row * N, N, k_sel, sink, hist_all[warp], idx + row * k_sel, lane);
+}
+
+// ---------------------------------------------------------------------------
+// Fused scores + top-k for a group of kSelRows query blocks: the group's score
+// rows live in shared memory only (no N x N matrix in HBM).  Each score is the
+// same fp32 computation as in scores_kernel (head dimension summed in ascending
+// order, then scale * acc + lambda * M_j), so both paths select the same sets.
+// 384 threads compute 4 x 4 score blocks from k-bar chunks of 256 blocks x 32
+// dimensions staged transposed in shared memory; then 12 warps take two rows
+// each through the radix select.
+// ---------------------------------------------------------------------------
+constexpr int kSelRows = 24;
+constexpr int kSelFusedMaxN = 512;  // longer rows: the two-pass path (measured faster)
+constexpr int kSelThreads = 384;
+constexpr int kSelCols = 256;      // k-bar blocks per staged chunk
+constexpr int kSelDims = 32;       // head dimensions per staged chunk
+
+__host__ __device__ inline int select_fused_smem(int N, int D) {
+  const int stage = (kSelDims * kSelCols + D * kSelRows) * 4;      // kbar^T chunk, qbar^T
+  const int hist = (kSelThreads / 32) * 256 * 4;
+  return kSelRows * N * 4 + (stage > hist ? stage : hist);
+}
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+    select_fused_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar,
+                        const float *__restrict__ cov, float cov_weight, float scale, int N,
+                        int D, int k_sel, int sink, int32_t *__restrict__ idx) {
+  extern __shared__ __align__(16) float sel_smem[];
+  float *S = sel_smem;                              // [kSelRows][N]
+  float *kT = S + (size_t)kSelRows * N;             // [kSelDims][kSelCols]
+  float *qT = kT + kSelDims * kSelCols;             // [D][kSelRows]
+  unsigned *hist = reinterpret_cast<unsigned *>(kT);   // after the scores: per-warp histograms
+  const int bh = blockIdx.y, i0 = blockIdx.x * kSelRows;
+  const int tid = threadIdx.x;
+  const float *qb = qbar + (size_t)bh * N * D;
+  const float *kb = kbar + (size_t)bh * N * D;
+  const int rg = tid >> 6, cg = tid & 63;           // rows 4 rg .. +3, columns 4 cg .. +3
+
+  for (int e = tid; e < D * kSelRows; e += kSelThreads) {
+    const int r = e % kSelRows, dd = e / kSelRows;
+    qT[e] = i0 + r < N ? qb[(size_t)(i0 + r) * D + dd] : 0.f;
+  }
+  for (int c0 = 0; c0 < N; c0 += kSelCols) {
+    float acc[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) acc[r][x] = 0.f;
+    for (int e0 = 0; e0 < D; e0 += kSelDims) {
+      __syncthreads();   // qT written / the previous chunk consumed
+      for (int f = tid; f < kSelCols * kSelDims / 4; f += kSelThreads) {
+        const int c = f % kSelCols, e4 = (f / kSelCols) * 4;
+        const int j = c0 + c;
+        const float4 v = j < N ? *reinterpret_cast<const float4 *>(kb + (size_t)j * D + e0 + e4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        kT[(e4 + 0) * kSelCols + c] = v.x;
+        kT[(e4 + 1) * kSelCols + c] = v.y;
+        kT[(e4 + 2) * kSelCols + c] = v.z;
+        kT[(e4 + 3) * kSelCols + c] = v.w;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int e = 0; e < kSelDims; ++e) {
+        const float4 a = *reinterpret_cast<const float4 *>(qT + (e0 + e) * kSelRows + 4 * rg);
+        const float4 b = *reinterpret_cast<const float4 *>(kT + e * kSelCols + 4 * cg);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int x = 0; x < 4; ++x) acc[r][x] = fmaf(av[r], bv[x], acc[r][x]);
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int j = c0 + 4 * cg + x;
+      if (j >= N) continue;
+      const float cw = cov_weight != 0.f ? cov_weight * cov[(size_t)bh * N + j] : 0.f;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) S[(size_t)(4 * rg + r) * N + j] = fmaf(scale, acc[r][x], cw);
+    }
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = 2 * warp + h;
+    if (i0 + r < N)
+      topk_row(S + (size_t)r * N, N, k_sel, sink, hist + warp * 256,
+               idx + ((size_t)bh * N + i0 + r) * k_sel, lane);
+  }
 }
 
 }  // namespace pisa

@@ -205,6 +205,17 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
 static pisa_status launch_select(const float *qbar, const float *kbar, const float *cov,
                                  float cov_weight, float scale, int BH, int N, int d, int k_sel,
                                  int sink, int32_t *idx, float *scores, cudaStream_t st) {
+  const int fsmem = select_fused_smem(N, d);
+  if (N <= kSelFusedMaxN && fsmem <= 227 * 1024) {
+    // short sequences: the score rows of a query-block group stay in shared
+    // memory (for long ones the tiled two-pass path is faster: it streams each
+    // k-bar tile once per 128 x 128 score tile instead of once per 24 rows)
+    PISA_CUDA(cudaFuncSetAttribute(select_fused_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, fsmem));
+    select_fused_kernel<<<dim3(ceil_div(N, kSelRows), BH), kSelThreads, fsmem, st>>>(
+        qbar, kbar, cov, cov_weight, scale, N, d, k_sel, sink, idx);
+    return check_launch();
+  }
   dim3 g1(ceil_div(N, kScoreTile), ceil_div(N, kScoreTile), BH);
   scores_kernel<<<g1, 256, 0, st>>>(qbar, kbar, cov, cov_weight, scale, N, d, scores);
   PISA_TRY(check_launch());
