@@ -99,6 +99,8 @@ def bwd_flops(wl, idx: torch.Tensor, heads: int = 2):
     k_sel = idx.shape[-1]
     pairs_alg = wl.L * (k_sel * b + (N - k_sel))
     alg = BH * 10.0 * d * pairs_alg
+    if b != 64:
+        return alg, None   # the executed-tile replay models the 64-token-block schedule
     idx_np = idx.reshape(-1, N, k_sel).cpu().numpy()
     use = min(heads, idx_np.shape[0])
     unit = 2.0 * 64 * 64 * d
@@ -557,7 +559,7 @@ def run_pisa(args, wl):
 
     # ---- backward of the zeroth-order variant (training), same inputs -----------
     bwd = None
-    if not args.no_backward and wl.dtype == "bf16" and wl.block_size == 64:
+    if not args.no_backward and wl.dtype == "bf16":
         G = torch.randn(Q.shape, generator=torch.Generator(device=dev).manual_seed(11),
                         device=dev).to(Q.dtype)
         lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
@@ -588,7 +590,8 @@ def run_pisa(args, wl):
         f_alg_b, f_exec_b = bwd_flops(wl, idx)
         pk = _peaks()[0]
         p_sus_b = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-        bwd = {"ms": bms, "mode": "0th", "launches": 11,
+        ex_tf = f_exec_b / (bms * 1e-3) / 1e12 if f_exec_b else None
+        bwd = {"ms": bms, "mode": "0th", "launches": 11 if wl.block_size == 64 else 9,
                "kernels": "dq: bwd_dq_tc (tcgen05, two sweeps); dk/dv of exact keys: "
                           "bwd_kv_tc (tcgen05); centroid gradients: bwd_centroid (mma.sync); "
                           "packing, bitmap, pairing, padding, list kernels",
@@ -596,8 +599,8 @@ def run_pisa(args, wl):
                             "peak": p_sus_b, "unit": "TFLOP/s",
                             "frac": f_alg_b / (bms * 1e-3) / 1e12 / p_sus_b,
                             "algorithmic_tflop": f_alg_b / 1e12,
-                            "executed_tflop": f_exec_b / 1e12,
-                            "executed_frac": f_exec_b / (bms * 1e-3) / 1e12 / p_sus_b}}
+                            "executed_tflop": f_exec_b / 1e12 if f_exec_b else None,
+                            "executed_frac": ex_tf / p_sus_b if ex_tf else None}}
         del grads, G
 
     # ---- e2e: public API with pinned host buffers ------------------------------

@@ -45,20 +45,23 @@ namespace pisa {
 // ---------------------------------------------------------------------------
 // preprocessing
 // ---------------------------------------------------------------------------
-// kbar16[bh, j] = bf16(kbar_j), vbar16[bh, j] = bf16(vsum_j / n_j); rows N..Npad-1 zero
+// kbar16[bh, j] = bf16(kbar_j), vbar16[bh, j] = bf16(vsum_j / n_j); rows N..Npad-1
+// zero.  N blocks of block_size tokens (the last may be partial).
 __global__ void bwd_pack_centroids_kernel(const float *__restrict__ kbar,
                                           const float *__restrict__ vsum, int N, int Npad, int D,
-                                          int BH, int L, __nv_bfloat16 *__restrict__ kbar16,
+                                          int BH, int L, int block_size,
+                                          __nv_bfloat16 *__restrict__ kbar16,
                                           __nv_bfloat16 *__restrict__ vbar16) {
   const size_t n = (size_t)BH * Npad * D;
-  const float inv_last = 1.f / (float)(L - 64 * (N - 1));
+  const float inv_full = 1.f / (float)block_size;
+  const float inv_last = 1.f / (float)(L - block_size * (N - 1));
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
        e += (size_t)gridDim.x * blockDim.x) {
     const size_t bh = e / ((size_t)Npad * D), rem = e % ((size_t)Npad * D);
     const int j = (int)(rem / D), c = (int)(rem % D);
     const bool ok = j < N;
     const size_t src = (bh * N + (ok ? j : 0)) * D + c;
-    const float inv_n = j == N - 1 ? inv_last : (1.f / 64.f);
+    const float inv_n = j == N - 1 ? inv_last : inv_full;
     kbar16[e] = __float2bfloat16_rn(ok ? kbar[src] : 0.f);
     vbar16[e] = __float2bfloat16_rn(ok ? vsum[src] * inv_n : 0.f);
   }

@@ -68,9 +68,10 @@ template <int D> struct DqTcCfg {
   static constexpr int kBarTeardown = kBarFinal + 1;
   static_assert(kBarTeardown < kNumBars, "barrier slots");
 
-  __host__ __device__ static int smem_bytes(int N) {
-    const int nwords = (N + 31) / 32;
-    return kOffDyn + (2 * nwords + N + (N + 63) / 64) * 4 + 1024;   // + alignment slack
+  // N 64-token tiles, Nc blocks (= centroids)
+  __host__ __device__ static int smem_bytes(int N, int Nc) {
+    const int nwords = (N + 31) / 32, cwords = (Nc + 31) / 32;
+    return kOffDyn + (2 * nwords + 2 * cwords + N + (Nc + 63) / 64) * 4 + 1024;   // + slack
   }
 };
 
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(352, 1)
                      const __grid_constant__ CUtensorMap tm_kbar,
                      const __grid_constant__ CUtensorMap tm_vbar,
                      const int32_t *__restrict__ idx, const int2 *__restrict__ pairs, int k_sel,
-                     int L, int N, float scale, const float *__restrict__ lse,
+                     int L, int N, int bsub, int Nc, float scale, const float *__restrict__ lse,
                      float *__restrict__ delta_out, int Lpad, __nv_bfloat16 *__restrict__ dq) {
   using C = DqTcCfg<D>;
   using namespace sm100;
@@ -101,17 +102,28 @@ __global__ void __launch_bounds__(352, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
   volatile int *misc = reinterpret_cast<volatile int *>(smem + C::kOffMisc);  // [0] tiles, [1] abort
   float *delta_sm = reinterpret_cast<float *>(smem + C::kOffDelta);
-  const int nwords = (N + 31) / 32;
+  // bm_*: selected 64-token tiles per half; cbm_*: selected blocks (the
+  // centroid index space) per half.  With 64-token blocks the two coincide;
+  // with 128-token blocks both halves are one query block and share them.
+  const int nwords = (N + 31) / 32, cwords = (Nc + 31) / 32;
   uint32_t *bm_lo = reinterpret_cast<uint32_t *>(smem + C::kOffDyn);
-  uint32_t *bm_hi = bm_lo + nwords;
-  int *tiles = reinterpret_cast<int *>(bm_hi + nwords);
+  uint32_t *bm_hi = bsub == 1 ? bm_lo + nwords : bm_lo;
+  uint32_t *cbm_lo = bsub == 1 ? bm_lo : bm_lo + 2 * nwords;
+  uint32_t *cbm_hi = bsub == 1 ? bm_hi : cbm_lo;
+  int *tiles = reinterpret_cast<int *>(bm_lo + 2 * nwords + 2 * cwords);
 
   const int pair = blockIdx.x, bh = blockIdx.y;
   int qb0 = 2 * pair, qb1 = 2 * pair + 1 < N ? 2 * pair + 1 : -1;
-  if (pairs) {
+  int sr0 = qb0, sr1 = qb1;                     // selection rows of the halves
+  if (bsub == 2) {
+    sr0 = pair;
+    sr1 = pair;
+  } else if (pairs) {
     const int2 pr = pairs[(size_t)bh * ((N + 1) / 2) + pair];
     qb0 = pr.x;
     qb1 = pr.y;
+    sr0 = qb0;
+    sr1 = qb1;
   }
   const bool has_hi = qb1 >= 0;
   const int tid = threadIdx.x, lane = tid & 31;
@@ -149,16 +161,29 @@ __global__ void __launch_bounds__(352, 1)
     prefetch_tmap(&tm_kbar);
     prefetch_tmap(&tm_vbar);
   }
-  for (int w = tid; w < 2 * nwords; w += C::kThreads) bm_lo[w] = 0u;
+  for (int w = tid; w < 2 * nwords + 2 * cwords; w += C::kThreads) bm_lo[w] = 0u;
   __syncthreads();
-  {
-    const int32_t *r0 = idx + ((size_t)bh * N + qb0) * k_sel;
-    const int32_t *r1 = idx + ((size_t)bh * N + (has_hi ? qb1 : qb0)) * k_sel;
+  if (bsub == 1) {
+    const int32_t *r0 = idx + ((size_t)bh * Nc + sr0) * k_sel;
+    const int32_t *r1 = idx + ((size_t)bh * Nc + (has_hi ? sr1 : sr0)) * k_sel;
     for (int t = tid; t < (has_hi ? 2 : 1) * k_sel; t += C::kThreads) {
       const int j = t < k_sel ? r0[t] : r1[t - k_sel];
       uint32_t *bm = t < k_sel ? bm_lo : bm_hi;
       if (j >= 0 && j < N) atomicOr(&bm[j >> 5], 1u << (j & 31));
       else report_device_error(kDevErrRange);
+    }
+  } else {
+    // one selection row: block j covers the 64-token tiles 2j and 2j + 1
+    const int32_t *r0 = idx + ((size_t)bh * Nc + sr0) * k_sel;
+    for (int t = tid; t < k_sel; t += C::kThreads) {
+      const int j = r0[t];
+      if (j >= 0 && j < Nc) {
+        atomicOr(&cbm_lo[j >> 5], 1u << (j & 31));
+        for (int u = bsub * j; u < bsub * j + bsub && u < N; ++u)
+          atomicOr(&bm_lo[u >> 5], 1u << (u & 31));
+      } else {
+        report_device_error(kDevErrRange);
+      }
     }
   }
   __syncthreads();
@@ -185,15 +210,15 @@ __global__ void __launch_bounds__(352, 1)
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
     // centroid chunks that hold an unselected block for either half
-    const int nch = (N + 63) / 64;
+    const int nch = (Nc + 63) / 64;
     for (int c0 = 0; c0 < nch; c0 += 32) {
       const int c = c0 + lane;
       bool need = false;
       if (c < nch) {
         for (int h = 0; h < (has_hi ? 2 : 1); ++h) {
-          const uint32_t *bm = h ? bm_hi : bm_lo;
-          const uint32_t m0 = ~bm[2 * c] & dq_valid_bits(2 * c, N);
-          const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & dq_valid_bits(2 * c + 1, N)) : 0u;
+          const uint32_t *cb = h ? cbm_hi : cbm_lo;
+          const uint32_t m0 = ~cb[2 * c] & dq_valid_bits(2 * c, Nc);
+          const uint32_t m1 = (2 * c + 1 < cwords) ? (~cb[2 * c + 1] & dq_valid_bits(2 * c + 1, Nc)) : 0u;
           need = need || ((m0 | m1) != 0u);
         }
       }
@@ -359,12 +384,14 @@ __global__ void __launch_bounds__(352, 1)
     const bool exists = half == 0 || has_hi;
     const int grow = (half ? qb1 : qb0) * 64 + (row & 63);
     const bool valid = exists && grow < L;
-    const uint32_t *bm = half ? bm_hi : bm_lo;
+    const uint32_t *cbm = half ? cbm_hi : cbm_lo;
     const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
     const uint32_t s_addr = lane_addr + C::kColBuf + 128 * g, dp_addr = s_addr + 64;
     const float sl2 = scale * kLog2e;
     const float lse2 = valid ? lse[(size_t)bh * L + grow] * kLog2e : INFINITY;
-    const int n_last = L - (N - 1) * 64;
+    const int n_last = L - (N - 1) * 64;                 // tokens in the last 64-token tile
+    const float wblk = 64.f * (float)bsub;               // n_j of a full block
+    const int nc_last = L - (Nc - 1) * 64 * bsub;        // n_j of the last block
     float dpart = 0.f, dfull = 0.f;
     bool exchanged = false, ok = true;
     auto warp_wait = [&](uint32_t b_addr, uint32_t parity) -> bool {
@@ -409,13 +436,13 @@ __global__ void __launch_bounds__(352, 1)
         }
       } else {
         const int c = -e - 1;
-        const uint32_t m0 = ~bm[2 * c] & dq_valid_bits(2 * c, N);
-        const uint32_t m1 = (2 * c + 1 < nwords) ? (~bm[2 * c + 1] & dq_valid_bits(2 * c + 1, N)) : 0u;
+        const uint32_t m0 = ~cbm[2 * c] & dq_valid_bits(2 * c, Nc);
+        const uint32_t m1 = (2 * c + 1 < cwords) ? (~cbm[2 * c + 1] & dq_valid_bits(2 * c + 1, Nc)) : 0u;
         keep = (uint64_t)m0 | ((uint64_t)m1 << 32);
-        w_full = 64.f;
-        if (c == (N - 1) / 64 && n_last < 64) {
-          last_col = (N - 1) % 64;
-          w_last = (float)n_last;
+        w_full = wblk;
+        if (c == (Nc - 1) / 64 && nc_last < 64 * bsub) {
+          last_col = (Nc - 1) % 64;
+          w_last = (float)nc_last;
         }
       }
       const bool active = __any_sync(0xffffffffu, keep != 0ull);

@@ -37,25 +37,47 @@ namespace pisa {
 // ---------------------------------------------------------------------------
 // query-block lists of key-block pairs (CSR per head)
 // ---------------------------------------------------------------------------
-// entry = (i << 2) | (selected 2p) | (selected 2p+1) << 1, ascending i.
-// fill == 0: counts[bh * P + p] = list length; fill == 1: write the entries
-// at entries + bh * cap + offsets[bh * P + p].  One warp per (p, bh).
-__global__ void kvlist_kernel(const uint32_t *__restrict__ bm, int N, int nwords, int P,
-                              int fill, int *__restrict__ counts,
+// entry = (t << 2) | (flag: key tile 2p selected) | (flag: key tile 2p+1) << 1,
+// ascending query tile t (64 tokens).  bm: the selection bitmap at block level
+// [BH, Nc, cwords].  With 64-token blocks (bsub = 1) query and key tiles are
+// blocks: pair p holds blocks 2p, 2p+1, each flagged on its own.  With 128-token
+// blocks (bsub = 2) pair p is block p and a selecting query block i contributes
+// its two query tiles 2i, 2i+1, with both key halves flagged.
+// fill == 0: counts[bh * P + p] = list length; fill == 1: write the entries at
+// entries + bh * cap + offsets[bh * P + p].  One warp per (p, bh).
+__global__ void kvlist_kernel(const uint32_t *__restrict__ bm, int N, int Nc, int cwords,
+                              int bsub, int P, int fill, int *__restrict__ counts,
                               const long long *__restrict__ offsets, long long cap,
                               int *__restrict__ entries) {
   const int p = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
-  const int j0 = 2 * p;
-  const int w = j0 >> 5, sh = j0 & 31;
-  const uint32_t mask = (j0 + 1 < N) ? 3u : 1u;
+  const int jb = bsub == 1 ? 2 * p : p;                 // first block of the pair
+  const int w = jb >> 5, sh = jb & 31;
+  const uint32_t fmask = (2 * p + 1 < N) ? 3u : 1u;     // key tiles that exist
+  const uint32_t bmask = bsub == 1 ? fmask : 1u;
   int total = 0;
   int *out = fill ? entries + bh * cap + offsets[(size_t)bh * P + p] : nullptr;
-  for (int i0 = 0; i0 < N; i0 += 32) {
+  for (int i0 = 0; i0 < Nc; i0 += 32) {
     const int i = i0 + lane;
-    const uint32_t f = i < N ? (bm[((size_t)bh * N + i) * nwords + w] >> sh) & mask : 0u;
-    const unsigned bal = __ballot_sync(0xffffffffu, f != 0u);
-    if (fill && f) out[total + __popc(bal & ((1u << lane) - 1u))] = (i << 2) | (int)f;
-    total += __popc(bal);
+    const uint32_t bits = i < Nc ? (bm[((size_t)bh * Nc + i) * cwords + w] >> sh) & bmask : 0u;
+    // query tiles this lane contributes, in order
+    int n = 0;
+    if (bits) n = bsub == 1 ? 1 : (2 * i + 1 < N ? 2 : 1);
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (fill && n) {
+      const int pos = total + incl - n;
+      if (bsub == 1) {
+        out[pos] = (i << 2) | (int)bits;
+      } else {
+        out[pos] = ((2 * i) << 2) | (int)fmask;
+        if (n == 2) out[pos + 1] = ((2 * i + 1) << 2) | (int)fmask;
+      }
+    }
+    total += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (!fill && lane == 0) counts[(size_t)bh * P + p] = total;
 }
@@ -151,7 +173,8 @@ __global__ void __launch_bounds__(320, 1)
                      const __grid_constant__ CUtensorMap tm_delta,
                      const int *__restrict__ counts, const long long *__restrict__ offsets,
                      long long cap, const int *__restrict__ entries,
-                     const uint32_t *__restrict__ bm, int nwords, int L, int N, float scale,
+                     const uint32_t *__restrict__ bm, int cwords, int bsub, int Nc, int L,
+                     int N, float scale,
                      float *__restrict__ dkbar, float *__restrict__ dvbar, int Npad,
                      __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV) {
   using C = KvTcCfg<D>;
@@ -338,8 +361,9 @@ __global__ void __launch_bounds__(320, 1)
     const int half = row >> 6;
     const int jb = half ? j1 : j0;
     const int key = jb * 64 + (row & 63);          // key token, or centroid index
-    const bool kvalid = jb >= 0 && key < (CENT ? N : L);
-    const float wn = (CENT && key == N - 1) ? (float)(L - 64 * (N - 1)) : 64.f;   // n_j
+    const bool kvalid = jb >= 0 && key < (CENT ? Nc : L);
+    // centroid rows: n_j (64 bsub, or the last block's size)
+    const float wn = (CENT && key == Nc - 1) ? (float)(L - 64 * bsub * (Nc - 1)) : 64.f * bsub;
     const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
     const uint32_t s_addr = lane_addr + C::kColBuf + 128 * g, dp_addr = s_addr + 64;
     const float sl2 = scale * kLog2e;
@@ -351,7 +375,7 @@ __global__ void __launch_bounds__(320, 1)
       if (__any_sync(0xffffffffu, misc[1] != 0)) { ok = false; break; }
       // centroid rows: was block `key` left unselected by query block u?
       const uint32_t selw =
-          (CENT && kvalid) ? bm[((size_t)bh * N + u) * nwords + (key >> 5)] : 0u;
+          (CENT && kvalid) ? bm[((size_t)bh * Nc + u / bsub) * cwords + (key >> 5)] : 0u;
       if (!warp_wait(bar(C::kBarSFull + g), (u >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const int sl = u % C::kStages;
@@ -437,8 +461,9 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     if (!CENT && ok && !__any_sync(0xffffffffu, misc[1] != 0)) {
-      const float *ck = dkbar + ((size_t)bh * Npad + (jb >= 0 ? jb : 0)) * D;
-      const float *cv = dvbar + ((size_t)bh * Npad + (jb >= 0 ? jb : 0)) * D;
+      const int blk = jb >= 0 ? jb / bsub : 0;          // the key's block
+      const float *ck = dkbar + ((size_t)bh * Npad + blk) * D;
+      const float *cv = dvbar + ((size_t)bh * Npad + blk) * D;
       const size_t obase = ((size_t)bh * L + (size_t)(kvalid ? key : 0)) * D;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {

@@ -73,9 +73,9 @@ static bool fused_fits(int d, int L, int block_size) {
   const int smem = d == 128 ? TcCfg<128>::smem_bytes(N, Nc) : TcCfg<64>::smem_bytes(N, Nc);
   return smem <= 227 * 1024;
 }
-static bool bwd_fits(int d, int L) {
-  const int N = ceil_div(L, 64);
-  const int smem = d == 128 ? DqTcCfg<128>::smem_bytes(N) : DqTcCfg<64>::smem_bytes(N);
+static bool bwd_fits(int d, int L, int block_size) {
+  const int N = ceil_div(L, 64), Nc = ceil_div(L, block_size);
+  const int smem = d == 128 ? DqTcCfg<128>::smem_bytes(N, Nc) : DqTcCfg<64>::smem_bytes(N, Nc);
   return smem <= 227 * 1024;
 }
 
@@ -373,8 +373,10 @@ struct BwdLayout {
       total;
   long long cap;   // list entries per head
 };
-static BwdLayout bwd_layout(int B, int H, int L, int d, int k_sel) {
-  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+static BwdLayout bwd_layout(int B, int H, int L, int d, int k_sel, int block_size) {
+  // N 64-token tiles; Nc blocks (= N with 64-token blocks)
+  const int N = ceil_div(L, 64), Nc = ceil_div(L, block_size);
+  const int Npad = ceil_div(Nc, 64) * 64, nwords = ceil_div(Nc, 32);
   const int Lpad = N * 64, P = (N + 1) / 2;
   const size_t BH = (size_t)B * H;
   BwdLayout p;
@@ -390,8 +392,9 @@ static BwdLayout bwd_layout(int B, int H, int L, int d, int k_sel) {
   p.dvbar = o; o += align_up(BH * Npad * d * 4, 256);
   p.counts = o; o += align_up(BH * P * 4, 256);
   p.offsets = o; o += align_up(BH * P * 8, 256);
-  // the lists of a head hold each selected (query block, key block) pair at most once
-  p.cap = (long long)N * k_sel;
+  // the lists of a head hold each selected (query block, key block) pair at most
+  // once, as one (64-token blocks) or two (128-token blocks) query tiles
+  p.cap = (long long)(block_size == 64 ? N : 2 * Nc) * k_sel;
   p.entries = o; o += align_up(BH * (size_t)p.cap * 4, 256);
   p.total = o;
   return p;
@@ -422,10 +425,13 @@ static pisa_status make_map_f32_rows(CUtensorMap *m, const void *base, uint64_t 
 template <int D>
 static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                               const __nv_bfloat16 *v, const __nv_bfloat16 *dout, const float *lse,
-                              const int32_t *idx, int k_sel, int BH, int L, float scale,
+                              const int32_t *idx, int k_sel, int BH, int L, int bsub, float scale,
                               const BwdLayout &lay, unsigned char *ws, __nv_bfloat16 *dq,
                               __nv_bfloat16 *dk, __nv_bfloat16 *dv, cudaStream_t st) {
-  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
+  // N 64-token tiles, Nc blocks of bsub tiles (the selection's and the
+  // centroids' index space)
+  const int N = ceil_div(L, 64), Nc = ceil_div(L, 64 * bsub);
+  const int Ncpad = ceil_div(Nc, 64) * 64, cwords = ceil_div(Nc, 32);
   const int Lpad = N * 64, P = (N + 1) / 2;
   float *lse_pad = (float *)(ws + lay.lse_pad);
   float *delta = (float *)(ws + lay.delta);
@@ -438,57 +444,61 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   int *entries = (int *)(ws + lay.entries);
   pad_lse_kernel<<<grid_1d((size_t)BH * Lpad, 256), 256, 0, st>>>(lse, L, Lpad, BH, lse_pad);
   PISA_TRY(check_launch());
-  // dq on the tensor cores: query blocks paired like the forward's
-  uint16_t *ov = (uint16_t *)(ws + lay.ov);
-  int2 *pairs = (int2 *)(ws + lay.pairs);
-  pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, nwords, ov);
-  PISA_TRY(check_launch());
-  const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
-  const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
-  if (pair_smem > 48 * 1024)
-    PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   pair_smem));
-  pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
-  PISA_TRY(check_launch());
-  const int dq_smem = DqTcCfg<D>::smem_bytes(N);
+  // dq on the tensor cores: with 64-token blocks the query blocks are paired
+  // like the forward's; with 128-token blocks a CTA is one query block
+  int2 *pairs = nullptr;
+  if (bsub == 1) {
+    uint16_t *ov = (uint16_t *)(ws + lay.ov);
+    pairs = (int2 *)(ws + lay.pairs);
+    pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, cwords, ov);
+    PISA_TRY(check_launch());
+    const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
+    const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
+    if (pair_smem > 48 * 1024)
+      PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     pair_smem));
+    pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
+    PISA_TRY(check_launch());
+  }
+  const int dq_smem = DqTcCfg<D>::smem_bytes(N, Nc);
   if (dq_smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
   CUtensorMap mq, mdo, mk, mv, mkb, mvb, mlse, mdel;
   PISA_TRY(make_map(&mq, q, D, L, BH, 64));
   PISA_TRY(make_map(&mdo, dout, D, L, BH, 64));
   PISA_TRY(make_map(&mk, k, D, L, BH, 64));
   PISA_TRY(make_map(&mv, v, D, L, BH, 64));
-  PISA_TRY(make_map(&mkb, kb, D, Npad, BH, 64));
-  PISA_TRY(make_map(&mvb, vb, D, Npad, BH, 64));
+  PISA_TRY(make_map(&mkb, kb, D, Ncpad, BH, 64));
+  PISA_TRY(make_map(&mvb, vb, D, Ncpad, BH, 64));
   PISA_TRY(make_map_f32_rows(&mlse, lse_pad, Lpad, BH));
   PISA_TRY(make_map_f32_rows(&mdel, delta, Lpad, BH));
   PISA_CUDA(cudaFuncSetAttribute(bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dq_smem));
   bwd_dq_tc_kernel<D><<<dim3(P, BH), DqTcCfg<D>::kThreads, dq_smem, st>>>(
-      mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, scale, lse, delta, Lpad, dq);
+      mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, bsub, Nc, scale, lse, delta, Lpad, dq);
   PISA_TRY(check_launch());
   // centroid gradients, then the exact keys' dk, dv, both on the tensor cores
-  // (the exact pass over the query-block lists of each key-block pair)
+  // (the exact pass over the query-tile lists of each key-block pair)
   const int kvtc_smem = KvTcCfg<D>::kSmem;
   PISA_CUDA(cudaFuncSetAttribute(bwd_kv_tc_kernel<D, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kvtc_smem));
   PISA_CUDA(cudaFuncSetAttribute(bwd_kv_tc_kernel<D, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kvtc_smem));
-  bwd_kv_tc_kernel<D, true><<<dim3(Npad / 128 + (Npad % 128 ? 1 : 0), BH), KvTcCfg<D>::kThreads,
-                              kvtc_smem, st>>>(
-      mq, mdo, mkb, mvb, mlse, mdel, nullptr, nullptr, 0, nullptr, bm, nwords, L, N, scale,
-      dkbar, dvbar, Npad, nullptr, nullptr);
+  bwd_kv_tc_kernel<D, true><<<dim3(ceil_div(Ncpad, 128), BH), KvTcCfg<D>::kThreads, kvtc_smem,
+                              st>>>(
+      mq, mdo, mkb, mvb, mlse, mdel, nullptr, nullptr, 0, nullptr, bm, cwords, bsub, Nc, L, N,
+      scale, dkbar, dvbar, Ncpad, nullptr, nullptr);
   PISA_TRY(check_launch());
-  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, nwords, P, 0, counts, offsets, lay.cap,
-                                            entries);
+  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, 0, counts, offsets,
+                                            lay.cap, entries);
   PISA_TRY(check_launch());
   kvlist_scan_kernel<<<BH, 1024, 0, st>>>(counts, P, offsets);
   PISA_TRY(check_launch());
-  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, nwords, P, 1, counts, offsets, lay.cap,
-                                            entries);
+  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, 1, counts, offsets,
+                                            lay.cap, entries);
   PISA_TRY(check_launch());
   bwd_kv_tc_kernel<D, false><<<dim3(P, BH), KvTcCfg<D>::kThreads, kvtc_smem, st>>>(
-      mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, bm, nwords, L, N, scale,
-      dkbar, dvbar, Npad, dk, dv);
+      mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, bm, cwords, bsub, Nc, L, N,
+      scale, dkbar, dvbar, Ncpad, dk, dv);
   return check_launch();
 }
 
@@ -664,9 +674,9 @@ pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *
 
 size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size,
                                                  int k_sel) {
-  if (check_shape(B, H, L, d, block_size) != PISA_OK || block_size != 64) return 0;
-  if (k_sel < 1 || k_sel > ceil_div(L, 64)) return 0;
-  return bwd_layout(B, H, L, d, k_sel).total;
+  if (check_shape(B, H, L, d, block_size) != PISA_OK) return 0;
+  if (k_sel < 1 || k_sel > ceil_div(L, block_size)) return 0;
+  return bwd_layout(B, H, L, d, k_sel, block_size).total;
 }
 
 pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *v,
@@ -676,10 +686,11 @@ pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *
                                       float scale, void *dq, void *dk, void *dv, void *workspace,
                                       size_t ws_bytes, pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, block_size));
-  if (block_size != 64) return PISA_ERR_UNSUPPORTED;
-  if (!bwd_fits(d, L)) return PISA_ERR_UNSUPPORTED;
-  const int N = ceil_div(L, 64), Npad = ceil_div(N, 64) * 64, nwords = ceil_div(N, 32);
-  if (k_sel < 1 || k_sel > N) return PISA_ERR_INVALID_ARG;
+  if (!bwd_fits(d, L, block_size)) return PISA_ERR_UNSUPPORTED;
+  // Nc blocks of block_size tokens (the selection's index space)
+  const int Nc = ceil_div(L, block_size), Ncpad = ceil_div(Nc, 64) * 64,
+            cwords = ceil_div(Nc, 32);
+  if (k_sel < 1 || k_sel > Nc) return PISA_ERR_INVALID_ARG;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return PISA_ERR_INVALID_ARG;
   const void *ins[] = {q, k, v, dout};
   void *outs[] = {dq, dk, dv};
@@ -694,25 +705,25 @@ pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *
   if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(kbar) || !aligned16(vsum) ||
       !idx || !aligned16(workspace))
     return PISA_ERR_INVALID_ARG;
-  const BwdLayout lay = bwd_layout(B, H, L, d, k_sel);
+  const BwdLayout lay = bwd_layout(B, H, L, d, k_sel, block_size);
   if (ws_bytes < lay.total) return PISA_ERR_WORKSPACE;
   const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
   const int BH = B * H;
   cudaStream_t st = (cudaStream_t)stream;
   unsigned char *ws = (unsigned char *)workspace;
-  bwd_pack_centroids_kernel<<<grid_1d((size_t)BH * Npad * d, 256), 256, 0, st>>>(
-      kbar, vsum, N, Npad, d, BH, L, (__nv_bfloat16 *)(ws + lay.kbar16),
+  bwd_pack_centroids_kernel<<<grid_1d((size_t)BH * Ncpad * d, 256), 256, 0, st>>>(
+      kbar, vsum, Nc, Ncpad, d, BH, L, block_size, (__nv_bfloat16 *)(ws + lay.kbar16),
       (__nv_bfloat16 *)(ws + lay.vbar16));
   PISA_TRY(check_launch());
-  selection_bitmap_kernel<<<dim3(N, BH), 64, nwords * sizeof(uint32_t), st>>>(
-      idx, N, k_sel, nwords, (uint32_t *)(ws + lay.bm));
+  selection_bitmap_kernel<<<dim3(Nc, BH), 64, cwords * sizeof(uint32_t), st>>>(
+      idx, Nc, k_sel, cwords, (uint32_t *)(ws + lay.bm));
   PISA_TRY(check_launch());
   const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
                       *v16 = (const __nv_bfloat16 *)v, *g16 = (const __nv_bfloat16 *)dout;
   if (d == 128)
-    return launch_bwd<128>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, s, lay, ws,
+    return launch_bwd<128>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, block_size / 64, s, lay, ws,
                            (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, st);
-  return launch_bwd<64>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, s, lay, ws,
+  return launch_bwd<64>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, block_size / 64, s, lay, ws,
                         (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, st);
 }
 

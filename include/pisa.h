@@ -28,8 +28,8 @@
  *    by the kernels themselves (an index out of range, a bounded wait that ran
  *    out) are recorded in a device status word that pisa_device_status reads.
  *  - Supported now: d in {64, 128}; block_size 64 or 128 (the block-wise
- *    first-order mode, the backward and the score histogram: 64 only; the
- *    authors' README uses 64, the skill page gives 64-128); dtype bf16 or f32 (f32
+ *    first-order mode and the score histogram: 64 only; the authors' README
+ *    uses 64, the skill page gives 64-128); dtype bf16 or f32 (f32
  *    inputs are rounded to bf16 for the tensor-core products; statistics are
  *    accumulated in float32 from the inputs as given); all data pointers
  *    16-byte aligned.

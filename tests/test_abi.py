@@ -60,7 +60,8 @@ def test_workspace_sizes(lib):
     assert lib.pisa_workspace_bytes(1, 1, 1024, 96, 64, 0.25, L.PISA_BF16, 0) == 0
     assert lib.pisa_workspace_bytes(1, 1, 1024, 128, 32, 0.25, L.PISA_BF16, 0) == 0
     assert lib.pisa_workspace_bytes(1, 1, 1024, 128, 128, 0.25, L.PISA_BF16, 0) > 0
-    assert lib.pisa_sparse_attention_bwd_workspace_bytes(1, 1, 1024, 128, 128, 4) == 0
+    assert lib.pisa_sparse_attention_bwd_workspace_bytes(1, 1, 1024, 128, 128, 4) > 0
+    assert lib.pisa_sparse_attention_bwd_workspace_bytes(1, 1, 1024, 128, 128, 9) == 0
     assert lib.pisa_sparse_attention_bwd_workspace_bytes(1, 1, 1024, 128, 64, 4) > 0
     assert lib.pisa_sparse_attention_bwd_workspace_bytes(1, 1, 1024, 128, 64, 17) == 0
 

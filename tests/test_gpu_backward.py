@@ -111,6 +111,22 @@ def test_backward_matches_oracle(P, L, d, density, sink):
     _check_head(P, wl, 0, 0)
 
 
+@pytest.mark.parametrize("L,d,density,sink", [
+    (4608, 128, 0.15, -1),     # FLUX-like shape, 36 blocks of 128 tokens
+    (1000, 128, 0.25, None),   # last block 104 tokens: its second tile is partial
+    (777, 64, 0.25, 0),        # d = 64; last block 9 tokens in one tile, odd tile count
+    (129, 128, 0.5, -1),       # N = 2 with a one-token sink block
+])
+def test_backward_block_size_128(P, L, d, density, sink):
+    """128-token blocks: dq per query block (both halves share S_i), dk/dv per key
+    block over the query tiles of the blocks that selected it, centroid gradients
+    with n_j = 128."""
+    wl = WORKLOADS["flux"].with_(B=1, H=1, L=L, d=d, block_size=128, density=density,
+                                 sink_idx=sink, cov_weight=0.0, mode="0th",
+                                 cluster_kind="image" if L == 4608 else "block")
+    _check_head(P, wl, 0, 0)
+
+
 def test_single_token(P):
     """L = 1: the output is v_0 whatever q and k are, so the exact gradient is
     dq = 0, dk = 0, dv = dout (a relative comparison is meaningless at 0)."""
