@@ -179,8 +179,8 @@ size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int
                                                  int k_sel);
 
 /* Gradients of the zeroth-order forward (the authors' README, "Kernel
- * variants": piecewise_sparse_attention_0th "supports training"; the forward
- * is the equation above without the hyd term).  Given dout = dL/d out, writes
+ * variants": piecewise_sparse_attention_0th is the variant meant for training;
+ * the forward is the equation above without the hyd term).  Given dout = dL/d out, writes
  *   dq = dL/dq,  dk = dL/dk,  dv = dL/dv        bf16 [B,H,L,d]
  * with the selection idx held fixed (a discrete step) and the statistics
  * differentiated: kbar_j is the mean key and vsum_j the value sum of block j,
