@@ -36,7 +36,7 @@ namespace pisa {
 
 template <int D> struct DqTcCfg {
   static constexpr int kThreads = 352;
-  static constexpr int kStages = 2;
+  static constexpr int kStages = 3;
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kBoxQBytes = 128 * 128;     // one 64-column box of 128 rows
   static constexpr int kBoxKBytes = 64 * 128;      // one 64-column box of 64 rows
@@ -46,7 +46,7 @@ template <int D> struct DqTcCfg {
   static constexpr int kOffK = 2 * kQBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 20;
+  static constexpr int kNumBars = 24;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffMisc = kOffTmemSlot + 16;
   static constexpr int kOffDelta = kOffMisc + 16;               // [2][128] f32

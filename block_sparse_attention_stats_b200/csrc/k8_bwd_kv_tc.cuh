@@ -127,7 +127,7 @@ __global__ void pad_lse_kernel(const float *__restrict__ lse, int L, int Lpad, i
 // ---------------------------------------------------------------------------
 template <int D> struct KvTcCfg {
   static constexpr int kThreads = 320;
-  static constexpr int kStages = 2;
+  static constexpr int kStages = 3;
   static constexpr int kPairBytes = 128 * D * 2;   // K or V of the two key blocks
   static constexpr int kBoxPairBytes = 128 * 128;  // one 64-column box of 128 rows
   static constexpr int kBoxRowBytes = 64 * 128;    // one 64-column box of 64 rows
