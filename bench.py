@@ -593,7 +593,8 @@ def run_pisa(args, wl):
         ex_tf = f_exec_b / (bms * 1e-3) / 1e12 if f_exec_b else None
         bwd = {"ms": bms, "mode": "0th", "launches": 11 if wl.block_size == 64 else 9,
                "kernels": "dq: bwd_dq_tc (tcgen05, two sweeps); dk/dv of exact keys: "
-                          "bwd_kv_tc (tcgen05); centroid gradients: bwd_centroid (mma.sync); "
+                          "bwd_kv_tc<false> (tcgen05); centroid gradients: bwd_kv_tc<true> "
+                          "(tcgen05, centroid rows weighted by n_j); "
                           "packing, bitmap, pairing, padding, list kernels",
                "roofline": {"bound": "tensor", "achieved": f_alg_b / (bms * 1e-3) / 1e12,
                             "peak": p_sus_b, "unit": "TFLOP/s",
