@@ -80,7 +80,7 @@ def dense_flops(wl):
     return 4.0 * wl.B * wl.H * wl.L * wl.L * wl.d
 
 
-def bwd_flops(wl, idx: torch.Tensor, heads: int = 2):
+def bwd_flops(wl, idx: torch.Tensor, heads: int = 2, dq_products: int = 3):
     """(algorithmic, executed) FLOPs of one zeroth-order backward.
 
     Algorithmic: five products per (query row, key) pair of the augmented
@@ -88,10 +88,11 @@ def bwd_flops(wl, idx: torch.Tensor, heads: int = 2):
     dQ += dz k), 2 d FLOPs each, over the exact keys of S_i and the centroids of
     U_i.  Executed, replayed on `heads` heads and scaled: the dq kernel's
     128 x 64 tiles over each query pair's union of exact tiles plus its centroid
-    chunks, five products each (logits and dP in both sweeps, dQ in the second);
-    the dk/dv kernel's 128 x 64 tiles over each key pair's union of query
-    blocks, four products each; the centroid kernel's 64 x 64 tiles over every
-    (chunk, query block) it visits, four products each."""
+    chunks, `dq_products` products each (logits, dP and dQ with Delta given by
+    the forward's float32 output; five with the extra Delta sweep); the dk/dv
+    kernel's 128 x 64 tiles over each key pair's union of query blocks, four
+    products each; the centroid instance's 128-centroid x 64-query tiles over
+    every query tile, four products each."""
     b, d = wl.block_size, wl.d
     N = -(-wl.L // b)
     C = -(-N // 64)
@@ -113,13 +114,11 @@ def bwd_flops(wl, idx: torch.Tensor, heads: int = 2):
             chunks = sum(int((~bits[i, c * 64:min(N, c * 64 + 64)]).any() or
                              (j >= 0 and (~bits[j, c * 64:min(N, c * 64 + 64)]).any()))
                          for c in range(C))
-            tot += 5 * 2 * unit * (int(sel.sum()) + chunks)
+            tot += dq_products * 2 * unit * (int(sel.sum()) + chunks)
         for p in range(-(-N // 2)):
             cols = bits[:, 2 * p] | (bits[:, 2 * p + 1] if 2 * p + 1 < N else False)
             tot += 4 * 2 * unit * int(cols.sum())
-        for c in range(C):
-            need = (~bits[:, c * 64:min(N, c * 64 + 64)]).any(axis=1)
-            tot += 4 * unit * int(need.sum())
+        tot += 4 * 2 * unit * (-(-C // 2)) * N
     return alg, tot * BH / use
 
 
@@ -563,15 +562,17 @@ def run_pisa(args, wl):
         G = torch.randn(Q.shape, generator=torch.Generator(device=dev).manual_seed(11),
                         device=dev).to(Q.dtype)
         lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+        o32 = torch.empty(Q.shape, dtype=torch.float32, device=dev)
         P.pisa_sparse_attention_fwd(Q, K, V, stt["kbar"], stt["vsum"], stt["hbar"], idx, "0th",
-                                    wl.block_size, out=out, lse=lse, workspace=k3_ws)
+                                    wl.block_size, out=out, lse=lse, workspace=k3_ws,
+                                    out_f32=o32)
         bws = mk(lib.pisa_sparse_attention_bwd_workspace_bytes(wl.B, wl.H, wl.L, wl.d,
                                                                 wl.block_size, idx.shape[-1]))
         grads = tuple(torch.empty_like(Q) for _ in range(3))
 
         def bstep():
             P.pisa_sparse_attention_bwd(Q, K, V, G, lse, stt["kbar"], stt["vsum"], idx,
-                                        wl.block_size, grads=grads, workspace=bws)
+                                        wl.block_size, grads=grads, workspace=bws, out_f32=o32)
 
         for _ in range(3):
             bstep()
@@ -591,8 +592,9 @@ def run_pisa(args, wl):
         pk = _peaks()[0]
         p_sus_b = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         ex_tf = f_exec_b / (bms * 1e-3) / 1e12 if f_exec_b else None
-        bwd = {"ms": bms, "mode": "0th", "launches": 11 if wl.block_size == 64 else 9,
-               "kernels": "dq: bwd_dq_tc (tcgen05, two sweeps); dk/dv of exact keys: "
+        bwd = {"ms": bms, "mode": "0th", "launches": 12 if wl.block_size == 64 else 10,
+               "delta": "dout . o from the forward's float32 output (bwd_delta_kernel)",
+               "kernels": "dq: bwd_dq_tc (tcgen05, one sweep); dk/dv of exact keys: "
                           "bwd_kv_tc<false> (tcgen05); centroid gradients: bwd_kv_tc<true> "
                           "(tcgen05, centroid rows weighted by n_j); "
                           "packing, bitmap, pairing, padding, list kernels",
@@ -602,7 +604,7 @@ def run_pisa(args, wl):
                             "algorithmic_tflop": f_alg_b / 1e12,
                             "executed_tflop": f_exec_b / 1e12 if f_exec_b else None,
                             "executed_frac": ex_tf / p_sus_b if ex_tf else None}}
-        del grads, G
+        del grads, G, o32
 
     # ---- e2e: public API with pinned host buffers ------------------------------
     e2e = None

@@ -49,9 +49,9 @@ SIGNATURES = {
     "pisa_sparse_attention": (_I, [_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                    _F, _I, _P, _P, _Z, _P]),
     "pisa_sparse_attention_fwd": (_I, [_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
-                                       _F, _I, _P, _P, _P, _Z, _P]),
+                                       _F, _I, _P, _P, _P, _P, _Z, _P]),
     "pisa_sparse_attention_bwd_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I]),
-    "pisa_sparse_attention_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+    "pisa_sparse_attention_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
                                        _I, _F, _P, _P, _P, _P, _Z, _P]),
     "pisa_attention": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _D, _I, _I, _P]),
     "pisa_attention_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _D, _I, _I,

@@ -174,8 +174,11 @@ def pisa_sparse_attention_fwd(q, k, v, kbar, vsum, hbar, idx, mode: str = "0th",
                               block_size: int = 64, scale: Optional[float] = None,
                               out: Optional[torch.Tensor] = None,
                               lse: Optional[torch.Tensor] = None,
-                              workspace: Optional[torch.Tensor] = None, stream=None):
-    """pisa_sparse_attention that also returns lse [B, H, L] float32 (ln D_t)."""
+                              workspace: Optional[torch.Tensor] = None, stream=None,
+                              out_f32: Optional[torch.Tensor] = None):
+    """pisa_sparse_attention that also returns lse [B, H, L] float32 (ln D_t).
+    `out_f32` (float32 [B, H, L, d]), if given, receives the output before its
+    rounding to the input dtype; the backward forms its row term from it."""
     lib = L.load()
     B, H, Ln, d = _qkv_dims(q, k, v)
     k_sel = idx.shape[-1]
@@ -186,15 +189,19 @@ def pisa_sparse_attention_fwd(q, k, v, kbar, vsum, hbar, idx, mode: str = "0th",
     _check("pisa_sparse_attention_fwd", lib.pisa_sparse_attention_fwd(
         _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(idx),
         k_sel, B, H, Ln, d, block_size, 0.0 if scale is None else float(scale), _MODE[mode],
-        _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+        _ptr(out), _ptr(lse), _ptr(out_f32), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
     return out, lse
 
 
 def pisa_sparse_attention_bwd(q, k, v, dout, lse, kbar, vsum, idx, block_size: int = 64,
                               scale: Optional[float] = None,
                               grads: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
-                              workspace: Optional[torch.Tensor] = None, stream=None):
-    """Gradients (dq, dk, dv) of the zeroth-order forward, bf16 [B, H, L, d]."""
+                              workspace: Optional[torch.Tensor] = None, stream=None,
+                              out_f32: Optional[torch.Tensor] = None):
+    """Gradients (dq, dk, dv) of the zeroth-order forward, bf16 [B, H, L, d].
+    With `out_f32` (the forward's float32 output) the row term
+    Delta_t = dout_t . out_t comes from it and dq takes one sweep, else two."""
     lib = L.load()
     B, H, Ln, d = _qkv_dims(q, k, v)
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
@@ -202,7 +209,7 @@ def pisa_sparse_attention_bwd(q, k, v, dout, lse, kbar, vsum, idx, block_size: i
     need = lib.pisa_sparse_attention_bwd_workspace_bytes(B, H, Ln, d, block_size, idx.shape[-1])
     ws = workspace if workspace is not None else _workspace(need, q.device)
     _check("pisa_sparse_attention_bwd", lib.pisa_sparse_attention_bwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(kbar), _ptr(vsum),
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(out_f32), _ptr(kbar), _ptr(vsum),
         _ptr(idx), idx.shape[-1], B, H, Ln, d, block_size,
         0.0 if scale is None else float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
@@ -217,17 +224,18 @@ class _PiecewiseAttention0th(torch.autograd.Function):
         q, k, v = (x.contiguous() for x in (q, k, v))
         st = pisa_block_stats(q, k, v, block_size)
         idx = pisa_select(st["qbar"], st["kbar"], density, sink_idx, scale=scale)
+        o32 = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         out, lse = pisa_sparse_attention_fwd(q, k, v, st["kbar"], st["vsum"], st["hbar"], idx,
-                                             "0th", block_size, scale)
-        ctx.save_for_backward(q, k, v, lse, st["kbar"], st["vsum"], idx)
+                                             "0th", block_size, scale, out_f32=o32)
+        ctx.save_for_backward(q, k, v, lse, o32, st["kbar"], st["vsum"], idx)
         ctx.block_size, ctx.scale = block_size, scale
         return out
 
     @staticmethod
     def backward(ctx, dout):
-        q, k, v, lse, kbar, vsum, idx = ctx.saved_tensors
+        q, k, v, lse, o32, kbar, vsum, idx = ctx.saved_tensors
         dq, dk, dv = pisa_sparse_attention_bwd(q, k, v, dout.contiguous(), lse, kbar, vsum, idx,
-                                               ctx.block_size, ctx.scale)
+                                               ctx.block_size, ctx.scale, out_f32=o32)
         return dq, dk, dv, None, None, None, None
 
 

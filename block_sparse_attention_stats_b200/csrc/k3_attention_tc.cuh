@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(192, 2)
                                   const int2 *__restrict__ pairs, int k_sel, int L, int N,
                                   int bsub, int Nc, float scale, int hyd, int dense, int blockwise,
                                   void *__restrict__ out, int out_f32,
-                                  float *__restrict__ lse) {
+                                  float *__restrict__ lse, float *__restrict__ o_keep) {
   using C = TcCfg<D>;
   using namespace sm100;
   extern __shared__ unsigned char smem_raw[];
@@ -552,12 +552,25 @@ __global__ void __launch_bounds__(192, 2)
         const float2 sl2x2 = make_float2(sl2, sl2), neg2 = make_float2(neg, neg);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};
+        if (o_keep == nullptr) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 x = fma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2x2, neg2);
-          const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          acc[i & 3] = add2(acc[i & 3], p);
-          pk[i] = pack_bf16x2(p.x, p.y);
+          for (int i = 0; i < 32; ++i) {
+            const float2 x = fma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2x2, neg2);
+            const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            acc[i & 3] = add2(acc[i & 3], p);
+            pk[i] = pack_bf16x2(p.x, p.y);
+          }
+        } else {
+          // the denominator sums the same bf16 weights the P V product uses, so
+          // o_t is normalised exactly and dout_t . o_t matches the backward's
+          // sum_m P_tm dP_tm to the rounding of each weight's deviation
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float2 x = fma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2x2, neg2);
+            pk[i] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+            acc[i & 3] = add2(acc[i & 3], make_float2(__uint_as_float(pk[i] << 16),
+                                                      __uint_as_float(pk[i] & 0xffff0000u)));
+          }
         }
         const float2 s2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
         const float ps = s2.x + s2.y;
@@ -569,6 +582,7 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
             for (int i = 0; i < 64; ++i)
               if (i == col) pl = ex2_approx(fmaf(sv[i], sl2, neg));
+            if (o_keep != nullptr) pl = __bfloat162float(__float2bfloat16_rn(pl));
           }
           a_run += ps;
           l_run += wblk * ps - (wblk - (float)nc_last) * pl;
@@ -612,6 +626,12 @@ __global__ void __launch_bounds__(192, 2)
             float acc = __uint_as_float(o[i]);
             if (hyd) acc = fmaf(fa, __uint_as_float(qh[i]), acc);
             v[i] = acc * inv;
+          }
+          if (store && o_keep != nullptr) {
+            float4 *dst = reinterpret_cast<float4 *>(o_keep + obase + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
           if (store) {
             if (out_f32) {

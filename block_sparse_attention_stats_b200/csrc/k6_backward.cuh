@@ -16,7 +16,8 @@
 //   dkbar_j   = s sum_t dz_tj q_t,  dvbar_j = sum_t P_tj dout_t   (t with j in U_i)
 // The selection is a discrete step and is held fixed.
 //
-// Kernels (11 launches per call):
+// Kernels (11 launches per call; 12 when the forward's float32 output is
+// given, which replaces the dq kernel's first sweep by bwd_delta_kernel):
 //   bwd_pack_centroids_kernel (this file) bf16 kbar_j and vbar_j = vsum_j / n_j,
 //                             rows >= N zero
 //   selection_bitmap_kernel, pair_overlap_kernel, pairing_kernel (k3_pack.cuh)
@@ -24,10 +25,12 @@
 //   pad_lse_kernel, kvlist_kernel (x2), kvlist_scan_kernel (k8_bwd_kv_tc.cuh)
 //                             padded lse; per key-block pair, the ascending list
 //                             of query blocks that selected either block
+//   bwd_delta_kernel          (this file, when the forward's float32 output
+//                             o is given) Delta_t = dout_t . o_t
 //   bwd_dq_tc_kernel          (k7_bwd_dq_tc.cuh, tcgen05) one CTA per pair of
-//                             query blocks, two sweeps over their exact tiles and
-//                             the centroid chunks: Delta_t = sum_m P_tm dP_tm,
-//                             then dq
+//                             query blocks over their exact tiles and the
+//                             centroid chunks: without a given Delta, a first
+//                             sweep forms Delta_t = sum_m P_tm dP_tm; then dq
 //   bwd_kv_tc_kernel<true>    (tcgen05) one CTA per 128 centroids, over every
 //                             query block -> dkbar_j / n_j, dvbar_j / n_j (float32)
 //   bwd_kv_tc_kernel<false>   (tcgen05) one CTA per pair of key blocks, over the
@@ -64,6 +67,37 @@ __global__ void bwd_pack_centroids_kernel(const float *__restrict__ kbar,
     const float inv_n = j == N - 1 ? inv_last : inv_full;
     kbar16[e] = __float2bfloat16_rn(ok ? kbar[src] : 0.f);
     vbar16[e] = __float2bfloat16_rn(ok ? vsum[src] * inv_n : 0.f);
+  }
+}
+
+// Delta_t = dout_t . o_t for t < L from the forward's float32 output o (the
+// same quantity as sum_m P_tm dP_tm, since o_t = sum_m P_tm value_m), 0 for
+// the padding rows L .. Lpad-1 of each head.  One warp per row; D a multiple
+// of 64; dout 8-byte and o 16-byte aligned.
+__global__ void bwd_delta_kernel(const __nv_bfloat16 *__restrict__ dout,
+                                 const float *__restrict__ o, int L, int Lpad, int D, int BH,
+                                 float *__restrict__ delta) {
+  const size_t rows = (size_t)BH * Lpad;
+  const int lane = threadIdx.x & 31;
+  const size_t warps = ((size_t)gridDim.x * blockDim.x) >> 5;
+  for (size_t r = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5; r < rows; r += warps) {
+    const size_t bh = r / Lpad;
+    const int t = (int)(r % Lpad);
+    float acc = 0.f;
+    if (t < L) {
+      const size_t base = (bh * L + t) * D;
+      for (int c = 4 * lane; c < D; c += 128) {
+        const uint2 g = *reinterpret_cast<const uint2 *>(dout + base + c);
+        const float4 x = *reinterpret_cast<const float4 *>(o + base + c);
+        acc = fmaf(__uint_as_float(g.x << 16), x.x, acc);
+        acc = fmaf(__uint_as_float(g.x & 0xffff0000u), x.y, acc);
+        acc = fmaf(__uint_as_float(g.y << 16), x.z, acc);
+        acc = fmaf(__uint_as_float(g.y & 0xffff0000u), x.w, acc);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) delta[r] = acc;
   }
 }
 

@@ -6,13 +6,15 @@
 // P_tm = w_m exp(s q_t.key_m - lse_t) (w = 1 for exact keys, n_j for
 // centroids), dP_tm = dout_t . value_m and Delta_t = sum_m P_tm dP_tm:
 //   dq_t = s sum_m P_tm (dP_tm - Delta_t) key_m
-// The kernel makes two sweeps over the tile list: the first forms Delta_t
-// from its own P and dP (so that sum_m dz_tm vanishes to f32 rounding), the
-// second accumulates dq in tensor memory.
+// Delta_t is either given (formed from the forward's float32 output, see
+// bwd_delta_kernel) and the kernel makes one sweep over the tile list, or the
+// kernel makes two sweeps: the first forms Delta_t from its own P and dP (so
+// that sum_m dz_tm vanishes to f32 rounding), the second accumulates dq in
+// tensor memory.
 //
 // Roles (352 threads):
 //   warp 0      TMA producer: Q and dout once, then K and V (or kbar and vbar)
-//               of every tile of both sweeps into 2-stage rings;
+//               of every tile of every sweep into 3-stage rings;
 //   warp 1      TMEM allocation; issues S_u = Q K^T into TMEM buffer u & 1;
 //   warp 10     issues dP_u = dout V^T into the same buffer and, in the second
 //               sweep, dQ += dS_u K_u with dS read from TMEM (one warp's issue
@@ -21,7 +23,8 @@
 //               u & 1 == g (buffer g), one thread per query row (TMEM lane):
 //               P and dP from TMEM, Delta partial sums (first sweep) or dS
 //               written to a dS buffer as bf16 (second sweep); the two Delta
-//               partials are combined through shared memory between sweeps;
+//               partials are combined through shared memory between sweeps
+//               (with Delta given, each thread reads its row's value);
 //               the epilogue scales dQ by s and stores it (half the columns
 //               each).
 // TMEM columns: dQ [0, D); buffer b: S [D + 128 b, D + 128 b + 64), dP the next
@@ -92,7 +95,8 @@ __global__ void __launch_bounds__(352, 1)
                      const __grid_constant__ CUtensorMap tm_vbar,
                      const int32_t *__restrict__ idx, const int2 *__restrict__ pairs, int k_sel,
                      int L, int N, int bsub, int Nc, float scale, const float *__restrict__ lse,
-                     float *__restrict__ delta_out, int Lpad, __nv_bfloat16 *__restrict__ dq) {
+                     float *__restrict__ delta, int delta_given, int Lpad,
+                     __nv_bfloat16 *__restrict__ dq) {
   using C = DqTcCfg<D>;
   using namespace sm100;
   extern __shared__ unsigned char smem_raw[];
@@ -233,7 +237,8 @@ __global__ void __launch_bounds__(352, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + C::kOffTmemSlot);
   const int T = misc[0];
-  const int U = 2 * T;                 // both sweeps
+  const int T1 = delta_given ? 0 : T;  // tiles of the Delta sweep
+  const int U = T1 + T;
 
   auto uwait = [&](uint32_t b_addr, uint32_t parity) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(b_addr, parity));
@@ -264,7 +269,7 @@ __global__ void __launch_bounds__(352, 1)
         if (!uwait(bar(C::kBarKEmpty + sl), ((u / C::kStages) - 1) & 1)) { ok = false; break; }
         if (!uwait(bar(C::kBarVEmpty + sl), ((u / C::kStages) - 1) & 1)) { ok = false; break; }
       }
-      const int e = tiles[u < T ? u : u - T];
+      const int e = tiles[u < T1 ? u : u - T1];
       const CUtensorMap *mk = e >= 0 ? &tm_k : &tm_kbar;
       const CUtensorMap *mv = e >= 0 ? &tm_v : &tm_vbar;
       const int row = e >= 0 ? (e >> 2) * 64 : (-e - 1) * 64;
@@ -312,16 +317,16 @@ __global__ void __launch_bounds__(352, 1)
     auto finish = [&](int w) -> bool {
       const int b = w & 1, sl = w % C::kStages;
       if (!uwait(bar(C::kBarPFull + b), (w >> 1) & 1)) return false;
-      if (w >= T) {
+      if (w >= T1) {
         tc_fence_after();
-        const int db = (w - T) & 1;
+        const int db = (w - T1) & 1;
         const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + C::kColDQ, tmem + C::kColDS + 32 * db + kk * 8,
                    smem_desc_sw128(kst + kk * 2048, C::kBoxKBytes, 1024), kIdDQ,
-                   (w > T || kk > 0) ? 1u : 0u);
+                   (w > T1 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::kBarKEmpty + sl));
           tc_commit(bar(C::kBarDsFree + db));
         }
@@ -344,7 +349,7 @@ __global__ void __launch_bounds__(352, 1)
                    smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024),
                    kIdQK, k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarSFull + b));
-          if (u < T) tc_commit(bar(C::kBarKEmpty + sl));
+          if (u < T1) tc_commit(bar(C::kBarKEmpty + sl));
         }
         __syncwarp();
       } else {
@@ -400,26 +405,31 @@ __global__ void __launch_bounds__(352, 1)
     // combine the two warpgroups' Delta partial sums (once, before the first
     // second-sweep tile of this warpgroup, or after its loop)
     auto exchange = [&]() -> bool {
+      if (delta_given) {
+        dfull = valid ? delta[(size_t)bh * Lpad + grow] : 0.f;
+        exchanged = true;
+        return true;
+      }
       delta_sm[g * 128 + row] = dpart;
       mbar_arrive(bar(C::kBarDelta));
       if (!warp_wait(bar(C::kBarDelta), 0)) return false;
       dfull = delta_sm[row] + delta_sm[128 + row];
       // Delta into the padded [BH, Lpad] array (0 for rows past L)
-      if (g == 0 && exists) delta_out[(size_t)bh * Lpad + grow] = valid ? dfull : 0.f;
+      if (g == 0 && exists) delta[(size_t)bh * Lpad + grow] = valid ? dfull : 0.f;
       exchanged = true;
       return true;
     };
     for (int u = g; u < U; u += 2) {
       if (__any_sync(0xffffffffu, misc[1] != 0)) { ok = false; break; }
-      const bool second = u >= T;
+      const bool second = u >= T1;
       if (second && !exchanged && !exchange()) { ok = false; break; }
       if (!warp_wait(bar(C::kBarSFull + g), (u >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      const int e = tiles[second ? u - T : u];
+      const int e = tiles[second ? u - T1 : u];
       const bool centroid = e < 0;
-      // dS of second-sweep tile u goes to dS buffer (u - T) & 1, free once the
+      // dS of second-sweep tile u goes to dS buffer (u - T1) & 1, free once the
       // dQ product of tile u - 2 has completed
-      const int r2 = u - T;
+      const int r2 = u - T1;
       const uint32_t ds_addr = lane_addr + C::kColDS + 32 * (r2 & 1);
       if (second && r2 >= 2 && !warp_wait(bar(C::kBarDsFree + (r2 & 1)), ((r2 - 2) >> 1) & 1)) {
         ok = false;

@@ -275,7 +275,7 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
                                            const int2 *pairs, int k_sel, int BH, int L, int bsub,
                                            float scale, int hyd, int dense, int blockwise,
                                            void *out, int out_f32, float *lse,
-                                           cudaStream_t st) {
+                                           float *o_keep, cudaStream_t st) {
   const int N = ceil_div(L, 64);
   const int Nc = ceil_div(L, 64 * bsub), Ncpad = ceil_div(Nc, 64) * 64;
   const int smem = TcCfg<D>::smem_bytes(N, Nc);
@@ -297,7 +297,7 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   piecewise_attention_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), TcCfg<D>::kThreads, smem, st>>>(
       mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, bsub, Nc, scale, hyd, dense, blockwise,
-      out, out_f32, lse);
+      out, out_f32, lse, o_keep);
   return check_launch();
 }
 
@@ -310,8 +310,8 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
                                         pisa_dtype dt, const float *kbar, const float *vsum,
                                         const float *hbar, const int32_t *idx, int k_sel, int BH,
                                         int L, int d, int bsub, float scale, pisa_mode mode,
-                                        void *out, float *lse, unsigned char *ws,
-                                        cudaStream_t st) {
+                                        void *out, float *lse, float *o_keep,
+                                        unsigned char *ws, cudaStream_t st) {
   // N 64-token tiles; Nc blocks of bsub tiles (the selection's and the
   // centroids' index space); with bsub = 1 they coincide
   const int N = ceil_div(L, 64), nwords = ceil_div(N, 32);
@@ -362,9 +362,11 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   const int of32 = dt == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel,
-                                        BH, L, bsub, scale, hyd, 0, blockwise, out, of32, lse, st);
+                                        BH, L, bsub, scale, hyd, 0, blockwise, out, of32, lse,
+                                        o_keep, st);
   return launch_attention_kernel<64>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel, BH,
-                                     L, bsub, scale, hyd, 0, blockwise, out, of32, lse, st);
+                                     L, bsub, scale, hyd, 0, blockwise, out, of32, lse, o_keep,
+                                     st);
 }
 
 // ---- backward of the zeroth-order variant ------------------------------------
@@ -425,8 +427,9 @@ static pisa_status make_map_f32_rows(CUtensorMap *m, const void *base, uint64_t 
 template <int D>
 static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                               const __nv_bfloat16 *v, const __nv_bfloat16 *dout, const float *lse,
-                              const int32_t *idx, int k_sel, int BH, int L, int bsub, float scale,
-                              const BwdLayout &lay, unsigned char *ws, __nv_bfloat16 *dq,
+                              const float *o32, const int32_t *idx, int k_sel, int BH, int L,
+                              int bsub, float scale, const BwdLayout &lay, unsigned char *ws,
+                              __nv_bfloat16 *dq,
                               __nv_bfloat16 *dk, __nv_bfloat16 *dv, cudaStream_t st) {
   // N 64-token tiles, Nc blocks of bsub tiles (the selection's and the
   // centroids' index space)
@@ -473,8 +476,15 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   PISA_TRY(make_map_f32_rows(&mdel, delta, Lpad, BH));
   PISA_CUDA(cudaFuncSetAttribute(bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dq_smem));
+  if (o32) {
+    // Delta from the forward's float32 output: the dq kernel then makes one sweep
+    bwd_delta_kernel<<<grid_1d((size_t)BH * Lpad * 32, 256), 256, 0, st>>>(dout, o32, L, Lpad, D,
+                                                                          BH, delta);
+    PISA_TRY(check_launch());
+  }
   bwd_dq_tc_kernel<D><<<dim3(P, BH), DqTcCfg<D>::kThreads, dq_smem, st>>>(
-      mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, bsub, Nc, scale, lse, delta, Lpad, dq);
+      mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, bsub, Nc, scale, lse, delta,
+      o32 != nullptr, Lpad, dq);
   PISA_TRY(check_launch());
   // centroid gradients, then the exact keys' dk, dv, both on the tensor cores
   // (the exact pass over the query-tile lists of each key-block pair)
@@ -630,8 +640,9 @@ static pisa_status sparse_attention_checked(const void *q, const void *k, const 
                                             const float *vsum, const float *hbar,
                                             const int32_t *idx, int k_sel, int B, int H, int L,
                                             int d, int block_size, float scale, pisa_mode mode,
-                                            void *out, float *lse, void *workspace,
-                                            size_t ws_bytes, pisa_stream_t stream) {
+                                            void *out, float *lse, float *o_keep,
+                                            void *workspace, size_t ws_bytes,
+                                            pisa_stream_t stream) {
   PISA_TRY(check_shape(B, H, L, d, block_size));
   if (dtype != PISA_BF16 && dtype != PISA_F32) return PISA_ERR_INVALID_ARG;
   if (mode != PISA_MODE_HYD && mode != PISA_MODE_0TH && mode != PISA_MODE_1ST) return PISA_ERR_INVALID_ARG;
@@ -644,11 +655,14 @@ static pisa_status sparse_attention_checked(const void *q, const void *k, const 
       !aligned16(vsum) || !aligned16(hbar) || !idx || !aligned16(workspace))
     return PISA_ERR_INVALID_ARG;
   if (out == q || out == k || out == v) return PISA_ERR_INVALID_ARG;
+  if (o_keep && (!aligned16(o_keep) || (void *)o_keep == out || (const void *)o_keep == q ||
+                 (const void *)o_keep == k || (const void *)o_keep == v))
+    return PISA_ERR_INVALID_ARG;
   if (ws_bytes < sparse_ws(B, H, L, d, dtype)) return PISA_ERR_WORKSPACE;
   const float s = scale == 0.f ? 1.f / std::sqrt((float)d) : scale;
   return run_sparse_attention(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B * H, L, d,
-                              block_size / 64, s, mode, out, lse, (unsigned char *)workspace,
-                              (cudaStream_t)stream);
+                              block_size / 64, s, mode, out, lse, o_keep,
+                              (unsigned char *)workspace, (cudaStream_t)stream);
 }
 
 pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, pisa_dtype dtype,
@@ -657,19 +671,20 @@ pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v, p
                                   int block_size, float scale, pisa_mode mode, void *out,
                                   void *workspace, size_t ws_bytes, pisa_stream_t stream) {
   return sparse_attention_checked(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B, H, L, d,
-                                  block_size, scale, mode, out, nullptr, workspace, ws_bytes,
-                                  stream);
+                                  block_size, scale, mode, out, nullptr, nullptr, workspace,
+                                  ws_bytes, stream);
 }
 
 pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *v,
                                       pisa_dtype dtype, const float *kbar, const float *vsum,
                                       const float *hbar, const int32_t *idx, int k_sel, int B,
                                       int H, int L, int d, int block_size, float scale,
-                                      pisa_mode mode, void *out, float *lse, void *workspace,
-                                      size_t ws_bytes, pisa_stream_t stream) {
+                                      pisa_mode mode, void *out, float *lse, float *out_f32,
+                                      void *workspace, size_t ws_bytes, pisa_stream_t stream) {
   if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u)) return PISA_ERR_INVALID_ARG;
   return sparse_attention_checked(q, k, v, dtype, kbar, vsum, hbar, idx, k_sel, B, H, L, d,
-                                  block_size, scale, mode, out, lse, workspace, ws_bytes, stream);
+                                  block_size, scale, mode, out, lse, out_f32, workspace, ws_bytes,
+                                  stream);
 }
 
 size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int block_size,
@@ -680,7 +695,7 @@ size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int
 }
 
 pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *v,
-                                      const void *dout, const float *lse,
+                                      const void *dout, const float *lse, const float *out_f32,
                                       const float *kbar, const float *vsum, const int32_t *idx,
                                       int k_sel, int B, int H, int L, int d, int block_size,
                                       float scale, void *dq, void *dk, void *dv, void *workspace,
@@ -702,6 +717,9 @@ pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *
       if (p == i) return PISA_ERR_INVALID_ARG;
   }
   if (dq == dk || dq == dv || dk == dv) return PISA_ERR_INVALID_ARG;
+  if (out_f32 && !aligned16(out_f32)) return PISA_ERR_INVALID_ARG;
+  for (void *p : outs)
+    if (out_f32 && p == (const void *)out_f32) return PISA_ERR_INVALID_ARG;
   if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(kbar) || !aligned16(vsum) ||
       !idx || !aligned16(workspace))
     return PISA_ERR_INVALID_ARG;
@@ -721,10 +739,12 @@ pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *
   const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,
                       *v16 = (const __nv_bfloat16 *)v, *g16 = (const __nv_bfloat16 *)dout;
   if (d == 128)
-    return launch_bwd<128>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, block_size / 64, s, lay, ws,
-                           (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, st);
-  return launch_bwd<64>(q16, k16, v16, g16, lse, idx, k_sel, BH, L, block_size / 64, s, lay, ws,
-                        (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, st);
+    return launch_bwd<128>(q16, k16, v16, g16, lse, out_f32, idx, k_sel, BH, L, block_size / 64,
+                           s, lay, ws, (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk,
+                           (__nv_bfloat16 *)dv, st);
+  return launch_bwd<64>(q16, k16, v16, g16, lse, out_f32, idx, k_sel, BH, L, block_size / 64, s,
+                        lay, ws, (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv,
+                        st);
 }
 
 pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void *out, int B,
@@ -782,7 +802,7 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
                       sink_block(sink_idx, N), idx, (float *)scratch, st);
   if (r == PISA_OK)
     r = run_sparse_attention(q, k, v, o.dtype, kbar, vsum, hbar, idx, k_sel, BH, L, d, sub, s,
-                             mode, out, nullptr, scratch, st);
+                             mode, out, nullptr, nullptr, scratch, st);
   if (owned) {
     cudaError_t e = cudaFreeAsync(ws, st);
     if (e != cudaSuccess && r == PISA_OK) {
@@ -836,9 +856,10 @@ pisa_status pisa_dense_attention(const void *q, const void *k, const void *v, vo
   const int of32 = dtype == PISA_F32;
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr,
-                                        nullptr, 0, BH, L, 1, s, 0, 1, 0, out, of32, nullptr, st);
+                                        nullptr, 0, BH, L, 1, s, 0, 1, 0, out, of32, nullptr,
+                                        nullptr, st);
   return launch_attention_kernel<64>(q16, k16, v16, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                     0, BH, L, 1, s, 0, 1, 0, out, of32, nullptr, st);
+                                     0, BH, L, 1, s, 0, 1, 0, out, of32, nullptr, nullptr, st);
 }
 
 pisa_status pisa_block_stats_noalloc(const void *q, const void *k, const void *v,

@@ -163,13 +163,16 @@ pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v,
 /* pisa_sparse_attention that also writes lse [B,H,L] float32 (4-byte
  * aligned): lse_t = ln D_t, the natural log of the denominator above (the
  * same in modes hyd and 0th, which differ only in the numerator).  It is what
- * pisa_sparse_attention_bwd needs from the forward. */
+ * pisa_sparse_attention_bwd needs from the forward.  out_f32 (may be NULL;
+ * else 16-byte aligned, [B,H,L,d], overlapping neither out nor an input)
+ * receives the same output in float32, before the rounding to `dtype`;
+ * given to pisa_sparse_attention_bwd it saves the backward one sweep. */
 pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *v,
                                       pisa_dtype dtype, const float *kbar, const float *vsum,
                                       const float *hbar, const int32_t *idx, int k_sel, int B,
                                       int H, int L, int d, int block_size, float scale,
-                                      pisa_mode mode, void *out, float *lse, void *workspace,
-                                      size_t ws_bytes, pisa_stream_t stream);
+                                      pisa_mode mode, void *out, float *lse, float *out_f32,
+                                      void *workspace, size_t ws_bytes, pisa_stream_t stream);
 
 /* ---- training: gradients of the zeroth-order variant ------------------------ */
 
@@ -187,13 +190,16 @@ size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int
  * so each tail term's gradient reaches every key and value of block j.
  * q, k, v, dout: bf16 [B,H,L,d]; lse from pisa_sparse_attention_fwd on the
  * same q, k, v, kbar, vsum, idx; kbar, vsum: float32 from pisa_block_stats.
- * The forward output itself is not needed: the row term
- * Delta_t = sum_m P_tm (dout_t . value_m) is formed from the recomputed
- * probabilities, consistent with the ones the gradients use.  dq, dk, dv must
- * not overlap any input or one another.  No atomics: bitwise reproducible.
+ * The row term Delta_t = sum_m P_tm (dout_t . value_m) equals dout_t . out_t.
+ * With out_f32 (the forward's float32 output, 16-byte aligned) it is formed
+ * that way; with out_f32 NULL it is formed from the recomputed probabilities
+ * in an extra sweep over the tiles.  The bf16 output alone is not enough:
+ * its rounding, amplified by the cancellation in P (dP - Delta), can move dq
+ * by several per cent on short sequences.  dq, dk, dv must not overlap any
+ * input or one another.  No atomics: bitwise reproducible.
  * `workspace`: pisa_sparse_attention_bwd_workspace_bytes(...) bytes. */
 pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *v,
-                                      const void *dout, const float *lse,
+                                      const void *dout, const float *lse, const float *out_f32,
                                       const float *kbar, const float *vsum, const int32_t *idx,
                                       int k_sel, int B, int H, int L, int d, int block_size,
                                       float scale, void *dq, void *dk, void *dv, void *workspace,
