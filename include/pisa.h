@@ -165,8 +165,12 @@ pisa_status pisa_sparse_attention(const void *q, const void *k, const void *v,
  * same in modes hyd and 0th, which differ only in the numerator).  It is what
  * pisa_sparse_attention_bwd needs from the forward.  out_f32 (may be NULL;
  * else 16-byte aligned, [B,H,L,d], overlapping neither out nor an input)
- * receives the same output in float32, before the rounding to `dtype`;
- * given to pisa_sparse_attention_bwd it saves the backward one sweep. */
+ * receives the output in float32, before its rounding to `dtype`; given to
+ * pisa_sparse_attention_bwd it saves the backward one sweep.  With out_f32
+ * the denominator D_t (and so out and lse) is the sum of the same
+ * bf16-rounded weights the numerator uses: out then differs from the call
+ * without out_f32 at the bf16 rounding level, and dout_t . out_t matches the
+ * backward's probabilities even when one key holds nearly all the weight. */
 pisa_status pisa_sparse_attention_fwd(const void *q, const void *k, const void *v,
                                       pisa_dtype dtype, const float *kbar, const float *vsum,
                                       const float *hbar, const int32_t *idx, int k_sel, int B,
