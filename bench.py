@@ -51,6 +51,8 @@ K3_TRAFFIC = {
     # H=4 ncu captures (dram read + write per launch) scaled by 10 to the 40 heads:
     # Wan-like 300.7 MB, Wan-like with 128-token blocks 296.8 MB
     "7974a8f98dec": {"wan": 3.007e9, "wan_b128": 2.968e9},
+    # after the optional float32 output: Wan-like 302.1 MB, 128-token blocks 297.6 MB
+    "bf19c92395d8": {"wan": 3.021e9, "wan_b128": 2.976e9},
 }
 
 
