@@ -101,3 +101,27 @@ def test_argument_checks_fail_before_any_launch(lib):
     assert lib.pisa_select(None, None, None, 0.0, 0.1, 1, 1, 4, 64, 0.5, 0, None, None, 0,
                            None) == L.PISA_ERR_INVALID_ARG
     assert lib.pisa_status_string(L.PISA_ERR_TIMEOUT).decode().startswith("device-side")
+
+
+def test_float32_output_argument_checks(lib):
+    """The optional float32 output of the training forward, and its use by the
+    backward, are refused before any launch when misaligned or aliased."""
+    q, k, v, out, lse = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    kbar, vsum, hbar, idx, ws = 0x600000, 0x700000, 0x800000, 0x900000, 0xA00000
+
+    def fwd(o32):
+        return lib.pisa_sparse_attention_fwd(q, k, v, L.PISA_BF16, kbar, vsum, hbar, idx, 1, 1,
+                                             1, 128, 128, 64, 0.0, L.PISA_MODE_0TH, out, lse,
+                                             o32, ws, 1 << 40, None)
+
+    assert fwd(0x400004) == L.PISA_ERR_INVALID_ARG      # misaligned
+    assert fwd(out) == L.PISA_ERR_INVALID_ARG           # aliases the output
+    assert fwd(q) == L.PISA_ERR_INVALID_ARG             # aliases an input
+    dq, dk, dv, g = 0xB00000, 0xC00000, 0xD00000, 0xE00000
+
+    def bwd(o32):
+        return lib.pisa_sparse_attention_bwd(q, k, v, g, lse, o32, kbar, vsum, idx, 1, 1, 1, 128,
+                                             128, 64, 0.0, dq, dk, dv, ws, 1 << 40, None)
+
+    assert bwd(0x400004) == L.PISA_ERR_INVALID_ARG      # misaligned
+    assert bwd(dq) == L.PISA_ERR_INVALID_ARG            # a gradient would overwrite it
