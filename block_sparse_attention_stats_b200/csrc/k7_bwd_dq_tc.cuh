@@ -16,19 +16,21 @@
 //   warp 0      TMA producer: Q and dout once, then K and V (or kbar and vbar)
 //               of every tile of every sweep into 3-stage rings;
 //   warp 1      TMEM allocation; issues S_u = Q K^T into TMEM buffer u & 1;
-//   warp 10     issues dP_u = dout V^T into the same buffer and, in the second
-//               sweep, dQ += dS_u K_u with dS read from TMEM (one warp's issue
-//               rate would otherwise bound the kernel);
+//   warp 10     issues dP_u = dout V^T into the same buffer and, in the dq
+//               sweep (the only one when Delta is given), dQ += dS_u K_u with
+//               dS read from TMEM (one warp's issue rate would otherwise bound
+//               the kernel);
 //   warps 2-9   two warpgroups of 4 warps; warpgroup g takes the tiles with
 //               u & 1 == g (buffer g), one thread per query row (TMEM lane):
-//               P and dP from TMEM, Delta partial sums (first sweep) or dS
-//               written to a dS buffer as bf16 (second sweep); the two Delta
+//               P and dP from TMEM, Delta partial sums (Delta sweep) or dS
+//               written to a dS buffer as bf16 (dq sweep); the two Delta
 //               partials are combined through shared memory between sweeps
 //               (with Delta given, each thread reads its row's value);
 //               the epilogue scales dQ by s and stores it (half the columns
 //               each).
 // TMEM columns: dQ [0, D); buffer b: S [D + 128 b, D + 128 b + 64), dP the next
-// 64; dS buffers (packed bf16) [D + 256 + 32 c, D + 256 + 32 c + 32).  Every mbarrier wait is bounded; on a timeout the CTA records the error,
+// 64; dS buffers (packed bf16) [D + 256 + 32 c, D + 256 + 32 c + 32).
+// Every mbarrier wait is bounded; on a timeout the CTA records the error,
 // stops issuing, drains its copies and MMAs, frees TMEM and exits.
 #pragma once
 
