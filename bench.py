@@ -100,8 +100,8 @@ def bwd_flops(wl, idx: torch.Tensor, heads: int = 2, dq_products: int = 3):
     C = -(-N // 64)
     BH = wl.B * wl.H
     k_sel = idx.shape[-1]
-    pairs_alg = wl.L * (k_sel * b + (N - k_sel))
-    alg = BH * 10.0 * d * pairs_alg
+    n_i, exact_keys = _row_key_counts(wl, idx)
+    alg = 10.0 * d * float((n_i * (exact_keys + (N - k_sel))).sum())
     if b != 64:
         return alg, None   # the executed-tile replay models the 64-token-block schedule
     idx_np = idx.reshape(-1, N, k_sel).cpu().numpy()
@@ -124,6 +124,19 @@ def bwd_flops(wl, idx: torch.Tensor, heads: int = 2, dq_products: int = 3):
     return alg, tot * BH / use
 
 
+def _row_key_counts(wl, idx: torch.Tensor):
+    """n_i (tokens of query block i, [N]) and sum_{j in S_i} n_j ([B, H, N]):
+    every block holds b tokens except the last."""
+    b, L = wl.block_size, wl.L
+    N = -(-L // b)
+    k_sel = idx.shape[-1]
+    n_last = L - (N - 1) * b
+    n_i = torch.full((N,), float(b), device=idx.device, dtype=torch.float64)
+    n_i[-1] = n_last
+    last_sel = (idx == N - 1).any(dim=-1).to(torch.float64)        # [B,H,N]
+    return n_i, k_sel * b - (b - n_last) * last_sel
+
+
 def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
     """4d sum_i n_i sum_{S_i} n_j + 4d sum_i n_i |U_i| + [hyd] 2 L d^2, per head, summed.
     Mode 1st reads every key of every unselected block as well: 4d L^2 per head."""
@@ -132,11 +145,7 @@ def k3_algorithmic_flops(wl, idx: torch.Tensor) -> float:
         return 4.0 * d * L * L * wl.B * wl.H
     N = -(-L // b)
     k_sel = idx.shape[-1]
-    n_last = L - (N - 1) * b
-    n_i = torch.full((N,), float(b), device=idx.device, dtype=torch.float64)
-    n_i[-1] = n_last
-    last_sel = (idx == N - 1).any(dim=-1).to(torch.float64)        # [B,H,N]
-    exact_keys = k_sel * b - (b - n_last) * last_sel                   # sum_{S_i} n_j
+    n_i, exact_keys = _row_key_counts(wl, idx)
     exact = 4.0 * d * float((n_i * exact_keys).sum())
     tail = 4.0 * d * float(n_i.sum()) * (N - k_sel) * wl.B * wl.H
     first = (2.0 * L * d * d * wl.B * wl.H) if wl.mode == "hyd" else 0.0

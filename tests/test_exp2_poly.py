@@ -1,8 +1,10 @@
-"""The FMA-pipe 2^x of the fused attention kernel, checked on the CPU.
+"""The FMA-pipe 2^x helper of sm100_primitives.cuh, checked on the CPU.
 
-The kernel computes half of its softmax exponentials with exp2_poly2
-(sm100_primitives.cuh): x = n + f, n = round(x) via the 1.5 * 2^23 constant,
-2^f from a cubic, 2^n added to the exponent bits.  This test replays those
+exp2_poly2 computes 2^x without the special-function unit: x = n + f,
+n = round(x) via the 1.5 * 2^23 constant, 2^f from a cubic, 2^n added to the
+exponent bits.  The shipped kernels do not call it (moving a half or a quarter
+of the softmax exponentials onto it measured slower); it is kept correct for
+kernels that are bound by the special-function unit.  This test replays those
 float32 steps in numpy with the coefficients read from the kernel source and
 bounds the relative error against numpy.exp2 (float64), which must stay far
 below the bf16 resolution (2^-9) of the probabilities it feeds.
