@@ -7,7 +7,7 @@
 // block (a list built beforehand, each entry flagged with which of the two
 // i selected); for a key row whose block i did not select, the probabilities
 // are zero.  With P_tn = exp(s q_t.k_n - lse_t), dP_tn = dout_t . v_n and the
-// row terms Delta_t from the dq kernel:
+// row terms Delta_t (from bwd_delta_kernel or the dq kernel's first sweep):
 //   dV_n += sum_t P_tn dout_t          dK_n += s sum_t P_tn (dP_tn - Delta_t) q_t
 // The epilogue adds the centroid chain terms dkbar_j / n_j, dvbar_j / n_j of
 // the key's block and stores bf16.
@@ -15,7 +15,7 @@
 // Roles (320 threads):
 //   warp 0      TMA producer: K and V of the two key blocks once, then Q_i,
 //               dout_i, lse_i and Delta_i of every listed query block into a
-//               2-stage ring;
+//               3-stage ring;
 //   warp 1      TMEM allocation; one elected lane issues every tcgen05.mma:
 //               S^T_u = K Q_i^T and dP^T_u = V dout_i^T into TMEM buffer u & 1,
 //               then dV += P^T_u dout_i and dK += dS^T_u Q_i with P^T and dS^T
