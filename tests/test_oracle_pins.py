@@ -107,11 +107,12 @@ def test_block_size_one_is_exact(density):
 
 
 @pytest.mark.parametrize("sink", [None, 0, -1])
-def test_identical_keys_per_block_is_exact(sink):
+@pytest.mark.parametrize("b,L", [(8, 60), (128, 300)])
+def test_identical_keys_per_block_is_exact(sink, b, L):
     """All keys of a block equal: exp(s q k_n) = alpha for every n, so the
     zeroth-order tail (alpha vsum, n_j alpha) is exact and H_j = 0; the ragged
-    last block (4 tokens) checks n_j in the denominator."""
-    b, L, d = 8, 60, 6
+    last block (4, or 44, tokens) checks n_j in the denominator."""
+    d = 6
     N = -(-L // b)
     centres = _rand((N, d), 7)
     k = np.repeat(centres, b, axis=0)[:L]
