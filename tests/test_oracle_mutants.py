@@ -40,6 +40,10 @@ MUTANTS = [
      "chosen = np.concatenate([[sink], others])", "chosen = order[:k_sel]"),
     ("k_sel rounded up",
      "math.floor(density * N + 1e-6)", "math.ceil(density * N - 1e-6)"),
+    ("histogram: a value equal to hi kept in the last bin",
+     "h[-1] += int((vals >= hi).sum())", "h[-1] += int((vals > hi).sum())"),
+    ("histogram: deviations not centred",
+     "y = scale * (qi @ (kb - kb.mean(axis=0)).T)", "y = scale * (qi @ kb.T)"),
     ("first block of the exact phase dropped",
      "ex = np.concatenate([np.arange(starts[j], starts[j] + counts[j]) for j in S])",
      "ex = np.concatenate([np.arange(starts[j], starts[j] + counts[j]) for j in S[1:]]"

@@ -465,3 +465,18 @@ def test_tail_histogram_bruteforce_and_identities():
     assert (r["hist_x"] == hx).all() and (r["hist_y"] == hy).all()
     assert r["n"] == n_tot == N * b * (N - 2) * b
     assert abs(r["sum_y"]) < 1e-9
+
+
+def test_tail_histogram_values_on_bin_edges():
+    """Hand-worked: d = 1, s = 1, every query 1, so x is the key itself.  Bins of
+    [-2, 2) are 0.5 wide and half-open; a value on an inner edge starts the next
+    bin, 2 goes to the overflow bin.  Query block 0 (8 tokens) sees block 1's keys
+    -2, -1.5, -1, -0.5, 0, 0.5, 1, 2 -> bins 1..7 and overflow, 8 each; query
+    block 1 sees block 0's keys -3, 3, -2.25, 1.75, 0.25, -0.75, 1.5, -1.25 ->
+    underflow, overflow, underflow, bin 8, bin 5, bin 3, bin 8, bin 2, 8 each."""
+    k = np.array([-3, 3, -2.25, 1.75, 0.25, -0.75, 1.5, -1.25,
+                  -2, -1.5, -1, -0.5, 0, 0.5, 1, 2], dtype=np.float64)[:, None]
+    q = np.ones((16, 1))
+    r = O.tail_score_histogram(q, k, 8, np.array([[0], [1]]), 1.0, -2.0, 2.0, 8)
+    want = 8 * np.array([2, 1, 2, 2, 1, 2, 1, 1, 2, 2])
+    assert r["hist_x"].tolist() == want.tolist()
