@@ -40,6 +40,12 @@ MUTANTS = [
      "chosen = np.concatenate([[sink], others])", "chosen = order[:k_sel]"),
     ("k_sel rounded up",
      "math.floor(density * N + 1e-6)", "math.ceil(density * N - 1e-6)"),
+    ("covariance norm squared",
+     "M[j] = math.sqrt(float(((Hj - hbar) ** 2).sum()))", "M[j] = float(((Hj - hbar) ** 2).sum())"),
+    ("covariance norm of H_j, not of H_j - Hbar",
+     "M[j] = math.sqrt(float(((Hj - hbar) ** 2).sum()))", "M[j] = math.sqrt(float((Hj ** 2).sum()))"),
+    ("covariance weight ignored",
+     "sc = sc + cov_weight * cov[None, :]", "sc = sc + 0.0 * cov[None, :]"),
     ("histogram: a value equal to hi kept in the last bin",
      "h[-1] += int((vals >= hi).sum())", "h[-1] += int((vals > hi).sum())"),
     ("histogram: deviations not centred",
