@@ -94,7 +94,9 @@ def bwd_flops(wl, idx: torch.Tensor, heads: int = 2, dq_products: int = 3):
     the forward's float32 output; five with the extra Delta sweep); the dk/dv
     kernel's 128 x 64 tiles over each key pair's union of query blocks, four
     products each; the centroid instance's 128-centroid x 64-query tiles over
-    every query tile, four products each."""
+    every query tile, four products each.  With 128-token blocks a dq CTA is one
+    query block over its selected blocks' 64-token tiles, and a dk/dv CTA one
+    key block over the 64-token tiles of the query blocks that selected it."""
     b, d = wl.block_size, wl.d
     N = -(-wl.L // b)
     C = -(-N // 64)
@@ -102,12 +104,25 @@ def bwd_flops(wl, idx: torch.Tensor, heads: int = 2, dq_products: int = 3):
     k_sel = idx.shape[-1]
     n_i, exact_keys = _row_key_counts(wl, idx)
     alg = 10.0 * d * float((n_i * (exact_keys + (N - k_sel))).sum())
-    if b != 64:
-        return alg, None   # the executed-tile replay models the 64-token-block schedule
+    if b not in (64, 128):
+        return alg, None
     idx_np = idx.reshape(-1, N, k_sel).cpu().numpy()
     use = min(heads, idx_np.shape[0])
     unit = 2.0 * 64 * 64 * d
     tot = 0.0
+    if b == 128:
+        n64 = -(-wl.L // 64)
+        tiles = np.array([min(2, n64 - 2 * j) for j in range(N)])   # 64-token tiles per block
+        for h in range(use):
+            bits = np.zeros((N, N), dtype=bool)
+            np.put_along_axis(bits, idx_np[h].astype(np.int64), True, axis=1)
+            for i in range(N):
+                chunks = sum(int((~bits[i, c * 64:min(N, c * 64 + 64)]).any()) for c in range(C))
+                tot += dq_products * 2 * unit * (int(tiles[bits[i]].sum()) + chunks)
+            for j in range(N):
+                tot += 4 * 2 * unit * int(tiles[bits[:, j]].sum())
+            tot += 4 * 2 * unit * (-(-C // 2)) * n64
+        return alg, tot * BH / use
     for h in range(use):
         bits = np.zeros((N, N), dtype=bool)
         np.put_along_axis(bits, idx_np[h].astype(np.int64), True, axis=1)
