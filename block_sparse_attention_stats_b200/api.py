@@ -61,7 +61,17 @@ def _qkv_dims(q, k, v):
         raise ValueError("q, k, v must be [B, H, L, d] with equal shapes")
     if q.dtype != k.dtype or q.dtype != v.dtype or q.dtype not in _DT:
         raise ValueError("q, k, v must share dtype bf16 or float32")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous [B, H, L, d] (the library reads rows of d)")
     return q.shape
+
+
+def _require(t, shape, dtype, name):
+    """A tensor argument the library reads or writes as a dense array."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
 
 
 def _workspace(nbytes: int, device) -> torch.Tensor:
@@ -182,6 +192,8 @@ def pisa_sparse_attention_fwd(q, k, v, kbar, vsum, hbar, idx, mode: str = "0th",
     lib = L.load()
     B, H, Ln, d = _qkv_dims(q, k, v)
     k_sel = idx.shape[-1]
+    _require(out_f32, q.shape, torch.float32, "out_f32")
+    _require(lse, (B, H, Ln), torch.float32, "lse")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, H, Ln, dtype=torch.float32, device=q.device) if lse is None else lse
     need = lib.pisa_sparse_attention_workspace_bytes(B, H, Ln, d, block_size, _DT[q.dtype])
@@ -204,8 +216,15 @@ def pisa_sparse_attention_bwd(q, k, v, dout, lse, kbar, vsum, idx, block_size: i
     Delta_t = dout_t . out_t comes from it and dq takes one sweep, else two."""
     lib = L.load()
     B, H, Ln, d = _qkv_dims(q, k, v)
+    if q.dtype != torch.bfloat16:
+        raise ValueError("the backward takes bf16 q, k, v, dout")
+    _require(dout, q.shape, torch.bfloat16, "dout")
+    _require(lse, (B, H, Ln), torch.float32, "lse")
+    _require(out_f32, q.shape, torch.float32, "out_f32")
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
                                                   torch.empty_like(v))
+    for g_, n_ in zip((dq, dk, dv), ("dq", "dk", "dv")):
+        _require(g_, q.shape, torch.bfloat16, n_)
     need = lib.pisa_sparse_attention_bwd_workspace_bytes(B, H, Ln, d, block_size, idx.shape[-1])
     ws = workspace if workspace is not None else _workspace(need, q.device)
     _check("pisa_sparse_attention_bwd", lib.pisa_sparse_attention_bwd(
@@ -221,6 +240,8 @@ class _PiecewiseAttention0th(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, density, block_size, sink_idx, scale):
+        if q.dtype != torch.bfloat16:
+            raise ValueError("piecewise_sparse_attention_0th trains on bf16 q, k, v")
         q, k, v = (x.contiguous() for x in (q, k, v))
         st = pisa_block_stats(q, k, v, block_size)
         idx = pisa_select(st["qbar"], st["kbar"], density, sink_idx, scale=scale)

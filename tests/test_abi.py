@@ -125,3 +125,30 @@ def test_float32_output_argument_checks(lib):
 
     assert bwd(0x400004) == L.PISA_ERR_INVALID_ARG      # misaligned
     assert bwd(dq) == L.PISA_ERR_INVALID_ARG            # a gradient would overwrite it
+
+
+def test_binding_checks_tensor_arguments():
+    """The Python binding refuses, before any pointer is taken, tensors the
+    library would misread: non-contiguous q/k/v, a non-bf16 backward, and
+    side outputs of the wrong dtype or shape."""
+    import torch
+    import block_sparse_attention_stats_b200 as P
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    t = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16).transpose(1, 2)   # [1,2,128,64], strided
+    lse = torch.zeros(1, 2, 128)
+    with pytest.raises(ValueError, match="contiguous"):
+        P.pisa_sparse_attention(t, q, q, None, None, None, torch.zeros(1, 2, 2, 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="bf16"):
+        P.pisa_sparse_attention_bwd(q.float(), q.float(), q.float(), q.float(), lse, None, None,
+                                    torch.zeros(1, 2, 2, 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="dout"):
+        P.pisa_sparse_attention_bwd(q, q, q, q[:, :1], lse, None, None,
+                                    torch.zeros(1, 2, 2, 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="out_f32"):
+        P.pisa_sparse_attention_bwd(q, q, q, q, lse, None, None,
+                                    torch.zeros(1, 2, 2, 1, dtype=torch.int32), out_f32=q)
+    with pytest.raises(ValueError, match="lse"):
+        P.pisa_sparse_attention_fwd(q, q, q, None, None, None,
+                                    torch.zeros(1, 2, 2, 1, dtype=torch.int32), lse=lse[:, :1])
+    with pytest.raises(ValueError, match="bf16"):
+        P.piecewise_sparse_attention_0th(q.float(), q.float(), q.float())
