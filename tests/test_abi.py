@@ -152,3 +152,29 @@ def test_binding_checks_tensor_arguments():
                                     torch.zeros(1, 2, 2, 1, dtype=torch.int32), lse=lse[:, :1])
     with pytest.raises(ValueError, match="bf16"):
         P.piecewise_sparse_attention_0th(q.float(), q.float(), q.float())
+
+
+def test_plain_c_program_links_and_calls_the_abi(lib, tmp_path):
+    """The boundary is a C ABI: a C99 program that includes only include/pisa.h
+    compiles with -pedantic, links against libpisa.so and makes host-side calls
+    (no GPU needed for these)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_pisa.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "pisa.h"\n'
+        "int main(void) {\n"
+        "  printf(\"%d %d %s\\n\", pisa_num_blocks(75600, 64), pisa_num_selected(1182, 0.125),\n"
+        "         pisa_status_string(PISA_ERR_UNSUPPORTED));\n"
+        "  return 0;\n}\n")
+    libdir = os.path.dirname(L.LIB_PATH)
+    exe = tmp_path / "use_pisa"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.dirname(HEADER), str(src), "-o", str(exe), libdir + "/libpisa.so",
+                    "-Wl,-rpath," + libdir], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[:2] == ["1182", "147"]
+    assert len(" ".join(out[2:])) > 0
