@@ -617,6 +617,7 @@ def run_pisa(args, wl):
         f_alg_b, f_exec_b = bwd_flops(wl, idx)
         pk = _peaks()[0]
         p_sus_b = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        p_burst_b = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         ex_tf = f_exec_b / (bms * 1e-3) / 1e12 if f_exec_b else None
         bwd = {"ms": bms, "mode": "0th", "launches": 12 if wl.block_size == 64 else 10,
                "delta": "dout . o from the forward's float32 output (bwd_delta_kernel)",
@@ -625,11 +626,13 @@ def run_pisa(args, wl):
                           "(tcgen05, centroid rows weighted by n_j); "
                           "packing, bitmap, pairing, padding, list kernels",
                "roofline": {"bound": "tensor", "achieved": f_alg_b / (bms * 1e-3) / 1e12,
-                            "peak": p_sus_b, "unit": "TFLOP/s",
-                            "frac": f_alg_b / (bms * 1e-3) / 1e12 / p_sus_b,
+                            "peak": p_burst_b, "peak_kind": "bf16 dense, burst",
+                            "unit": "TFLOP/s",
+                            "frac": f_alg_b / (bms * 1e-3) / 1e12 / p_burst_b,
+                            "frac_vs_sustained": f_alg_b / (bms * 1e-3) / 1e12 / p_sus_b,
                             "algorithmic_tflop": f_alg_b / 1e12,
                             "executed_tflop": f_exec_b / 1e12 if f_exec_b else None,
-                            "executed_frac": ex_tf / p_sus_b if ex_tf else None}}
+                            "executed_frac": ex_tf / p_burst_b if ex_tf else None}}
         del grads, G, o32
 
     # ---- e2e: public API with pinned host buffers ------------------------------
@@ -746,12 +749,16 @@ def run_pisa(args, wl):
         },
         "roofline": {
             "kernel": "piecewise_attention (fused exact + centroid tail + first-order)",
-            "bound": "tensor", "achieved": achieved, "peak": p_sus,
-            "peak_kind": f"bf16 dense, sustained, {peak_kind}", "unit": "TFLOP/s",
-            "frac": achieved / p_sus, "frac_vs_burst": achieved / p_burst,
+            # the kernel is timed launch by launch (tens of ms each, between
+            # other kernels), so the burst peak is its denominator; the
+            # sustained one is kept beside it
+            "bound": "tensor", "achieved": achieved, "peak": p_burst,
+            "peak_kind": f"bf16 dense, burst, {peak_kind}", "unit": "TFLOP/s",
+            "frac": achieved / p_burst, "frac_vs_sustained": achieved / p_sus,
+            "peak_sustained": p_sus,
             "traffic": traffic, "algorithmic_tflop_per_launch": f_alg / 1e12,
             "executed_tflop_per_launch": f_exec / 1e12,
-            "executed_frac": f_exec / (t_k3 * 1e-3) / 1e12 / p_sus,
+            "executed_frac": f_exec / (t_k3 * 1e-3) / 1e12 / p_burst,
             "kernel_src": src,
         },
         "step_roofline": {
@@ -767,6 +774,9 @@ def run_pisa(args, wl):
         "clocks": clocks,
     }
     line["step_roofline"]["frac"] = line["step_roofline"]["t_star_ms"] / t_step
+    # the stated goal for the video shapes: at least half of the roofline
+    line["step_roofline"]["target_frac"] = 0.5
+    line["step_roofline"]["target_met"] = line["step_roofline"]["frac"] >= 0.5
     if e2e:
         line["e2e"] = {"value": weak_scaling_value(world, dense_flops(wl), t_e2e), "unit": UNIT,
                        "ms_per_step": t_e2e, "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],

@@ -527,10 +527,43 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[PISA_NOALLOC_SC
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
+// per device: the array's device address and the unique id of the context it
+// was looked up in (0 = not looked up yet)
 void *g_noalloc_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {0};
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the first call on a device does the lookup).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (cuCtxGetId: ids are never
+// reused within a process), or 0 when there is none or the driver lacks the call.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device.  Looked up with
+// the device current on the first call on each device, and again whenever the
+// device's context has changed since (cudaDeviceReset destroys the context and
+// the array with it; the next context holds a fresh copy at a new address).
 pisa_status noalloc_scratch(void **out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -538,9 +571,14 @@ pisa_status noalloc_scratch(void **out) {
     set_last_error(e);
     return PISA_ERR_CUDA;
   }
-  if (dev < 0 || dev >= kMaxDevices) return PISA_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= kMaxDevices) {
+    t_last_error = "pisa_block_stats_noalloc: device ordinal " + std::to_string(dev) +
+                   " is beyond the " + std::to_string(kMaxDevices) + " devices it supports";
+    return PISA_ERR_UNSUPPORTED;
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) {
@@ -548,6 +586,8 @@ pisa_status noalloc_scratch(void **out) {
       return PISA_ERR_CUDA;
     }
     g_noalloc_ptr[dev] = p;
+    // the lookup makes the device's primary context current if none was
+    g_noalloc_ctx[dev] = current_context_id();
   }
   *out = g_noalloc_ptr[dev];
   return PISA_OK;

@@ -77,29 +77,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of floats on the FMA pipe (offloads the special-function
-// unit).  Method: Cody-Waite style argument split x = n + f with n = round(x)
-// (the 1.5 * 2^23 rounding constant) and f in [-0.5, 0.5]; 2^f from a cubic
-// whose coefficients are a minimax fit of 2^f on [-0.5, 0.5] (iteratively
-// reweighted least squares; max relative error 7.5e-5, below the bf16
-// resolution of the probabilities it feeds); 2^n is added to the exponent
-// field.  Inputs below -126 are clamped (the result is then at most a
-// denormal); inputs must be <= 127.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99992807f, c1 = 0.69326099f, c2 = 0.24261112f, c3 = 0.05517166f;
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 y = add2(x, make_float2(kRound, kRound));
-  const float2 n = add2(y, make_float2(-kRound, -kRound));
-  const float2 f = fma2(n, make_float2(-1.0f, -1.0f), x);
-  float2 p = fma2(make_float2(c3, c3), f, make_float2(c2, c2));
-  p = fma2(p, f, make_float2(c1, c1));
-  p = fma2(p, f, make_float2(c0, c0));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23)));
-}
-
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

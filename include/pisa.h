@@ -284,7 +284,10 @@ size_t pisa_dense_attention_workspace_bytes(int B, int H, int L, int d, pisa_dty
  *    needs 20 MiB.
  *  - The first call on each device looks up that device's address of the
  *    array (cudaGetSymbolAddress) with the device current; make that first
- *    call before any stream capture begins on the device.
+ *    call before any stream capture begins on the device.  A context that
+ *    replaces the device's context (after cudaDeviceReset, say) holds a fresh,
+ *    zero-filled copy of the array at another address: the first call in it
+ *    looks the address up again, so it too belongs before any capture.
  *  - All calls on a device share the one array, which keeps whatever the last
  *    call left there.  Nothing in it needs to start at zero: each call writes
  *    every partial it later reads.  Calls whose kernels may overlap on the GPU

@@ -4,14 +4,12 @@ Some callers cannot allocate device memory: hosts that hand a library only
 the buffers of one call and forbid cudaMalloc, or loops that cannot take the
 device synchronisation an allocation may cause.  For them the library keeps
 the statistics pass's scratch in a static device array.  This file checks,
-through the C ABI, that two calls in a row give the same statistics as the
-workspace entry point pisa_block_stats, and that a shape too large for the
-static array is refused.  It is collected last so that a failure here cannot
-stop the other GPU tests from running.
+through the C ABI, that calls in a row give bit for bit the statistics of the
+workspace entry point pisa_block_stats (same kernels, same reduction order),
+that repeated calls leave the device's free memory unchanged, and that a shape
+too large for the static array is refused.  It is collected last so that a
+failure here cannot stop the other GPU tests from running.
 """
-import ctypes
-
-import numpy as np
 import pytest
 import torch
 
@@ -19,11 +17,21 @@ from workloads import WORKLOADS, generate_qkv
 
 pytestmark = pytest.mark.gpu
 
+KEYS = ("qbar", "kbar", "vsum", "hbar", "cov")
 
-def _close(a, b):
-    a = a.double().cpu().numpy()
-    b = b.double().cpu().numpy()
-    np.testing.assert_allclose(a, b, rtol=1e-4, atol=1e-4 * max(1.0, np.abs(b).max()))
+
+def _outputs(ref):
+    # preallocated outputs of the same shapes, filled with NaN so that an
+    # element the call fails to write cannot match
+    return {k: (None if ref[k] is None else torch.full_like(ref[k], float("nan"))) for k in KEYS}
+
+
+def _assert_equal(got, ref, what):
+    for k in KEYS:
+        if ref[k] is None:
+            assert got[k] is None
+            continue
+        assert torch.equal(got[k], ref[k]), f"{what}: {k} differs from pisa_block_stats"
 
 
 def test_noalloc_block_stats_matches_workspace_entry_point():
@@ -34,19 +42,40 @@ def test_noalloc_block_stats_matches_workspace_entry_point():
 
     lib = _lib.load()
     cases = [
-        # first call: Wan2.1-like rows with 2 heads, bf16, no covariance
-        (WORKLOADS["wan"].with_(H=2), False),
-        # second call in a row: different shape, f32, covariance on; the static
-        # array still holds the first call's partial sums
-        (WORKLOADS["tiny"].with_(L=1000, B=2), True),
+        # Wan2.1-like rows with 2 heads, bf16, no covariance
+        ("wan h2", WORKLOADS["wan"].with_(H=2), False),
+        # a different shape, f32 inputs, covariance on, ragged last block; the
+        # static array still holds the previous call's partial sums
+        ("tiny L1000 B2", WORKLOADS["tiny"].with_(L=1000, B=2), True),
     ]
-    for wl, cov in cases:
+    runs = []
+    for name, wl, cov in cases:
         Q, K, V = (x.cuda() for x in generate_qkv(wl, "cpu"))
-        got = P.pisa_block_stats_noalloc(Q, K, V, wl.block_size, want_cov=cov)
         ref = P.pisa_block_stats(Q, K, V, wl.block_size, want_cov=cov)
+        out = _outputs(ref)
+        got = P.pisa_block_stats_noalloc(Q, K, V, wl.block_size, want_cov=cov, out=out)
         P.pisa_device_status()
-        for key in ("qbar", "kbar", "vsum", "hbar") + (("cov",) if cov else ()):
-            _close(got[key], ref[key])
+        _assert_equal(got, ref, name)
+        runs.append((name, wl, cov, (Q, K, V), ref, out))
+
+    # two more calls in a row, into fresh NaN-filled outputs, with the device's
+    # free memory measured around them: nothing may be allocated
+    for _, _, _, _, _, out in runs:
+        for k in KEYS:
+            if out[k] is not None:
+                out[k].fill_(float("nan"))
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    torch_alloc0 = torch.cuda.memory_allocated()
+    for name, wl, cov, (Q, K, V), ref, out in runs:
+        P.pisa_block_stats_noalloc(Q, K, V, wl.block_size, want_cov=cov, out=out)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
+    assert torch.cuda.memory_allocated() == torch_alloc0
+    P.pisa_device_status()
+    for name, wl, cov, _, ref, out in runs:
+        _assert_equal(out, ref, name + " (second call)")
 
     # a shape whose scratch exceeds the static array is refused up front
     B, H, L, d = 1, 600, 128, 128
