@@ -506,6 +506,39 @@ def run_pisa(args, wl):
                  "replays": greps}
         del g
 
+    # ---- 128-token blocks: the step with the selection inside the fused kernel --
+    fused_select = None
+    if wl.block_size == 128:
+        out2 = torch.empty_like(out)
+
+        def fstep():
+            P.pisa_attention_ex(Q, K, V, wl.density, wl.block_size, wl.sink_idx, wl.mode,
+                                cov_weight=wl.cov_weight, workspace=ws, out=out2,
+                                fuse_select=True)
+
+        for _ in range(3):
+            fstep()
+        torch.cuda.synchronize()
+        freps = max(3, min(args.steps, 10))
+        fev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * freps)]
+        for r_ in range(freps):
+            if l2_flush is not None:
+                l2_flush.zero_()
+            fev[2 * r_].record(stream)
+            fstep()
+            fev[2 * r_ + 1].record(stream)
+        torch.cuda.synchronize()
+        P.pisa_device_status()
+        step()
+        torch.cuda.synchronize()
+        fms = sum(fev[2 * r_].elapsed_time(fev[2 * r_ + 1]) for r_ in range(freps)) / freps
+        fused_select = {"ms_per_step": fms, "steps": freps,
+                        "launches": 2 + (1 if want_cov else 0) + 1 + 1,
+                        "same_output_as_separate_selection": bool(torch.equal(out, out2)),
+                        "path": "statistics, then the fused kernel selecting per CTA "
+                                "(no separate selection step)"}
+        del out2
+
     # ---- per-kernel breakdown (same kernels, step by step through the C ABI) --
     lib = _lib.load()
     mk = lambda n: torch.empty(max(256, int(n)), dtype=torch.uint8, device=dev)
@@ -720,7 +753,8 @@ def run_pisa(args, wl):
     # statistics: pass 1 + hbar reduction (+ covariance pass); selection: scores +
     # top-k; fused step: statistics packing (+ bitmap, overlaps, pairing with
     # 64-token blocks) (+ three f32 -> bf16 copies) + the fused kernel
-    launches_per_step = (2 + (1 if want_cov else 0) + 2
+    n_sel = 1 if N <= 512 else (3 if N <= 2048 else 2)
+    launches_per_step = (2 + (1 if want_cov else 0) + n_sel
                          + (5 if wl.block_size == 64 else 2) + (3 if wl.dtype == "f32" else 0))
     line = {
         "metric": METRIC,
@@ -743,6 +777,10 @@ def run_pisa(args, wl):
                             "frac": stats_bytes(wl) / (part_ms["block_stats"] * 1e-3) / 1e9
                             / peaks.get("hbm_gbs", 6650.0)},
             "select": {"bound": "on-chip (fp32 score contraction, top-k)",
+                       "path": ("fused scores + top-k" if N <= 512 else
+                                "certified: tensor-core approximate scores, float32 scores "
+                                "only inside the error band" if N <= 2048 else
+                                "two-pass: float32 score matrix + radix top-k"),
                        "score_gflop": 2.0 * wl.B * wl.H * N * N * wl.d / 1e9,
                        "score_tflops": 2.0 * wl.B * wl.H * N * N * wl.d
                        / (part_ms["select"] * 1e-3) / 1e12},
@@ -768,6 +806,7 @@ def run_pisa(args, wl):
         },
         "dense_baseline": dense,
         "graph_replay": graph,
+        "fused_select": fused_select,
         "tail_diagnostic": diag,
         "backward_0th": bwd,
         "gpu_launches": launches_per_step * args.steps,

@@ -33,7 +33,8 @@ _P, _I, _Z, _D, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_do
 class PisaOptions(ctypes.Structure):
     _fields_ = [("scale", ctypes.c_float), ("cov_weight", ctypes.c_float),
                 ("dtype", ctypes.c_int), ("workspace", ctypes.c_void_p),
-                ("ws_bytes", ctypes.c_size_t)]
+                ("ws_bytes", ctypes.c_size_t), ("fuse_select", ctypes.c_int),
+                ("idx_out", ctypes.c_void_p)]
 
 
 SIGNATURES = {

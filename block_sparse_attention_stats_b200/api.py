@@ -297,9 +297,13 @@ def pisa_attention_ex(q, k, v, density: float, block_size: int = 64,
                       sink_idx: Optional[int] = None, mode: str = "hyd",
                       scale: Optional[float] = None, cov_weight: float = 0.0,
                       workspace: Optional[torch.Tensor] = None,
-                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                      out: Optional[torch.Tensor] = None, stream=None,
+                      fuse_select: bool = False,
+                      idx_out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """pisa_attention with options; the workspace (if given) is caller-owned scratch
-    of pisa_workspace_bytes(...) bytes and nothing is allocated by the library."""
+    of pisa_workspace_bytes(...) bytes and nothing is allocated by the library.
+    fuse_select (block_size 128): each CTA of the fused kernel selects its own
+    exact blocks.  idx_out: int32 [B, H, N, k_sel] receiving the selection used."""
     lib = L.load()
     B, H, Ln, d = _qkv_dims(q, k, v)
     out = torch.empty_like(q) if out is None else out
@@ -307,6 +311,15 @@ def pisa_attention_ex(q, k, v, density: float, block_size: int = 64,
     opts.scale = 0.0 if scale is None else float(scale)
     opts.cov_weight = float(cov_weight)
     opts.dtype = _DT[q.dtype]
+    opts.fuse_select = int(bool(fuse_select))
+    if idx_out is not None:
+        N = lib.pisa_num_blocks(Ln, block_size)
+        shape = (B, H, N, lib.pisa_num_selected(N, float(density)))
+        if idx_out.dtype != torch.int32 or tuple(idx_out.shape) != shape \
+                or not idx_out.is_contiguous() or idx_out.device != q.device:
+            raise ValueError(f"idx_out must be a contiguous int32 tensor of shape {shape} "
+                             "on the inputs' device")
+        opts.idx_out = _ptr(idx_out)
     if workspace is not None:
         opts.workspace = _ptr(workspace)
         opts.ws_bytes = workspace.numel() * workspace.element_size()

@@ -22,6 +22,7 @@
 #pragma once
 
 #include "pisa_common.cuh"
+#include "sm100_primitives.cuh"
 
 namespace pisa {
 
@@ -238,6 +239,323 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
       *reinterpret_cast<float2 *>(P + (size_t)(a0 + 8) * D + c0) =
           make_float2(acc[mt][nt][2], acc[mt][nt][3]);
     }
+}
+
+// ---------------------------------------------------------------------------
+// bf16 pass 1, streamed: one CTA per SM walks a contiguous range of the
+// B*H*N blocks (its range may end inside a head and the next CTA's begin
+// there), with Q, K and V tiles arriving by TMA (cp.async.bulk.tensor, no
+// multicast) into a four-stage mbarrier ring.  Warp 0 issues the copies;
+// warps 1-8 form column sums and K^T V with the tensor cores (mma.sync; the
+// pass is bound by HBM, at 64 flop per byte) exactly as the chunked kernel
+// above, and write one partial sum of H_j per head segment.  Segment s of head
+// bh is the s-th CTA whose range meets that head; hbar_reduce_seg_kernel adds
+// a head's segments in order, so the result is bitwise reproducible.
+// ---------------------------------------------------------------------------
+constexpr int kStatsCtas = 148;       // one per SM of a B200
+constexpr int kStatsStages = 4;
+
+__host__ __device__ inline int stats_stream_ctas(long long total_blocks) {
+  return total_blocks < kStatsCtas ? (int)total_blocks : kStatsCtas;
+}
+// first global block (bh * N + j) of CTA c's range
+__host__ __device__ inline long long stats_first_block(int c, long long total, int nc) {
+  return (long long)c * total / nc;
+}
+// the CTA whose range holds global block G
+__host__ __device__ inline int stats_cta_of(long long G, long long total, int nc) {
+  return (int)(((G + 1) * nc + total - 1) / total) - 1;
+}
+// an upper bound on the CTAs whose range meets one head of N blocks
+__host__ __device__ inline int stats_max_segments(int BH, int N) {
+  const long long total = (long long)BH * N;
+  const int nc = stats_stream_ctas(total);
+  long long per = total / nc;
+  if (per < 1) per = 1;
+  return (int)(N / per) + 2;
+}
+
+template <int D> struct StatsTmaCfg {
+  static constexpr int kThreads = 32 * 9;
+  static constexpr int kTileBytes = kBlk * D * 2;           // one 64-token tile of one tensor
+  static constexpr int kStageBytes = 3 * kTileBytes;        // Q, K, V
+  static constexpr int kOffColsum = kStatsStages * kStageBytes;
+  static constexpr int kOffBar = kOffColsum + 3 * D * 4;
+  static constexpr int kOffMisc = kOffBar + 2 * kStatsStages * 8;
+  static constexpr int kSmem = kOffMisc + 16 + 1024;        // + alignment slack
+};
+
+// byte offset of (row, col) in a tile written by TMA with the 128-byte swizzle
+// in 64-column boxes (64 rows x 128 bytes each)
+__device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
+  return (uint32_t)((col >> 6) * (kBlk * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
+                    (col & 7) * 2);
+}
+
+template <int D>
+__device__ __forceinline__ void ktv_mma_sw128(
+    float (&acc)[StatsMmaCfg<D>::kMT][StatsMmaCfg<D>::kNT][4], uint32_t sK, uint32_t sV,
+    int warp_m0, int warp_n0, int lane) {
+  using C = StatsMmaCfg<D>;
+  const int mi = lane >> 3, r = lane & 7;
+#pragma unroll
+  for (int k0 = 0; k0 < kBlk; k0 += 16) {
+    uint32_t a[C::kMT][4];
+#pragma unroll
+    for (int mt = 0; mt < C::kMT; ++mt) {
+      const int tok = k0 + r + 8 * (mi >> 1);
+      const int dim = warp_m0 + mt * 16 + 8 * (mi & 1);
+      ldmatrix_x4_trans(sK + sw128_offset(tok, dim), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < C::kNT; nt += 2) {
+      const int tok = k0 + r + 8 * (mi & 1);
+      const int dim = warp_n0 + nt * 8 + 8 * (mi >> 1);
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(sV + sw128_offset(tok, dim), b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < C::kMT; ++mt) {
+        mma_bf16_16816(acc[mt][nt], a[mt], b0, b1);
+        mma_bf16_16816(acc[mt][nt + 1], a[mt], b2, b3);
+      }
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void colsum_mma_sw128(uint32_t tiles, float *colsum, int warp,
+                                                 int lane, bool accumulate) {
+  using C = StatsMmaCfg<D>;
+  constexpr int kNT = 3 * D / 8;
+  constexpr int kPerWarp = kNT / 8;
+  const uint32_t one2 = 0x3F803F80u;
+  const uint32_t ones[4] = {one2, one2, one2, one2};
+  float acc[kPerWarp][4];
+#pragma unroll
+  for (int i = 0; i < kPerWarp; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+  const int mi = lane >> 3, r = lane & 7;
+#pragma unroll
+  for (int k0 = 0; k0 < kBlk; k0 += 16) {
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+      const int nt = warp * kPerWarp + i;
+      const int which = nt / (D / 8), col = (nt % (D / 8)) * 8;
+      const int tok = k0 + r + 8 * (mi & 1);
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(tiles + which * C::kTileBytes + sw128_offset(tok, col), b0, b1, b2, b3);
+      (void)b2;
+      (void)b3;
+      mma_bf16_16816(acc[i], ones, b0, b1);
+    }
+  }
+  if (lane < 4) {
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+      const int nt = warp * kPerWarp + i;
+      const int which = nt / (D / 8), col = (nt % (D / 8)) * 8 + 2 * lane;
+      colsum[which * D + col] = accumulate ? colsum[which * D + col] + acc[i][0] : acc[i][0];
+      colsum[which * D + col + 1] =
+          accumulate ? colsum[which * D + col + 1] + acc[i][1] : acc[i][1];
+    }
+  }
+}
+
+__device__ __forceinline__ void stats_consumer_barrier() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(32 * 9, 1)
+    stats_pass_tma_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, int L, int N, int sub,
+                          int BH, int maxseg, float *__restrict__ qbar,
+                          float *__restrict__ kbar, float *__restrict__ vsum,
+                          float *__restrict__ partial) {
+  using C = StatsMmaCfg<D>;
+  using T = StatsTmaCfg<D>;
+  using namespace sm100;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  unsigned char *smem = smem_raw + (sbase - raw);
+  float *colsum = reinterpret_cast<float *>(smem + T::kOffColsum);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + T::kOffMisc);
+  volatile int *cflag = abort_flag + 1;   // [2]: consumers' abort, by tile parity
+  auto full = [&](int s) -> uint32_t { return sbase + T::kOffBar + 8 * s; };
+  auto empty = [&](int s) -> uint32_t { return sbase + T::kOffBar + 8 * (kStatsStages + s); };
+
+  const long long total = (long long)BH * N;
+  const int nc = gridDim.x, c = blockIdx.x;
+  const long long g0 = stats_first_block(c, total, nc), g1 = stats_first_block(c + 1, total, nc);
+  const int ntile = ceil_div(L, kBlk);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
+  // tiles of global block G: j * sub .. (the last block may have only the first)
+  auto tiles_of = [&](long long G) -> int {
+    const int j = (int)(G % N);
+    const int u0 = j * sub;
+    return min(sub, ntile - u0);
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < kStatsStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 8);
+    }
+    fence_mbar_init();
+    abort_flag[0] = 0;
+    abort_flag[1] = 0;
+    abort_flag[2] = 0;
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ======================= TMA producer =====================================
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int t = 0;
+      bool ok = true;
+      for (long long G = g0; ok && G < g1; ++G) {
+        const int bh = (int)(G / N), j = (int)(G % N);
+        const int nt = tiles_of(G);
+        for (int s = 0; s < nt; ++s, ++t) {
+          const int slot = t % kStatsStages;
+          if (t >= kStatsStages && !mbar_wait(empty(slot), ((t / kStatsStages) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          if (*abort_flag) { ok = false; break; }
+          const uint32_t dst = sbase + slot * T::kStageBytes;
+          const int row = (j * sub + s) * kBlk;
+          mbar_expect_tx(full(slot), T::kStageBytes);
+#pragma unroll
+          for (int b = 0; b < D / 64; ++b) {
+            tma_load_3d(dst + b * (kBlk * 128), &tm_q, full(slot), 64 * b, row, bh);
+            tma_load_3d(dst + T::kTileBytes + b * (kBlk * 128), &tm_k, full(slot), 64 * b, row, bh);
+            tma_load_3d(dst + 2 * T::kTileBytes + b * (kBlk * 128), &tm_v, full(slot), 64 * b, row,
+                        bh);
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // copies in flight land before the CTA exits (at most one per stage)
+        for (int u = (t >= kStatsStages ? t - kStatsStages : 0); u < t; ++u)
+          mbar_wait(full(u % kStatsStages), (u / kStatsStages) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ======================= consumers ========================================
+    const int cw = warp - 1, ctid = tid - 32;
+    const int warp_m0 = (cw / C::kWarpsN) * C::kWarpRows;
+    const int warp_n0 = (cw % C::kWarpsN) * C::kWarpCols;
+    const int g = lane >> 2, tq = lane & 3;
+    float acc[C::kMT][C::kNT][4];
+    auto zero_acc = [&]() {
+#pragma unroll
+      for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::kNT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    };
+    auto flush = [&](int bh) {
+      const int seg = c - stats_cta_of((long long)bh * N, total, nc);
+      float *P = partial + ((size_t)bh * maxseg + seg) * D * D;
+#pragma unroll
+      for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::kNT; ++nt) {
+          const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
+          *reinterpret_cast<float2 *>(P + (size_t)a0 * D + c0) =
+              make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+          *reinterpret_cast<float2 *>(P + (size_t)(a0 + 8) * D + c0) =
+              make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+        }
+    };
+    zero_acc();
+    int cur_bh = (int)(g0 / N);
+    int t = 0;
+    bool ok = true;
+    for (long long G = g0; ok && G < g1; ++G) {
+      const int bh = (int)(G / N), j = (int)(G % N);
+      if (bh != cur_bh) {
+        flush(cur_bh);
+        zero_acc();
+        cur_bh = bh;
+      }
+      const int nt = tiles_of(G);
+      for (int s = 0; s < nt; ++s, ++t) {
+        const int slot = t % kStatsStages;
+        const bool got = __all_sync(0xffffffffu, mbar_wait(full(slot), (t / kStatsStages) & 1));
+        // every consumer warp takes the same decision: the flag of this tile's
+        // parity is written only before this barrier and read only after it
+        if (!got) {
+          cflag[t & 1] = 1;
+          *abort_flag = 1;   // the producer stops too
+        }
+        stats_consumer_barrier();
+        if (cflag[t & 1]) { ok = false; break; }
+        const uint32_t st = sbase + slot * T::kStageBytes;
+        // column sums of Q, K, V (rows past L were filled with zeros), summed
+        // over the tiles of block j
+        colsum_mma_sw128<D>(st, colsum, cw, lane, s > 0);
+        ktv_mma_sw128<D>(acc, st + T::kTileBytes, st + 2 * T::kTileBytes, warp_m0, warp_n0, lane);
+        // this warp has read the stage
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(slot));
+        stats_consumer_barrier();   // column sums complete
+        if (s == nt - 1) {
+          const int n_j = min(sub * kBlk, L - j * sub * kBlk);
+          const float inv_n = 1.f / (float)n_j;
+          const size_t so = ((size_t)bh * N + j) * D;
+          for (int e = ctid; e < 3 * D; e += 256) {
+            const int which = e / D, col = e % D;
+            if (which == 0) qbar[so + col] = colsum[e] * inv_n;
+            else if (which == 1) kbar[so + col] = colsum[e] * inv_n;
+            else vsum[so + col] = colsum[e];
+          }
+          // acc -= kbar_j^T vsum_j
+#pragma unroll
+          for (int mt = 0; mt < C::kMT; ++mt)
+#pragma unroll
+            for (int nt2 = 0; nt2 < C::kNT; ++nt2) {
+              const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt2 * 8 + 2 * tq;
+              const float ka = colsum[D + a0] * inv_n, kb = colsum[D + a0 + 8] * inv_n;
+              const float v0 = colsum[2 * D + c0], v1 = colsum[2 * D + c0 + 1];
+              acc[mt][nt2][0] -= ka * v0;
+              acc[mt][nt2][1] -= ka * v1;
+              acc[mt][nt2][2] -= kb * v0;
+              acc[mt][nt2][3] -= kb * v1;
+            }
+          stats_consumer_barrier();   // column sums free for the next block
+        }
+      }
+    }
+    if (ok && g0 < g1) flush(cur_bh);
+  }
+}
+
+// pass 2 of the streamed pass: hbar = (1/N) sum of the head's segment partials,
+// in segment order.
+__global__ void hbar_reduce_seg_kernel(const float *__restrict__ partial, int maxseg, int DD,
+                                       int N, int BH, int nc, float *__restrict__ hbar) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= DD) return;
+  const long long total = (long long)BH * N;
+  const int c0 = stats_cta_of((long long)bh * N, total, nc);
+  const int c1 = stats_cta_of((long long)(bh + 1) * N - 1, total, nc);
+  const float *p = partial + (size_t)bh * maxseg * DD + e;
+  float s = 0.f;
+  for (int seg = 0; seg <= c1 - c0; ++seg) s += p[(size_t)seg * DD];
+  hbar[(size_t)bh * DD + e] = s / (float)N;
 }
 
 // ---------------------------------------------------------------------------

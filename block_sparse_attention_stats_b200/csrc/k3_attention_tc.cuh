@@ -43,10 +43,24 @@
 // frees TMEM and exits.
 #pragma once
 
+#include "k2_select.cuh"
 #include "pisa_common.cuh"
 #include "sm100_primitives.cuh"
 
 namespace pisa {
+
+// Selection inside the fused kernel (128-token blocks only, where a CTA is one
+// query block and needs no partner): the CTA scores its own pooled query
+// against every block centroid, in the same float32 order as scores_kernel,
+// and takes the top k_sel with the sink forced in, exactly as pisa_select.
+struct FusedSelect {
+  const float *qbar;   // [BH, Nc, D] (NULL: the selection comes from idx)
+  const float *kbar;   // [BH, Nc, D]
+  const float *cov;    // [BH, Nc] or NULL
+  float cov_weight;
+  int sink;            // forced block, or -1
+  int32_t *idx_out;    // optional [BH, Nc, k_sel] copy of the selection
+};
 
 template <int D> struct TcCfg {
   static constexpr int kThreads = 192;
@@ -112,7 +126,8 @@ __global__ void __launch_bounds__(192, 2)
                                   const int2 *__restrict__ pairs, int k_sel, int L, int N,
                                   int bsub, int Nc, float scale, int hyd, int dense, int blockwise,
                                   void *__restrict__ out, int out_f32,
-                                  float *__restrict__ lse, float *__restrict__ o_keep) {
+                                  float *__restrict__ lse, float *__restrict__ o_keep,
+                                  const FusedSelect fsel) {
   using C = TcCfg<D>;
   using namespace sm100;
   extern __shared__ unsigned char smem_raw[];
@@ -207,6 +222,40 @@ __global__ void __launch_bounds__(192, 2)
     // one selection row for the 128-token query block: block j covers the
     // 64-token tiles 2j and 2j + 1 (the last block may have only the first)
     const int32_t *r0 = idx + ((size_t)bh * Nc + sr0) * k_sel;
+    if (fsel.qbar != nullptr) {
+      // select here: scores of this query block against every centroid (the
+      // tile list's space holds them and, after them, the selected indices;
+      // the V ring, not yet in use, holds the pooled query and the radix
+      // histogram)
+      float *sc = reinterpret_cast<float *>(tiles);
+      int32_t *sel = tiles + Nc;
+      float *qrow = reinterpret_cast<float *>(smem + C::kOffV);
+      unsigned *hist = reinterpret_cast<unsigned *>(smem + C::kOffV + D * 4);
+      const float *qb = fsel.qbar + ((size_t)bh * Nc + sr0) * D;
+      for (int e = tid; e < D; e += C::kThreads) qrow[e] = qb[e];
+      __syncthreads();
+      for (int j = tid; j < Nc; j += C::kThreads) {
+        const float4 *kr = reinterpret_cast<const float4 *>(fsel.kbar + ((size_t)bh * Nc + j) * D);
+        float acc = 0.f;
+#pragma unroll 8
+        for (int e4 = 0; e4 < D / 4; ++e4) {
+          const float4 kv = __ldg(kr + e4);
+          acc = fmaf(qrow[4 * e4 + 0], kv.x, acc);
+          acc = fmaf(qrow[4 * e4 + 1], kv.y, acc);
+          acc = fmaf(qrow[4 * e4 + 2], kv.z, acc);
+          acc = fmaf(qrow[4 * e4 + 3], kv.w, acc);
+        }
+        const float cw = fsel.cov_weight != 0.f ? fsel.cov_weight * fsel.cov[(size_t)bh * Nc + j] : 0.f;
+        sc[j] = fmaf(scale, acc, cw);
+      }
+      __syncthreads();
+      if (tid < 32) topk_row(sc, Nc, k_sel, fsel.sink, hist, sel, lane);
+      __syncthreads();
+      if (fsel.idx_out != nullptr)
+        for (int t = tid; t < k_sel; t += C::kThreads)
+          fsel.idx_out[((size_t)bh * Nc + sr0) * k_sel + t] = sel[t];
+      r0 = sel;
+    }
     for (int t = tid; t < k_sel; t += C::kThreads) {
       const int j = r0[t];
       if (j >= 0 && j < Nc) {

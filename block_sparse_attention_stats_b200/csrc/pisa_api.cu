@@ -15,6 +15,7 @@
 #include "pisa_common.cuh"
 #include "k1_block_stats.cuh"
 #include "k2_select.cuh"
+#include "k2_select_tc.cuh"
 #include "k3_pack.cuh"
 #include "k3_attention_tc.cuh"
 #include "k5_tail_histogram.cuh"
@@ -89,13 +90,32 @@ static bool sink_valid(int sink_idx) {
 }
 
 // ---- scratch sizes --------------------------------------------------------
+// chunk partials of the f32 pass, or head-segment partials of the streamed bf16 pass
 static size_t stats_ws(int B, int H, int L, int d, int block_size) {
   const int N = ceil_div(L, block_size), BH = B * H;
-  return align_up((size_t)BH * stats_num_chunks(BH, N) * d * d * sizeof(float), 256);
+  const int parts = std::max(stats_num_chunks(BH, N), stats_max_segments(BH, N));
+  return align_up((size_t)BH * parts * d * d * sizeof(float), 256);
 }
-static size_t select_ws(int B, int H, int N) {
-  return align_up((size_t)B * H * N * N * sizeof(float), 256);
+// selection scratch: the float32 score matrix of the two-pass path, or for
+// the certified path (512 < N <= 2048) the approximate scores with rows padded
+// to 128 columns, the two bf16 terms of qbar and kbar (head dimension up to
+// 128) and the row norms
+struct SelectLayout {
+  size_t approx, q16, k16, qn, kn, total;
+};
+static SelectLayout select_layout(int B, int H, int N) {
+  const size_t BH = (size_t)B * H, Npad = (size_t)ceil_div(N, kCertTile) * kCertTile;
+  SelectLayout p;
+  size_t o = 0;
+  p.approx = o; o += align_up(BH * N * Npad * sizeof(float), 256);
+  p.q16 = o; o += align_up(2 * BH * Npad * 128 * 2, 256);   // high and low bf16 terms
+  p.k16 = o; o += align_up(2 * BH * Npad * 128 * 2, 256);
+  p.qn = o; o += align_up(BH * N * sizeof(float), 256);
+  p.kn = o; o += align_up(BH * N * sizeof(float), 256);
+  p.total = o;
+  return p;
 }
+static size_t select_ws(int B, int H, int N) { return select_layout(B, H, N).total; }
 // scratch of the fused-attention step: bf16 kbar/vsum/hbar, query-block
 // pairing (selection bitmaps, overlaps, pairs), bf16 copies of f32 inputs
 struct SparseLayout {
@@ -154,6 +174,9 @@ static unsigned grid_1d(size_t n, int threads) {
   return (unsigned)(b ? b : 1);
 }
 
+static pisa_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                            uint64_t planes, uint32_t box_rows);
+
 // ---- launches ---------------------------------------------------------------
 template <int D>
 static pisa_status launch_stats(const void *q, const void *k, const void *v, pisa_dtype dt,
@@ -164,12 +187,23 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
   const int nchunk = stats_num_chunks(BH, N);
   dim3 grid(nchunk, BH);
   if (dt == PISA_BF16) {
-    const int smem = 2 * 3 * StatsMmaCfg<D>::kTileBytes + 3 * D * (int)sizeof(float);
-    PISA_CUDA(cudaFuncSetAttribute(stats_pass_bf16_kernel<D>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    stats_pass_bf16_kernel<D><<<grid, kStatsThreads, smem, st>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N, sub,
-        nchunk, qbar, kbar, vsum, partial);
+    // one CTA per SM streams a contiguous range of blocks through a TMA ring
+    const long long total = (long long)BH * N;
+    const int nc = stats_stream_ctas(total);
+    const int maxseg = stats_max_segments(BH, N);
+    CUtensorMap mq, mk, mv;
+    PISA_TRY(make_map(&mq, q, D, L, BH, kBlk));
+    PISA_TRY(make_map(&mk, k, D, L, BH, kBlk));
+    PISA_TRY(make_map(&mv, v, D, L, BH, kBlk));
+    PISA_CUDA(cudaFuncSetAttribute(stats_pass_tma_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   StatsTmaCfg<D>::kSmem));
+    stats_pass_tma_kernel<D><<<nc, StatsTmaCfg<D>::kThreads, StatsTmaCfg<D>::kSmem, st>>>(
+        mq, mk, mv, L, N, sub, BH, maxseg, qbar, kbar, vsum, partial);
+    PISA_TRY(check_launch());
+    hbar_reduce_seg_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(
+        partial, maxseg, D * D, N, BH, nc, hbar);
+    PISA_TRY(check_launch());
   } else {
     const int smem = 3 * kBlk * D * (int)sizeof(float) + 3 * D * (int)sizeof(float);
     PISA_CUDA(cudaFuncSetAttribute(stats_pass_f32_kernel<D>,
@@ -177,11 +211,11 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
     stats_pass_f32_kernel<D><<<grid, kStatsThreads, smem, st>>>(
         (const float *)q, (const float *)k, (const float *)v, L, N, sub, nchunk, qbar, kbar,
         vsum, partial);
+    PISA_TRY(check_launch());
+    hbar_reduce_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(partial, nchunk, D * D,
+                                                                        N, hbar);
+    PISA_TRY(check_launch());
   }
-  PISA_TRY(check_launch());
-  hbar_reduce_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(partial, nchunk, D * D, N,
-                                                                      hbar);
-  PISA_TRY(check_launch());
   if (want_cov) {
     if (dt == PISA_BF16) {
       const int smem = 2 * 2 * StatsMmaCfg<D>::kTileBytes + 32 * (int)sizeof(float);
@@ -202,9 +236,45 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
   return PISA_OK;
 }
 
+// certified selection (k2_select_tc.cuh): pack, approximate scores on the
+// tensor cores, exact float32 scores only where the bound cannot decide
+template <int D>
+static pisa_status launch_select_certified(const float *qbar, const float *kbar,
+                                           const float *cov, float cov_weight, float scale,
+                                           int BH, int N, int k_sel, int sink, int32_t *idx,
+                                           unsigned char *ws, cudaStream_t st) {
+  const SelectLayout lay = select_layout(1, BH, N);
+  const int Npad = ceil_div(N, kCertTile) * kCertTile;
+  float *approx = (float *)(ws + lay.approx);
+  __nv_bfloat16 *q16 = (__nv_bfloat16 *)(ws + lay.q16), *k16 = (__nv_bfloat16 *)(ws + lay.k16);
+  float *qn = (float *)(ws + lay.qn), *kn = (float *)(ws + lay.kn);
+  const size_t pack_threads = (size_t)2 * BH * Npad * 32;
+  select_pack_kernel<D><<<grid_1d(pack_threads, 256), 256, 0, st>>>(qbar, kbar, N, Npad, BH, q16,
+                                                                   k16, qn, kn);
+  PISA_TRY(check_launch());
+  CUtensorMap mq, mk;
+  PISA_TRY(make_map(&mq, q16, D, Npad, 2 * BH, kCertTile));
+  PISA_TRY(make_map(&mk, k16, D, Npad, 2 * BH, kCertTile));
+  PISA_CUDA(cudaFuncSetAttribute(select_approx_tc_kernel<D>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SelTcCfg<D>::kSmem));
+  select_approx_tc_kernel<D><<<dim3(Npad / kCertTile, BH), SelTcCfg<D>::kThreads,
+                               SelTcCfg<D>::kSmem, st>>>(mq, mk, cov, cov_weight, scale, N, Npad,
+                                                         BH, approx);
+  PISA_TRY(check_launch());
+  const size_t rows = (size_t)BH * N;
+  const unsigned blocks = (unsigned)((rows + kCertWarps - 1) / kCertWarps);
+  const int csmem = certified_smem(N, D);
+  PISA_CUDA(cudaFuncSetAttribute(select_certified_kernel<D>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, csmem));
+  select_certified_kernel<D><<<blocks, kCertWarps * 32, csmem, st>>>(
+      approx, Npad, qbar, kbar, qn, kn, cov, cov_weight, scale, N, k_sel, sink, rows, idx);
+  return check_launch();
+}
+
 static pisa_status launch_select(const float *qbar, const float *kbar, const float *cov,
                                  float cov_weight, float scale, int BH, int N, int d, int k_sel,
-                                 int sink, int32_t *idx, float *scores, cudaStream_t st) {
+                                 int sink, int32_t *idx, unsigned char *ws, cudaStream_t st) {
+  float *scores = (float *)ws;
   const int fsmem = select_fused_smem(N, d);
   if (N <= kSelFusedMaxN && fsmem <= 227 * 1024) {
     // short sequences: the score rows of a query-block group stay in shared
@@ -215,6 +285,15 @@ static pisa_status launch_select(const float *qbar, const float *kbar, const flo
     select_fused_kernel<<<dim3(ceil_div(N, kSelRows), BH), kSelThreads, fsmem, st>>>(
         qbar, kbar, cov, cov_weight, scale, N, d, k_sel, sink, idx);
     return check_launch();
+  }
+  if (N <= kCertMaxN) {
+    // long rows: most scores are decided by the tensor-core approximation and
+    // its error bound; the float32 score is formed only near the threshold
+    if (d == 128)
+      return launch_select_certified<128>(qbar, kbar, cov, cov_weight, scale, BH, N, k_sel, sink,
+                                          idx, ws, st);
+    return launch_select_certified<64>(qbar, kbar, cov, cov_weight, scale, BH, N, k_sel, sink,
+                                       idx, ws, st);
   }
   dim3 g1(ceil_div(N, kScoreTile), ceil_div(N, kScoreTile), BH);
   scores_kernel<<<g1, 256, 0, st>>>(qbar, kbar, cov, cov_weight, scale, N, d, scores);
@@ -275,7 +354,8 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
                                            const int2 *pairs, int k_sel, int BH, int L, int bsub,
                                            float scale, int hyd, int dense, int blockwise,
                                            void *out, int out_f32, float *lse,
-                                           float *o_keep, cudaStream_t st) {
+                                           float *o_keep, cudaStream_t st,
+                                           const FusedSelect &fsel = FusedSelect{}) {
   const int N = ceil_div(L, 64);
   const int Nc = ceil_div(L, 64 * bsub), Ncpad = ceil_div(Nc, 64) * 64;
   const int smem = TcCfg<D>::smem_bytes(N, Nc);
@@ -297,7 +377,7 @@ static pisa_status launch_attention_kernel(const __nv_bfloat16 *q, const __nv_bf
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   piecewise_attention_tc_kernel<D><<<dim3(ceil_div(N, 2), BH), TcCfg<D>::kThreads, smem, st>>>(
       mq, mk, mv, mkb, mvs, mh, idx, pairs, k_sel, L, N, bsub, Nc, scale, hyd, dense, blockwise,
-      out, out_f32, lse, o_keep);
+      out, out_f32, lse, o_keep, fsel);
   return check_launch();
 }
 
@@ -311,7 +391,8 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
                                         const float *hbar, const int32_t *idx, int k_sel, int BH,
                                         int L, int d, int bsub, float scale, pisa_mode mode,
                                         void *out, float *lse, float *o_keep,
-                                        unsigned char *ws, cudaStream_t st) {
+                                        unsigned char *ws, cudaStream_t st,
+                                        const FusedSelect &fsel = FusedSelect{}) {
   // N 64-token tiles; Nc blocks of bsub tiles (the selection's and the
   // centroids' index space); with bsub = 1 they coincide
   const int N = ceil_div(L, 64), nwords = ceil_div(N, 32);
@@ -363,10 +444,10 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   if (d == 128)
     return launch_attention_kernel<128>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel,
                                         BH, L, bsub, scale, hyd, 0, blockwise, out, of32, lse,
-                                        o_keep, st);
+                                        o_keep, st, fsel);
   return launch_attention_kernel<64>(q16, k16, v16, kbar16, vsum16, hbar16, idx, pairs, k_sel, BH,
                                      L, bsub, scale, hyd, 0, blockwise, out, of32, lse, o_keep,
-                                     st);
+                                     st, fsel);
 }
 
 // ---- backward of the zeroth-order variant ------------------------------------
@@ -672,7 +753,8 @@ pisa_status pisa_select(const float *qbar, const float *kbar, const float *cov, 
   if (cov_weight != 0.f && !cov) return PISA_ERR_INVALID_ARG;
   if (ws_bytes < select_ws(B, H, N)) return PISA_ERR_WORKSPACE;
   return launch_select(qbar, kbar, cov, cov_weight, scale, B * H, N, d, k_sel,
-                       sink_block(sink_idx, N), idx, (float *)workspace, (cudaStream_t)stream);
+                       sink_block(sink_idx, N), idx, (unsigned char *)workspace,
+                       (cudaStream_t)stream);
 }
 
 static pisa_status sparse_attention_checked(const void *q, const void *k, const void *v,
@@ -800,10 +882,12 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
   if (!(o.scale >= 0.f) || !std::isfinite(o.scale) || !std::isfinite(o.cov_weight))
     return PISA_ERR_INVALID_ARG;
   if (mode == PISA_MODE_1ST && block_size != 64) return PISA_ERR_UNSUPPORTED;
+  if (o.fuse_select && block_size != 128) return PISA_ERR_UNSUPPORTED;
   if (!fused_fits(d, L, block_size)) return PISA_ERR_UNSUPPORTED;
   const int N = ceil_div(L, block_size);
   const int k_sel = pisa_num_selected(N, density);
   if (k_sel < 1) return PISA_ERR_INVALID_ARG;
+  if (o.idx_out && ((uintptr_t)o.idx_out & 3u)) return PISA_ERR_INVALID_ARG;
   if ((long long)N * 4 > 200 * 1024) return PISA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return PISA_ERR_INVALID_ARG;
@@ -827,22 +911,31 @@ pisa_status pisa_attention_ex(const void *q, const void *k, const void *v, void 
   float *qbar = (float *)(ws + p.qbar), *kbar = (float *)(ws + p.kbar),
         *vsum = (float *)(ws + p.vsum), *hbar = (float *)(ws + p.hbar),
         *cov = want_cov ? (float *)(ws + p.cov) : nullptr;
-  int32_t *idx = (int32_t *)(ws + p.idx);
+  int32_t *idx = o.idx_out ? o.idx_out : (int32_t *)(ws + p.idx);
   unsigned char *scratch = ws + p.scratch;
   pisa_status r;
   const int sub = block_size / 64;
+  FusedSelect fsel{};
+  if (o.fuse_select) {
+    fsel.qbar = qbar;
+    fsel.kbar = kbar;
+    fsel.cov = cov;
+    fsel.cov_weight = o.cov_weight;
+    fsel.sink = sink_block(sink_idx, N);
+    fsel.idx_out = o.idx_out;
+  }
   if (d == 128)
     r = launch_stats<128>(q, k, v, o.dtype, BH, L, sub, want_cov, qbar, kbar, vsum, hbar, cov,
                           (float *)scratch, st);
   else
     r = launch_stats<64>(q, k, v, o.dtype, BH, L, sub, want_cov, qbar, kbar, vsum, hbar, cov,
                          (float *)scratch, st);
-  if (r == PISA_OK)
+  if (r == PISA_OK && !o.fuse_select)
     r = launch_select(qbar, kbar, cov, o.cov_weight, s, BH, N, d, k_sel,
-                      sink_block(sink_idx, N), idx, (float *)scratch, st);
+                      sink_block(sink_idx, N), idx, (unsigned char *)scratch, st);
   if (r == PISA_OK)
     r = run_sparse_attention(q, k, v, o.dtype, kbar, vsum, hbar, idx, k_sel, BH, L, d, sub, s,
-                             mode, out, nullptr, nullptr, scratch, st);
+                             mode, out, nullptr, nullptr, scratch, st, fsel);
   if (owned) {
     cudaError_t e = cudaFreeAsync(ws, st);
     if (e != cudaSuccess && r == PISA_OK) {

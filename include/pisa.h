@@ -86,6 +86,14 @@ typedef struct {
   pisa_dtype dtype;   /* dtype of q, k, v and out */
   void *workspace;    /* device scratch; NULL = allocate per call (stream-ordered) */
   size_t ws_bytes;    /* size of `workspace` */
+  int fuse_select;    /* block_size 128 only (else PISA_ERR_UNSUPPORTED): no
+                         separate selection step; each CTA of the fused kernel,
+                         which holds one query block, scores that block against
+                         every centroid and takes its own top k_sel (the same
+                         float32 scores, tie rule and sink as pisa_select, so
+                         the same sets) before its exact tiles start */
+  int32_t *idx_out;   /* optional (NULL = not wanted): device [B,H,N,k_sel] int32,
+                         4-byte aligned, receives the selection the call used */
 } pisa_options;
 
 /* ---- sizes ------------------------------------------------------------- */

@@ -48,6 +48,18 @@ def test_num_blocks_and_selected_match_oracle(lib):
     assert lib.pisa_num_blocks(0, 64) == -1
 
 
+def test_selection_workspace_covers_every_path(lib):
+    """The selection scratch holds the float32 score matrix of the two-pass
+    path and, for the certified path, the approximate scores with rows padded
+    to 128 columns, two bf16 terms of qbar and of kbar and two norm vectors."""
+    for BH, N in ((40, 1182), (24, 1861), (24, 72), (1, 2100), (3, 600)):
+        need = lib.pisa_select_workspace_bytes(1, BH, N)
+        npad = -(-N // 128) * 128
+        assert need >= BH * N * N * 4
+        assert need >= BH * N * npad * 4 + 4 * BH * npad * 128 * 2 + 2 * BH * N * 4
+        assert need % 256 == 0
+
+
 def test_workspace_sizes(lib):
     w = lib.pisa_workspace_bytes(1, 40, 75600, 128, 64, 0.125, L.PISA_BF16, 0)
     assert w > 0 and w % 256 == 0
@@ -98,6 +110,13 @@ def test_argument_checks_fail_before_any_launch(lib):
     o = L.PisaOptions()
     o.scale = float("nan")
     assert _attn(lib, opts=o) == L.PISA_ERR_INVALID_ARG
+    # selection inside the fused kernel needs 128-token blocks; idx_out 4-byte aligned
+    o = L.PisaOptions()
+    o.fuse_select = 1
+    assert _attn(lib, opts=o) == L.PISA_ERR_UNSUPPORTED
+    o = L.PisaOptions()
+    o.idx_out = 0x5002
+    assert _attn(lib, bs=128, opts=o) == L.PISA_ERR_INVALID_ARG
     assert lib.pisa_select(None, None, None, 0.0, 0.1, 1, 1, 4, 64, 0.5, 0, None, None, 0,
                            None) == L.PISA_ERR_INVALID_ARG
     assert lib.pisa_status_string(L.PISA_ERR_TIMEOUT).decode().startswith("device-side")

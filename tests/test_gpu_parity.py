@@ -113,6 +113,52 @@ def test_block_size_128(P, L, d, sink, mode, cov):
     assert _run_case(P, wl) == 0
 
 
+@pytest.mark.parametrize("L,d,sink,mode,cov", [
+    (4608, 128, -1, "hyd", 0.1),    # FLUX-like shape, 36 blocks of 128 tokens
+    (1000, 128, None, "hyd", 0.0),  # last block 104 tokens
+    (4673, 128, -1, "0th", 0.1),    # last block 65 tokens
+    (900, 64, 0, "hyd", 0.1),       # odd tile count, d = 64
+    (129, 128, -1, "hyd", 0.0),     # N = 2
+    (100, 64, None, "0th", 0.0),    # N = 1
+    (70000, 128, None, "hyd", 0.0), # 547 blocks: the separate step takes its certified path
+])
+def test_block_size_128_selection_in_fused_kernel(P, L, d, sink, mode, cov):
+    """With 128-token blocks the fused kernel can select inside (each CTA is
+    one query block): the sets equal the separate selection step's bit for
+    bit (same float32 scores and tie rule), so does the output, and both
+    match the oracle."""
+    wl = WORKLOADS["flux"].with_(B=1, H=2, L=L, d=d, block_size=128, sink_idx=sink, mode=mode,
+                                 cov_weight=cov, cluster_kind="block", density=0.2)
+    Q, K, V = generate_qkv(wl, "cpu")
+    q, k, v = (x.cuda() for x in (Q, K, V))
+    N = -(-L // 128)
+    k_sel = O.num_selected(N, wl.density)
+    idx_f = torch.full((1, 2, N, k_sel), -1, dtype=torch.int32, device="cuda")
+    idx_s = torch.full_like(idx_f, -1)
+    out_f = P.pisa_attention_ex(q, k, v, wl.density, 128, sink, mode, cov_weight=cov,
+                                fuse_select=True, idx_out=idx_f)
+    out_s = P.pisa_attention_ex(q, k, v, wl.density, 128, sink, mode, cov_weight=cov,
+                                idx_out=idx_s)
+    P.pisa_device_status()
+    assert torch.equal(idx_f, idx_s)
+    assert torch.equal(out_f, out_s)
+    heads = [(0, 0), (0, 1)] if L < 20000 else [(0, 1)]
+    for (b, h) in heads:
+        r = O.pisa_attention_head(to64(Q[b, h]), to64(K[b, h]), to64(V[b, h]), 128, wl.density,
+                                  sink, mode, cov_weight=cov)
+        rep = compare_selection(idx_f[b, h].cpu().numpy(), r, wl.scale, cov, sink)
+        assert not rep.bad_rows and not rep.tie_rows, (rep.bad_rows, rep.tie_rows)
+        ma, rf = output_errors(to64(out_f[b, h]), r["out"])
+        assert ma <= MAX_ABS_TOL and rf <= REL_FRO_TOL, (h, ma, rf)
+
+
+def test_selection_in_fused_kernel_needs_128_token_blocks(P):
+    wl = WORKLOADS["flux"].with_(H=1, L=1000, cluster_kind="block")
+    Q, K, V = (x.cuda() for x in generate_qkv(wl, "cpu"))
+    with pytest.raises(RuntimeError):
+        P.pisa_attention_ex(Q, K, V, wl.density, 64, wl.sink_idx, "hyd", fuse_select=True)
+
+
 def test_block_size_128_f32(P):
     """f32 inputs with 128-token blocks (the f32 statistics kernels)."""
     assert _run_case(P, WORKLOADS["tiny"].with_(block_size=128, cov_weight=0.1)) == 0
