@@ -53,6 +53,8 @@ K3_TRAFFIC = {
     "7974a8f98dec": {"wan": 3.007e9, "wan_b128": 2.968e9},
     # after the optional float32 output: Wan-like 302.1 MB, 128-token blocks 297.6 MB
     "bf19c92395d8": {"wan": 3.021e9, "wan_b128": 2.976e9},
+    # with the in-kernel selection option (unused by this workload): Wan-like 301.3 MB
+    "26564cebed3a": {"wan": 3.013e9},
 }
 
 
@@ -753,7 +755,7 @@ def run_pisa(args, wl):
     # statistics: pass 1 + hbar reduction (+ covariance pass); selection: scores +
     # top-k; fused step: statistics packing (+ bitmap, overlaps, pairing with
     # 64-token blocks) (+ three f32 -> bf16 copies) + the fused kernel
-    n_sel = 1 if N <= 512 else (3 if N <= 2048 else 2)
+    n_sel = 1 if N <= 512 else 2
     launches_per_step = (2 + (1 if want_cov else 0) + n_sel
                          + (5 if wl.block_size == 64 else 2) + (3 if wl.dtype == "f32" else 0))
     line = {
@@ -778,8 +780,6 @@ def run_pisa(args, wl):
                             / peaks.get("hbm_gbs", 6650.0)},
             "select": {"bound": "on-chip (fp32 score contraction, top-k)",
                        "path": ("fused scores + top-k" if N <= 512 else
-                                "certified: tensor-core approximate scores, float32 scores "
-                                "only inside the error band" if N <= 2048 else
                                 "two-pass: float32 score matrix + radix top-k"),
                        "score_gflop": 2.0 * wl.B * wl.H * N * N * wl.d / 1e9,
                        "score_tflops": 2.0 * wl.B * wl.H * N * N * wl.d

@@ -244,13 +244,21 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
 // ---------------------------------------------------------------------------
 // bf16 pass 1, streamed: one CTA per SM walks a contiguous range of the
 // B*H*N blocks (its range may end inside a head and the next CTA's begin
-// there), with Q, K and V tiles arriving by TMA (cp.async.bulk.tensor, no
-// multicast) into a four-stage mbarrier ring.  Warp 0 issues the copies;
-// warps 1-8 form column sums and K^T V with the tensor cores (mma.sync; the
-// pass is bound by HBM, at 64 flop per byte) exactly as the chunked kernel
-// above, and write one partial sum of H_j per head segment.  Segment s of head
-// bh is the s-th CTA whose range meets that head; hbar_reduce_seg_kernel adds
-// a head's segments in order, so the result is bitwise reproducible.
+// there).  Q, K and V tiles arrive by TMA (cp.async.bulk.tensor, no multicast)
+// into a four-stage mbarrier ring.
+//   warp 0      issues the copies;
+//   warp 1      allocates TMEM and issues G_j = K_j^T V_j of each block as
+//               tcgen05 MMAs (M = N = D, both operands MN-major straight from
+//               the tiles, 16 tokens per MMA) into one of two TMEM buffers;
+//   warps 2-9   sum the columns of Q, K and V on the CUDA cores (float32, in
+//               token order), write qbar, kbar, vsum at the end of each block,
+//               then read G_j back and add G_j - kbar_j^T vsum_j to a float32
+//               register accumulator of sum_j H_j (warps w and w + 4 take the
+//               rows of TMEM sub-partition w % 4 and half of the columns each).
+// The accumulator goes to the partial of the head segment (segment s of head
+// bh is the s-th CTA whose range meets that head) when the head changes;
+// hbar_reduce_seg_kernel adds a head's segments in order, so the result is
+// bitwise reproducible.
 // ---------------------------------------------------------------------------
 constexpr int kStatsCtas = 148;       // one per SM of a B200
 constexpr int kStatsStages = 4;
@@ -276,116 +284,47 @@ __host__ __device__ inline int stats_max_segments(int BH, int N) {
 }
 
 template <int D> struct StatsTmaCfg {
-  static constexpr int kThreads = 32 * 9;
+  static constexpr int kThreads = 32 * 10;
   static constexpr int kTileBytes = kBlk * D * 2;           // one 64-token tile of one tensor
   static constexpr int kStageBytes = 3 * kTileBytes;        // Q, K, V
-  static constexpr int kOffColsum = kStatsStages * kStageBytes;
-  static constexpr int kOffBar = kOffColsum + 3 * D * 4;
-  static constexpr int kOffMisc = kOffBar + 2 * kStatsStages * 8;
+  static constexpr int kBoxBytes = kBlk * 128;              // 64 tokens x 64 columns
+  // kbar_j and vsum_j of the block being finished, double-buffered by block parity
+  static constexpr int kOffKV = kStatsStages * kStageBytes;
+  static constexpr int kOffBar = kOffKV + 2 * 2 * D * 4;
+  // bars: full[4], empty[4], gfull[2], gempty[2], teardown
+  static constexpr int kNumBars = 2 * kStatsStages + 5;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kOffMisc = kOffTmemSlot + 16;
   static constexpr int kSmem = kOffMisc + 16 + 1024;        // + alignment slack
+  static constexpr uint32_t kTmemCols = 2 * D < 32 ? 32 : 2 * D;   // two G buffers
 };
-
-// byte offset of (row, col) in a tile written by TMA with the 128-byte swizzle
-// in 64-column boxes (64 rows x 128 bytes each)
-__device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
-  return (uint32_t)((col >> 6) * (kBlk * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
-                    (col & 7) * 2);
-}
-
-template <int D>
-__device__ __forceinline__ void ktv_mma_sw128(
-    float (&acc)[StatsMmaCfg<D>::kMT][StatsMmaCfg<D>::kNT][4], uint32_t sK, uint32_t sV,
-    int warp_m0, int warp_n0, int lane) {
-  using C = StatsMmaCfg<D>;
-  const int mi = lane >> 3, r = lane & 7;
-#pragma unroll
-  for (int k0 = 0; k0 < kBlk; k0 += 16) {
-    uint32_t a[C::kMT][4];
-#pragma unroll
-    for (int mt = 0; mt < C::kMT; ++mt) {
-      const int tok = k0 + r + 8 * (mi >> 1);
-      const int dim = warp_m0 + mt * 16 + 8 * (mi & 1);
-      ldmatrix_x4_trans(sK + sw128_offset(tok, dim), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-    }
-#pragma unroll
-    for (int nt = 0; nt < C::kNT; nt += 2) {
-      const int tok = k0 + r + 8 * (mi & 1);
-      const int dim = warp_n0 + nt * 8 + 8 * (mi >> 1);
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4_trans(sV + sw128_offset(tok, dim), b0, b1, b2, b3);
-#pragma unroll
-      for (int mt = 0; mt < C::kMT; ++mt) {
-        mma_bf16_16816(acc[mt][nt], a[mt], b0, b1);
-        mma_bf16_16816(acc[mt][nt + 1], a[mt], b2, b3);
-      }
-    }
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void colsum_mma_sw128(uint32_t tiles, float *colsum, int warp,
-                                                 int lane, bool accumulate) {
-  using C = StatsMmaCfg<D>;
-  constexpr int kNT = 3 * D / 8;
-  constexpr int kPerWarp = kNT / 8;
-  const uint32_t one2 = 0x3F803F80u;
-  const uint32_t ones[4] = {one2, one2, one2, one2};
-  float acc[kPerWarp][4];
-#pragma unroll
-  for (int i = 0; i < kPerWarp; ++i)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
-  const int mi = lane >> 3, r = lane & 7;
-#pragma unroll
-  for (int k0 = 0; k0 < kBlk; k0 += 16) {
-#pragma unroll
-    for (int i = 0; i < kPerWarp; ++i) {
-      const int nt = warp * kPerWarp + i;
-      const int which = nt / (D / 8), col = (nt % (D / 8)) * 8;
-      const int tok = k0 + r + 8 * (mi & 1);
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4_trans(tiles + which * C::kTileBytes + sw128_offset(tok, col), b0, b1, b2, b3);
-      (void)b2;
-      (void)b3;
-      mma_bf16_16816(acc[i], ones, b0, b1);
-    }
-  }
-  if (lane < 4) {
-#pragma unroll
-    for (int i = 0; i < kPerWarp; ++i) {
-      const int nt = warp * kPerWarp + i;
-      const int which = nt / (D / 8), col = (nt % (D / 8)) * 8 + 2 * lane;
-      colsum[which * D + col] = accumulate ? colsum[which * D + col] + acc[i][0] : acc[i][0];
-      colsum[which * D + col + 1] =
-          accumulate ? colsum[which * D + col + 1] + acc[i][1] : acc[i][1];
-    }
-  }
-}
 
 __device__ __forceinline__ void stats_consumer_barrier() {
   asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(32 * 9, 1)
+__global__ void __launch_bounds__(32 * 10, 1)
     stats_pass_tma_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, int L, int N, int sub,
                           int BH, int maxseg, float *__restrict__ qbar,
                           float *__restrict__ kbar, float *__restrict__ vsum,
                           float *__restrict__ partial) {
-  using C = StatsMmaCfg<D>;
   using T = StatsTmaCfg<D>;
   using namespace sm100;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   unsigned char *smem = smem_raw + (sbase - raw);
-  float *colsum = reinterpret_cast<float *>(smem + T::kOffColsum);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + T::kOffMisc);
-  volatile int *cflag = abort_flag + 1;   // [2]: consumers' abort, by tile parity
-  auto full = [&](int s) -> uint32_t { return sbase + T::kOffBar + 8 * s; };
-  auto empty = [&](int s) -> uint32_t { return sbase + T::kOffBar + 8 * (kStatsStages + s); };
+  volatile int *cflag = abort_flag + 1;   // [2]: consumers' abort, by block parity
+  auto bar = [&](int i) -> uint32_t { return sbase + T::kOffBar + 8 * i; };
+  auto full = [&](int s) { return bar(s); };
+  auto empty = [&](int s) { return bar(kStatsStages + s); };
+  auto gfull = [&](int g) { return bar(2 * kStatsStages + g); };
+  auto gempty = [&](int g) { return bar(2 * kStatsStages + 2 + g); };
+  const uint32_t teardown = bar(2 * kStatsStages + 4);
 
   const long long total = (long long)BH * N;
   const int nc = gridDim.x, c = blockIdx.x;
@@ -393,24 +332,34 @@ __global__ void __launch_bounds__(32 * 9, 1)
   const int ntile = ceil_div(L, kBlk);
   const int tid = threadIdx.x, lane = tid & 31;
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
-  // tiles of global block G: j * sub .. (the last block may have only the first)
   auto tiles_of = [&](long long G) -> int {
     const int j = (int)(G % N);
-    const int u0 = j * sub;
-    return min(sub, ntile - u0);
+    return min(sub, ntile - j * sub);
   };
 
+  if (warp == 1) {
+    tmem_alloc(sbase + T::kOffTmemSlot, T::kTmemCols);
+    tmem_relinquish();
+  }
   if (tid == 0) {
     for (int s = 0; s < kStatsStages; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), 8);
+      mbar_init(empty(s), 1 + 8);     // the MMA commit and the eight consumer warps
     }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(gfull(g), 1);
+      mbar_init(gempty(g), 8);
+    }
+    mbar_init(teardown, 1);
     fence_mbar_init();
     abort_flag[0] = 0;
     abort_flag[1] = 0;
     abort_flag[2] = 0;
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + T::kOffTmemSlot);
 
   if (warp == 0) {
     // ======================= TMA producer =====================================
@@ -435,9 +384,9 @@ __global__ void __launch_bounds__(32 * 9, 1)
           mbar_expect_tx(full(slot), T::kStageBytes);
 #pragma unroll
           for (int b = 0; b < D / 64; ++b) {
-            tma_load_3d(dst + b * (kBlk * 128), &tm_q, full(slot), 64 * b, row, bh);
-            tma_load_3d(dst + T::kTileBytes + b * (kBlk * 128), &tm_k, full(slot), 64 * b, row, bh);
-            tma_load_3d(dst + 2 * T::kTileBytes + b * (kBlk * 128), &tm_v, full(slot), 64 * b, row,
+            tma_load_3d(dst + b * T::kBoxBytes, &tm_q, full(slot), 64 * b, row, bh);
+            tma_load_3d(dst + T::kTileBytes + b * T::kBoxBytes, &tm_k, full(slot), 64 * b, row, bh);
+            tma_load_3d(dst + 2 * T::kTileBytes + b * T::kBoxBytes, &tm_v, full(slot), 64 * b, row,
                         bh);
           }
         }
@@ -450,95 +399,148 @@ __global__ void __launch_bounds__(32 * 9, 1)
       }
     }
     __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================================
+    if (lane == 0) {
+      // G = K^T V: A = K^T (M = D dimensions, MN-major), B = V (N = D, MN-major);
+      // 16 tokens (2048 bytes of a 128-byte-row tile) per instruction
+      constexpr uint32_t kId = idesc_bf16_f32(128, D, 1, 1);
+      int t = 0, blk = 0;
+      bool ok = true;
+      for (long long G = g0; ok && G < g1; ++G, ++blk) {
+        const int g = blk & 1;
+        // the consumers have read G of block blk - 2 out of this buffer
+        if (blk >= 2 && !mbar_wait(gempty(g), ((blk >> 1) - 1) & 1)) { ok = false; break; }
+        const int nt = tiles_of(G);
+        for (int s = 0; s < nt; ++s, ++t) {
+          const int slot = t % kStatsStages;
+          if (!mbar_wait(full(slot), (t / kStatsStages) & 1)) { ok = false; break; }
+          if (*abort_flag) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kst = sbase + slot * T::kStageBytes + T::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBlk / 16; ++kk)
+            mma_ss(tmem + D * g, smem_desc_sw128(kst + kk * 2048, T::kBoxBytes, 1024),
+                   smem_desc_sw128(kst + T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kId,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(empty(slot));
+        }
+        if (ok) tc_commit(gfull(g));
+      }
+      if (!ok) *abort_flag = 1;
+      // every MMA issued must finish before TMEM is released
+      tc_commit(teardown);
+      mbar_wait(teardown, 0);
+    }
+    __syncwarp();
   } else {
     // ======================= consumers ========================================
-    const int cw = warp - 1, ctid = tid - 32;
-    const int warp_m0 = (cw / C::kWarpsN) * C::kWarpRows;
-    const int warp_n0 = (cw % C::kWarpsN) * C::kWarpCols;
-    const int g = lane >> 2, tq = lane & 3;
-    float acc[C::kMT][C::kNT][4];
-    auto zero_acc = [&]() {
+    const int cw = warp - 2, ctid = tid - 64;
+    const int sp = warp & 3, ch = cw >> 2;      // TMEM sub-partition, column half of G
+    const int arow = sp * 32 + lane;            // row of G (a key dimension)
+    constexpr int kH = D / 2;                   // columns of G per thread
+    float hacc[kH];
 #pragma unroll
-      for (int mt = 0; mt < C::kMT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < C::kNT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-    };
+    for (int i = 0; i < kH; ++i) hacc[i] = 0.f;
+    // column sums: thread p < 3 D / 2 owns the column pair (2 lp, 2 lp + 1) of
+    // tensor p / (D / 2) (Q, K or V)
+    const int p = ctid, tns = p / (D / 2), lp = p % (D / 2);
+    const bool sums = p < 3 * (D / 2);
+    const uint32_t col_off = (uint32_t)(tns * T::kTileBytes + (lp / 32) * T::kBoxBytes);
+    const int chunk = (lp % 32) / 4, inword = (lp % 4) * 4;
+    float cs0 = 0.f, cs1 = 0.f;
     auto flush = [&](int bh) {
       const int seg = c - stats_cta_of((long long)bh * N, total, nc);
-      float *P = partial + ((size_t)bh * maxseg + seg) * D * D;
+      float *P = partial + ((size_t)bh * maxseg + seg) * D * D + (size_t)arow * D + ch * kH;
 #pragma unroll
-      for (int mt = 0; mt < C::kMT; ++mt)
+      for (int i = 0; i < kH; i += 4)
+        *reinterpret_cast<float4 *>(P + i) = make_float4(hacc[i], hacc[i + 1], hacc[i + 2], hacc[i + 3]);
 #pragma unroll
-        for (int nt = 0; nt < C::kNT; ++nt) {
-          const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt * 8 + 2 * tq;
-          *reinterpret_cast<float2 *>(P + (size_t)a0 * D + c0) =
-              make_float2(acc[mt][nt][0], acc[mt][nt][1]);
-          *reinterpret_cast<float2 *>(P + (size_t)(a0 + 8) * D + c0) =
-              make_float2(acc[mt][nt][2], acc[mt][nt][3]);
-        }
+      for (int i = 0; i < kH; ++i) hacc[i] = 0.f;
     };
-    zero_acc();
     int cur_bh = (int)(g0 / N);
-    int t = 0;
+    int t = 0, blk = 0;
     bool ok = true;
-    for (long long G = g0; ok && G < g1; ++G) {
-      const int bh = (int)(G / N), j = (int)(G % N);
+    for (long long G = g0; ok && G < g1; ++G, ++blk) {
+      const int bh = (int)(G / N), j = (int)(G % N), g = blk & 1;
       if (bh != cur_bh) {
         flush(cur_bh);
-        zero_acc();
         cur_bh = bh;
       }
       const int nt = tiles_of(G);
+      bool bad = false;
       for (int s = 0; s < nt; ++s, ++t) {
         const int slot = t % kStatsStages;
-        const bool got = __all_sync(0xffffffffu, mbar_wait(full(slot), (t / kStatsStages) & 1));
-        // every consumer warp takes the same decision: the flag of this tile's
-        // parity is written only before this barrier and read only after it
-        if (!got) {
-          cflag[t & 1] = 1;
-          *abort_flag = 1;   // the producer stops too
+        if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (t / kStatsStages) & 1))) {
+          bad = true;
+          break;
         }
-        stats_consumer_barrier();
-        if (cflag[t & 1]) { ok = false; break; }
-        const uint32_t st = sbase + slot * T::kStageBytes;
-        // column sums of Q, K, V (rows past L were filled with zeros), summed
-        // over the tiles of block j
-        colsum_mma_sw128<D>(st, colsum, cw, lane, s > 0);
-        ktv_mma_sw128<D>(acc, st + T::kTileBytes, st + 2 * T::kTileBytes, warp_m0, warp_n0, lane);
-        // this warp has read the stage
+        if (sums) {
+          const uint32_t base = sbase + slot * T::kStageBytes + col_off + inword;
+#pragma unroll 8
+          for (int r = 0; r < kBlk; ++r) {
+            uint32_t w;
+            asm volatile("ld.shared.b32 %0, [%1];"
+                         : "=r"(w)
+                         : "r"(base + r * 128 + ((chunk ^ (r & 7)) << 4)));
+            cs0 += __uint_as_float(w << 16);
+            cs1 += __uint_as_float(w & 0xffff0000u);
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty(slot));
-        stats_consumer_barrier();   // column sums complete
-        if (s == nt - 1) {
-          const int n_j = min(sub * kBlk, L - j * sub * kBlk);
-          const float inv_n = 1.f / (float)n_j;
-          const size_t so = ((size_t)bh * N + j) * D;
-          for (int e = ctid; e < 3 * D; e += 256) {
-            const int which = e / D, col = e % D;
-            if (which == 0) qbar[so + col] = colsum[e] * inv_n;
-            else if (which == 1) kbar[so + col] = colsum[e] * inv_n;
-            else vsum[so + col] = colsum[e];
-          }
-          // acc -= kbar_j^T vsum_j
-#pragma unroll
-          for (int mt = 0; mt < C::kMT; ++mt)
-#pragma unroll
-            for (int nt2 = 0; nt2 < C::kNT; ++nt2) {
-              const int a0 = warp_m0 + mt * 16 + g, c0 = warp_n0 + nt2 * 8 + 2 * tq;
-              const float ka = colsum[D + a0] * inv_n, kb = colsum[D + a0 + 8] * inv_n;
-              const float v0 = colsum[2 * D + c0], v1 = colsum[2 * D + c0 + 1];
-              acc[mt][nt2][0] -= ka * v0;
-              acc[mt][nt2][1] -= ka * v1;
-              acc[mt][nt2][2] -= kb * v0;
-              acc[mt][nt2][3] -= kb * v1;
-            }
-          stats_consumer_barrier();   // column sums free for the next block
+      }
+      // block end: statistics, then G_j - kbar_j^T vsum_j into the accumulator
+      const int n_j = min(sub * kBlk, L - j * sub * kBlk);
+      const float inv_n = 1.f / (float)n_j;
+      float *kv = reinterpret_cast<float *>(smem + T::kOffKV) + g * 2 * D;   // kbar, vsum
+      if (sums && !bad) {
+        const size_t so = ((size_t)bh * N + j) * D + 2 * lp;
+        if (tns == 0) {
+          *reinterpret_cast<float2 *>(qbar + so) = make_float2(cs0 * inv_n, cs1 * inv_n);
+        } else if (tns == 1) {
+          *reinterpret_cast<float2 *>(kbar + so) = make_float2(cs0 * inv_n, cs1 * inv_n);
+          kv[2 * lp] = cs0 * inv_n;
+          kv[2 * lp + 1] = cs1 * inv_n;
+        } else {
+          *reinterpret_cast<float2 *>(vsum + so) = make_float2(cs0, cs1);
+          kv[D + 2 * lp] = cs0;
+          kv[D + 2 * lp + 1] = cs1;
         }
       }
+      cs0 = cs1 = 0.f;
+      if (!__all_sync(0xffffffffu, mbar_wait(gfull(g), (blk >> 1) & 1))) bad = true;
+      // every consumer warp takes the same decision: the flag of this block's
+      // parity is written only before this barrier and read only after it
+      if (bad) {
+        cflag[blk & 1] = 1;
+        *abort_flag = 1;
+      }
+      stats_consumer_barrier();
+      if (cflag[blk & 1]) { ok = false; break; }
+      tc_fence_after();
+      const float ka = kv[arow];
+      const uint32_t taddr = tmem + ((uint32_t)(sp * 32) << 16) + D * g + ch * kH;
+#pragma unroll
+      for (int q = 0; q < kH / 32; ++q) {
+        uint32_t r[32];
+        tmem_ld_x32(taddr + 32 * q, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          hacc[32 * q + i] += __uint_as_float(r[i]) - ka * kv[D + ch * kH + 32 * q + i];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(gempty(g));
     }
     if (ok && g0 < g1) flush(cur_bh);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, T::kTmemCols);
   }
 }
 

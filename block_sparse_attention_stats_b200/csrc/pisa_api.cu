@@ -15,7 +15,6 @@
 #include "pisa_common.cuh"
 #include "k1_block_stats.cuh"
 #include "k2_select.cuh"
-#include "k2_select_tc.cuh"
 #include "k3_pack.cuh"
 #include "k3_attention_tc.cuh"
 #include "k5_tail_histogram.cuh"
@@ -96,26 +95,9 @@ static size_t stats_ws(int B, int H, int L, int d, int block_size) {
   const int parts = std::max(stats_num_chunks(BH, N), stats_max_segments(BH, N));
   return align_up((size_t)BH * parts * d * d * sizeof(float), 256);
 }
-// selection scratch: the float32 score matrix of the two-pass path, or for
-// the certified path (512 < N <= 2048) the approximate scores with rows padded
-// to 128 columns, the two bf16 terms of qbar and kbar (head dimension up to
-// 128) and the row norms
-struct SelectLayout {
-  size_t approx, q16, k16, qn, kn, total;
-};
-static SelectLayout select_layout(int B, int H, int N) {
-  const size_t BH = (size_t)B * H, Npad = (size_t)ceil_div(N, kCertTile) * kCertTile;
-  SelectLayout p;
-  size_t o = 0;
-  p.approx = o; o += align_up(BH * N * Npad * sizeof(float), 256);
-  p.q16 = o; o += align_up(2 * BH * Npad * 128 * 2, 256);   // high and low bf16 terms
-  p.k16 = o; o += align_up(2 * BH * Npad * 128 * 2, 256);
-  p.qn = o; o += align_up(BH * N * sizeof(float), 256);
-  p.kn = o; o += align_up(BH * N * sizeof(float), 256);
-  p.total = o;
-  return p;
+static size_t select_ws(int B, int H, int N) {
+  return align_up((size_t)B * H * N * N * sizeof(float), 256);
 }
-static size_t select_ws(int B, int H, int N) { return select_layout(B, H, N).total; }
 // scratch of the fused-attention step: bf16 kbar/vsum/hbar, query-block
 // pairing (selection bitmaps, overlaps, pairs), bf16 copies of f32 inputs
 struct SparseLayout {
@@ -186,23 +168,42 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
   const int N = ceil_div(L, 64 * sub);   // blocks of sub x 64 tokens
   const int nchunk = stats_num_chunks(BH, N);
   dim3 grid(nchunk, BH);
-  if (dt == PISA_BF16) {
-    // one CTA per SM streams a contiguous range of blocks through a TMA ring
-    const long long total = (long long)BH * N;
-    const int nc = stats_stream_ctas(total);
-    const int maxseg = stats_max_segments(BH, N);
-    CUtensorMap mq, mk, mv;
-    PISA_TRY(make_map(&mq, q, D, L, BH, kBlk));
-    PISA_TRY(make_map(&mk, k, D, L, BH, kBlk));
-    PISA_TRY(make_map(&mv, v, D, L, BH, kBlk));
-    PISA_CUDA(cudaFuncSetAttribute(stats_pass_tma_kernel<D>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   StatsTmaCfg<D>::kSmem));
-    stats_pass_tma_kernel<D><<<nc, StatsTmaCfg<D>::kThreads, StatsTmaCfg<D>::kSmem, st>>>(
-        mq, mk, mv, L, N, sub, BH, maxseg, qbar, kbar, vsum, partial);
+  bool streamed = false;
+  if constexpr (D == 128) {
+    if (dt == PISA_BF16) {
+      // one CTA per SM streams a contiguous range of blocks through a TMA ring
+      streamed = true;
+      const long long total = (long long)BH * N;
+      const int nc = stats_stream_ctas(total);
+      const int maxseg = stats_max_segments(BH, N);
+      CUtensorMap mq, mk, mv;
+      PISA_TRY(make_map(&mq, q, D, L, BH, kBlk));
+      PISA_TRY(make_map(&mk, k, D, L, BH, kBlk));
+      PISA_TRY(make_map(&mv, v, D, L, BH, kBlk));
+      PISA_CUDA(cudaFuncSetAttribute(stats_pass_tma_kernel<D>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     StatsTmaCfg<D>::kSmem));
+      stats_pass_tma_kernel<D><<<nc, StatsTmaCfg<D>::kThreads, StatsTmaCfg<D>::kSmem, st>>>(
+          mq, mk, mv, L, N, sub, BH, maxseg, qbar, kbar, vsum, partial);
+      PISA_TRY(check_launch());
+      hbar_reduce_seg_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(
+          partial, maxseg, D * D, N, BH, nc, hbar);
+      PISA_TRY(check_launch());
+    }
+  }
+  if (streamed) {
+    // done above
+  } else if (dt == PISA_BF16) {
+    // head dimension 64: chunked pass (cp.async double buffer, mma.sync)
+    const int smem = 2 * 3 * StatsMmaCfg<D>::kTileBytes + 3 * D * (int)sizeof(float);
+    PISA_CUDA(cudaFuncSetAttribute(stats_pass_bf16_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    stats_pass_bf16_kernel<D><<<grid, kStatsThreads, smem, st>>>(
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, L, N, sub,
+        nchunk, qbar, kbar, vsum, partial);
     PISA_TRY(check_launch());
-    hbar_reduce_seg_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(
-        partial, maxseg, D * D, N, BH, nc, hbar);
+    hbar_reduce_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(partial, nchunk, D * D,
+                                                                        N, hbar);
     PISA_TRY(check_launch());
   } else {
     const int smem = 3 * kBlk * D * (int)sizeof(float) + 3 * D * (int)sizeof(float);
@@ -236,45 +237,10 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
   return PISA_OK;
 }
 
-// certified selection (k2_select_tc.cuh): pack, approximate scores on the
-// tensor cores, exact float32 scores only where the bound cannot decide
-template <int D>
-static pisa_status launch_select_certified(const float *qbar, const float *kbar,
-                                           const float *cov, float cov_weight, float scale,
-                                           int BH, int N, int k_sel, int sink, int32_t *idx,
-                                           unsigned char *ws, cudaStream_t st) {
-  const SelectLayout lay = select_layout(1, BH, N);
-  const int Npad = ceil_div(N, kCertTile) * kCertTile;
-  float *approx = (float *)(ws + lay.approx);
-  __nv_bfloat16 *q16 = (__nv_bfloat16 *)(ws + lay.q16), *k16 = (__nv_bfloat16 *)(ws + lay.k16);
-  float *qn = (float *)(ws + lay.qn), *kn = (float *)(ws + lay.kn);
-  const size_t pack_threads = (size_t)2 * BH * Npad * 32;
-  select_pack_kernel<D><<<grid_1d(pack_threads, 256), 256, 0, st>>>(qbar, kbar, N, Npad, BH, q16,
-                                                                   k16, qn, kn);
-  PISA_TRY(check_launch());
-  CUtensorMap mq, mk;
-  PISA_TRY(make_map(&mq, q16, D, Npad, 2 * BH, kCertTile));
-  PISA_TRY(make_map(&mk, k16, D, Npad, 2 * BH, kCertTile));
-  PISA_CUDA(cudaFuncSetAttribute(select_approx_tc_kernel<D>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SelTcCfg<D>::kSmem));
-  select_approx_tc_kernel<D><<<dim3(Npad / kCertTile, BH), SelTcCfg<D>::kThreads,
-                               SelTcCfg<D>::kSmem, st>>>(mq, mk, cov, cov_weight, scale, N, Npad,
-                                                         BH, approx);
-  PISA_TRY(check_launch());
-  const size_t rows = (size_t)BH * N;
-  const unsigned blocks = (unsigned)((rows + kCertWarps - 1) / kCertWarps);
-  const int csmem = certified_smem(N, D);
-  PISA_CUDA(cudaFuncSetAttribute(select_certified_kernel<D>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, csmem));
-  select_certified_kernel<D><<<blocks, kCertWarps * 32, csmem, st>>>(
-      approx, Npad, qbar, kbar, qn, kn, cov, cov_weight, scale, N, k_sel, sink, rows, idx);
-  return check_launch();
-}
-
 static pisa_status launch_select(const float *qbar, const float *kbar, const float *cov,
                                  float cov_weight, float scale, int BH, int N, int d, int k_sel,
                                  int sink, int32_t *idx, unsigned char *ws, cudaStream_t st) {
-  float *scores = (float *)ws;
+  float *scores = (float *)ws;   // [BH, N, N] for the two-pass path
   const int fsmem = select_fused_smem(N, d);
   if (N <= kSelFusedMaxN && fsmem <= 227 * 1024) {
     // short sequences: the score rows of a query-block group stay in shared
@@ -285,15 +251,6 @@ static pisa_status launch_select(const float *qbar, const float *kbar, const flo
     select_fused_kernel<<<dim3(ceil_div(N, kSelRows), BH), kSelThreads, fsmem, st>>>(
         qbar, kbar, cov, cov_weight, scale, N, d, k_sel, sink, idx);
     return check_launch();
-  }
-  if (N <= kCertMaxN) {
-    // long rows: most scores are decided by the tensor-core approximation and
-    // its error bound; the float32 score is formed only near the threshold
-    if (d == 128)
-      return launch_select_certified<128>(qbar, kbar, cov, cov_weight, scale, BH, N, k_sel, sink,
-                                          idx, ws, st);
-    return launch_select_certified<64>(qbar, kbar, cov, cov_weight, scale, BH, N, k_sel, sink,
-                                       idx, ws, st);
   }
   dim3 g1(ceil_div(N, kScoreTile), ceil_div(N, kScoreTile), BH);
   scores_kernel<<<g1, 256, 0, st>>>(qbar, kbar, cov, cov_weight, scale, N, d, scores);

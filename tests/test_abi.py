@@ -48,15 +48,11 @@ def test_num_blocks_and_selected_match_oracle(lib):
     assert lib.pisa_num_blocks(0, 64) == -1
 
 
-def test_selection_workspace_covers_every_path(lib):
-    """The selection scratch holds the float32 score matrix of the two-pass
-    path and, for the certified path, the approximate scores with rows padded
-    to 128 columns, two bf16 terms of qbar and of kbar and two norm vectors."""
-    for BH, N in ((40, 1182), (24, 1861), (24, 72), (1, 2100), (3, 600)):
+def test_selection_workspace_holds_the_score_matrix(lib):
+    """The selection scratch holds the float32 score matrix of the two-pass path."""
+    for BH, N in ((40, 1182), (24, 1861), (24, 72), (1, 4205), (3, 600)):
         need = lib.pisa_select_workspace_bytes(1, BH, N)
-        npad = -(-N // 128) * 128
         assert need >= BH * N * N * 4
-        assert need >= BH * N * npad * 4 + 4 * BH * npad * 128 * 2 + 2 * BH * N * 4
         assert need % 256 == 0
 
 

@@ -120,7 +120,7 @@ def test_block_size_128(P, L, d, sink, mode, cov):
     (900, 64, 0, "hyd", 0.1),       # odd tile count, d = 64
     (129, 128, -1, "hyd", 0.0),     # N = 2
     (100, 64, None, "0th", 0.0),    # N = 1
-    (70000, 128, None, "hyd", 0.0), # 547 blocks: the separate step takes its certified path
+    (70000, 128, None, "hyd", 0.0), # 547 blocks: the separate step takes its two-pass path
 ])
 def test_block_size_128_selection_in_fused_kernel(P, L, d, sink, mode, cov):
     """With 128-token blocks the fused kernel can select inside (each CTA is

@@ -1,11 +1,10 @@
 """GPU parity of the selection step on long rows (more than 512 blocks).
 
-Rows of 512 < N <= 2048 blocks go through the certified path (approximate
-scores on the tensor cores, the float32 score only where the error bound
-cannot decide); longer rows through the two-pass path.  Both must give the
-exact top-k of the scores: the sets must equal the fp64 oracle's, except for
-certified rounding ties (reported, never hidden), and where the scores tie
-exactly the lower block index must win.
+Rows longer than 512 blocks go through the two-pass path: the float32 score
+matrix, then one warp per query block selecting from its row.  The sets must
+equal the fp64 oracle's, except for certified rounding ties (reported, never
+hidden; at most one row in a hundred), and where the scores tie exactly the
+lower block index must win.
 """
 import numpy as np
 import pytest
@@ -63,9 +62,9 @@ def _check(P, wl, Q, K, V, exact=False):
     (64 * 600, 0.125, None, 0.0),
     (64 * 600, 0.05, -1, 0.1),
     (64 * 1500 + 17, 0.3, 0, 0.0),      # ragged last block of 17 tokens
-    (64 * 2048, 0.1, -1, 0.1),          # the longest rows of the certified path
+    (64 * 2048, 0.1, -1, 0.1),          # 2048 blocks
 ])
-def test_certified_selection_clustered(P, L, density, sink, cov):
+def test_long_row_selection_clustered(P, L, density, sink, cov):
     wl = WORKLOADS["flux"].with_(H=2, L=L, density=density, sink_idx=sink, cov_weight=cov,
                                  cluster_kind="block")
     Q, K, V = generate_qkv(wl, "cpu")
@@ -73,15 +72,14 @@ def test_certified_selection_clustered(P, L, density, sink, cov):
     # within the float32 error bound) are valid and printed; any other
     # difference fails inside _check
     ties = _check(P, wl, Q, K, V)
-    assert ties <= 2, f"{ties} certified rounding ties"
+    assert ties <= wl.H * (L // 64) // 100, f"{ties} certified rounding ties"
 
 
 @pytest.mark.parametrize("cov", [0.0, 0.1])
-def test_certified_selection_zero_queries(P, cov):
+def test_long_row_selection_zero_queries(P, cov):
     """q = 0 makes every relevance term exactly 0: without the covariance term
     all scores tie and the lowest block indices must be chosen; with it the
-    order is that of M_j.  No score is decided by the bound, so every one goes
-    through the float32 path."""
+    order is that of M_j."""
     wl = WORKLOADS["flux"].with_(H=2, L=64 * 700, density=0.1, sink_idx=-1, cov_weight=cov,
                                  cluster_kind="block")
     Q, K, V = generate_qkv(wl, "cpu")
@@ -89,7 +87,7 @@ def test_certified_selection_zero_queries(P, cov):
     assert _check(P, wl, Q, K, V, exact=cov == 0.0) == 0
 
 
-def test_certified_selection_duplicate_blocks(P):
+def test_long_row_selection_duplicate_blocks(P):
     """The second half of the keys repeats the first, so pairs of blocks have
     bit-identical scores on both sides; ties go to the lower index."""
     wl = WORKLOADS["flux"].with_(H=1, L=64 * 800, density=0.15, sink_idx=None,
@@ -100,9 +98,9 @@ def test_certified_selection_duplicate_blocks(P):
     assert _check(P, wl, Q, K, V, exact=True) == 0
 
 
-def test_two_pass_selection_beyond_certified_rows(P):
-    """More than 2048 blocks: the two-pass path (float32 score matrix, radix top-k)."""
-    wl = WORKLOADS["flux"].with_(H=1, L=64 * 2100 + 5, density=0.1, sink_idx=-1,
+def test_selection_rows_of_4200_blocks(P):
+    """4201 blocks per row (the partial last one holds 5 tokens)."""
+    wl = WORKLOADS["flux"].with_(H=1, L=64 * 4200 + 5, density=0.05, sink_idx=-1,
                                  cov_weight=0.1, cluster_kind="block")
     Q, K, V = generate_qkv(wl, "cpu")
-    assert _check(P, wl, Q, K, V) <= 2
+    assert _check(P, wl, Q, K, V) <= 4201 // 100
