@@ -48,13 +48,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the fused attention kernel, from an ncu capture,
 # keyed by the sha1 of the kernel source it was taken on (see profiles/).
 K3_TRAFFIC = {
-    # H=4 ncu captures (dram read + write per launch) scaled by 10 to the 40 heads:
-    # Wan-like 300.7 MB, Wan-like with 128-token blocks 296.8 MB
-    "7974a8f98dec": {"wan": 3.007e9, "wan_b128": 2.968e9},
-    # after the optional float32 output: Wan-like 302.1 MB, 128-token blocks 297.6 MB
-    "bf19c92395d8": {"wan": 3.021e9, "wan_b128": 2.976e9},
-    # with the in-kernel selection option (unused by this workload): Wan-like 301.3 MB
-    "26564cebed3a": {"wan": 3.013e9},
+    # H=4 ncu capture (dram read 240.1 MB + write 60.8 MB per launch) scaled by
+    # 10 to the 40 heads; profiles/piecewise_attention_tc_wan_h4.md
+    "6d5287a9c780": {"wan": 3.009e9},
 }
 
 
@@ -67,9 +63,40 @@ def _peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def select_roofline(wl, N, k_sel, ms, peaks):
+    """Selection step against its floor.  Rows of up to 512 blocks: one fused
+    kernel, scores in shared memory (on chip).  Longer rows: the three-part
+    bf16 split of qbar and kbar, the score tiles on the tensor cores (six bf16
+    products per score), then the top-k from the float32 score matrix; the
+    floor adds the split's bytes, the score kernel's tensor time or its score
+    writes (whichever is longer) and the top-k's score reads, all at the
+    measured peaks."""
+    BH = wl.B * wl.H
+    flop = 2.0 * BH * N * N * wl.d
+    if N <= 512:
+        return {"bound": "on chip (fp32 score contraction in shared memory, top-k)",
+                "path": "fused scores + top-k", "score_gflop": flop / 1e9,
+                "score_tflops": flop / (ms * 1e-3) / 1e12}
+    hbm = peaks.get("hbm_gbs", 6650.0) * 1e9
+    tc = peaks.get("bf16_tflops", 1590.0) * 1e12
+    ld = -(-N // 32) * 32
+    split_bytes = BH * N * wl.d * (2 * 4 + 2 * 3 * 2)
+    score_bytes = BH * N * ld * 4
+    t_star = (split_bytes / hbm + max(6 * flop / tc, score_bytes / hbm)
+              + (score_bytes + BH * N * k_sel * 4) / hbm)
+    return {"bound": "tensor (score tiles) + hbm (score matrix)",
+            "path": "two-pass: three-part bf16 split, tcgen05 score tiles, "
+                    "one-histogram top-k from the float32 score matrix",
+            "score_gflop": flop / 1e9, "score_tensor_gflop_executed": 6 * flop / 1e9,
+            "score_matrix_bytes": score_bytes, "t_star_ms": t_star * 1e3,
+            "frac": t_star * 1e3 / ms}
+
+
 def _k3_source_hash():
+    # the files the fused kernel's own code comes from (the kernel, the
+    # in-kernel selection's top-k, the tcgen05 / TMA primitives)
     h = hashlib.sha1()
-    for n in ("k3_attention_tc.cuh", "k3_pack.cuh", "sm100_primitives.cuh"):
+    for n in ("k3_attention_tc.cuh", "k2_select.cuh", "sm100_primitives.cuh"):
         fn = os.path.join(ROOT, "block_sparse_attention_stats_b200", "csrc", n)
         if os.path.exists(fn):
             h.update(open(fn, "rb").read())
@@ -752,10 +779,10 @@ def run_pisa(args, wl):
     achieved = f_alg / (t_k3 * 1e-3) / 1e12
     src = _k3_source_hash()
     traffic = K3_TRAFFIC.get(src, {}).get(wl.name)
-    # statistics: pass 1 + hbar reduction (+ covariance pass); selection: scores +
-    # top-k; fused step: statistics packing (+ bitmap, overlaps, pairing with
+    # statistics: pass 1 + hbar reduction (+ covariance pass); selection: one
+    # fused kernel, or split + score tiles + top-k; fused step: statistics packing (+ bitmap, overlaps, pairing with
     # 64-token blocks) (+ three f32 -> bf16 copies) + the fused kernel
-    n_sel = 1 if N <= 512 else 2
+    n_sel = 1 if N <= 512 else 3
     launches_per_step = (2 + (1 if want_cov else 0) + n_sel
                          + (5 if wl.block_size == 64 else 2) + (3 if wl.dtype == "f32" else 0))
     line = {
@@ -771,19 +798,13 @@ def run_pisa(args, wl):
         "ms_per_step_median": statistics.median(step_ms),
         "kernels_roofline": {
             # statistics: HBM-bound (reads Q, K, V once, K and V again with the
-            # covariance pass); selection: on chip (the N x N fp32 score
-            # contraction and the radix top-k)
+            # covariance pass); selection: see select_roofline
             "block_stats": {"bound": "hbm", "bytes": stats_bytes(wl),
                             "achieved_gbs": stats_bytes(wl) / (part_ms["block_stats"] * 1e-3) / 1e9,
                             "peak_gbs": peaks.get("hbm_gbs", 6650.0),
                             "frac": stats_bytes(wl) / (part_ms["block_stats"] * 1e-3) / 1e9
                             / peaks.get("hbm_gbs", 6650.0)},
-            "select": {"bound": "on-chip (fp32 score contraction, top-k)",
-                       "path": ("fused scores + top-k" if N <= 512 else
-                                "two-pass: float32 score matrix + radix top-k"),
-                       "score_gflop": 2.0 * wl.B * wl.H * N * N * wl.d / 1e9,
-                       "score_tflops": 2.0 * wl.B * wl.H * N * N * wl.d
-                       / (part_ms["select"] * 1e-3) / 1e12},
+            "select": select_roofline(wl, N, k_sel, part_ms["select"], peaks),
         },
         "roofline": {
             "kernel": "piecewise_attention (fused exact + centroid tail + first-order)",

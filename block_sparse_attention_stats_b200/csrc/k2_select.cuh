@@ -9,109 +9,23 @@
 //   score_ij = scale * (qbar_i . kbar_j) + lambda * M_j      (float32)
 //
 // Fused path (select_fused_kernel, short sequences, N <= 512): a group of query
-// blocks computes its score rows into shared memory and selects from there
-// (FLUX shape: 0.028 ms against 0.032 ms; at N = 1182 it is 1.9x slower than the
-// two-pass path, which streams each k-bar tile once per 128 x 128 score tile).
+// blocks computes its score rows into shared memory (float32 FMAs, the head
+// dimension summed in ascending order) and selects from there (FLUX shape:
+// 0.028 ms against 0.032 ms two-pass).
 // Two-pass path otherwise:
-// Pass 1 (scores_kernel): a float32 FMA GEMM per head, 128 x 128 output tiles,
-// each score summed over the head dimension in ascending order.
-// Pass 2 (topk_kernel): one warp per query block.  Scores become 32-bit keys
-// whose unsigned order is the float order; an MSB-first radix select (4 x 8
-// bits) finds the k-th largest key T; every key > T is kept, and of the keys
-// equal to T the lowest block indices are kept (ties go to the lower index).
-// The sink block is set aside first and always kept.  Indices come out
-// ascending via warp ballots.
+// Pass 1 (k2_scores_tc.cuh): the score matrix on the tensor cores from
+// three-part bf16 splits of qbar and kbar, to float32 accuracy.
+// Pass 2 (topk_bins_kernel; topk_kernel for rows too long to stage in shared
+// memory): one warp per query block.  Scores map to 32-bit keys whose
+// unsigned order is the float order; the k-th largest key T is found, every
+// key > T is kept, and of the keys equal to T the lowest block indices are
+// kept (ties go to the lower index).  The sink block is set aside first and
+// always kept.  Indices come out ascending via warp ballots.
 #pragma once
 
 #include "pisa_common.cuh"
 
 namespace pisa {
-
-// Scores: C = scale * Qbar Kbar^T + lambda * cov over 128 x 128 tiles, 256
-// threads with 8 x 8 outputs each; operands staged in shared memory as
-// [dim][row] so every thread reads its 8 rows / 8 columns as two float4.
-// Each score is accumulated over the head dimension in ascending order.
-constexpr int kScoreTile = 128;
-constexpr int kScoreK = 16;
-constexpr int kScorePad = 4;
-
-__global__ void __launch_bounds__(256, 2)
-    scores_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar,
-                  const float *__restrict__ cov, float cov_weight, float scale, int N, int D,
-                  float *__restrict__ scores) {
-  __shared__ __align__(16) float As[kScoreK][kScoreTile + kScorePad];
-  __shared__ __align__(16) float Bs[kScoreK][kScoreTile + kScorePad];
-  const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
-  const float *qb = qbar + (size_t)bh * N * D;
-  const float *kb = kbar + (size_t)bh * N * D;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  float acc[8][8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
-
-  // 128 rows x 16 dims of each operand per chunk, two float4 per thread per
-  // operand; the next chunk is fetched into registers while this one is used
-  float4 pa[2], pb[2];
-  auto fetch = [&](int e0) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int t = tid + 256 * h;
-      const int row = t >> 2, e4 = (t & 3) * 4;
-      const int gi = i0 + row, gj = j0 + row;
-      pa[h] = gi < N ? *reinterpret_cast<const float4 *>(qb + (size_t)gi * D + e0 + e4)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-      pb[h] = gj < N ? *reinterpret_cast<const float4 *>(kb + (size_t)gj * D + e0 + e4)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  fetch(0);
-  for (int e0 = 0; e0 < D; e0 += kScoreK) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int t = tid + 256 * h;
-      const int row = t >> 2, e4 = (t & 3) * 4;
-      const float4 a = pa[h], b = pb[h];
-      As[e4 + 0][row] = a.x; As[e4 + 1][row] = a.y; As[e4 + 2][row] = a.z; As[e4 + 3][row] = a.w;
-      Bs[e4 + 0][row] = b.x; Bs[e4 + 1][row] = b.y; Bs[e4 + 2][row] = b.z; Bs[e4 + 3][row] = b.w;
-    }
-    __syncthreads();
-    if (e0 + kScoreK < D) fetch(e0 + kScoreK);
-#pragma unroll
-    for (int e = 0; e < kScoreK; ++e) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(&As[e][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&As[e][ty * 8 + 4]);
-      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[e][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[e][tx * 8 + 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-    __syncthreads();
-  }
-  float cw[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const int gj = j0 + tx * 8 + c;
-    cw[c] = (cov_weight != 0.f && gj < N) ? cov_weight * cov[(size_t)bh * N + gj] : 0.f;
-  }
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int gi = i0 + ty * 8 + r;
-    if (gi >= N) continue;
-    float *out = scores + ((size_t)bh * N + gi) * N;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int gj = j0 + tx * 8 + c;
-      if (gj < N) out[gj] = fmaf(scale, acc[r][c], cw[c]);
-    }
-  }
-}
 
 // Order-preserving map float32 -> uint32 (-0 is treated as +0).
 __device__ __forceinline__ uint32_t float_key(float f) {
@@ -227,22 +141,215 @@ __device__ __forceinline__ void topk_row(const float *sc, int N, int k_sel, int 
   if (lane == 0 && out_base != k_sel) report_device_error(kDevErrRange);
 }
 
-// One warp per query block over the N x N score matrix in global memory.
+// One warp per query block over the score matrix in global memory (row
+// stride ld >= N).
 __global__ void __launch_bounds__(kTopkThreads)
-    topk_kernel(const float *__restrict__ scores, int N, int k_sel, int sink, size_t rows,
-                int32_t *__restrict__ idx) {
+    topk_kernel(const float *__restrict__ scores, int N, int ld, int k_sel, int sink,
+                size_t rows, int32_t *__restrict__ idx) {
   __shared__ unsigned hist_all[kTopkThreads / 32][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t row = (size_t)blockIdx.x * (kTopkThreads / 32) + warp;
   if (row >= rows) return;
-  topk_row(scores + row * N, N, k_sel, sink, hist_all[warp], idx + row * k_sel, lane);
+  topk_row(scores + row * ld, N, k_sel, sink, hist_all[warp], idx + row * k_sel, lane);
+}
+
+// ---------------------------------------------------------------------------
+// The same selection with one histogram pass instead of four radix passes.
+// Each warp copies its row into shared memory, then finds the k-th largest key
+// T and the number of keys equal to T to keep:
+//  1. lo / hi = the smallest / largest candidate score; bin(x) =
+//     min(255, int((x - lo) * (256 / (hi - lo)))).  Every step of bin() is a
+//     monotone float32 operation, so x >= y implies bin(x) >= bin(y): the bins
+//     order the keys.
+//  2. One histogram of the candidates' bins; scanning from the top bin gives
+//     the bin b* that holds the `need`-th largest key and how many keys of b*
+//     are still to be taken.
+//  3. The (at most kBinCand) scores of b* are gathered and T is the one whose
+//     count of larger scores is below, and whose count of larger or equal
+//     scores reaches, the number still to be taken.
+// Comparing floats gives the key order (only -0 and +0 share a key, and they
+// compare equal).  Then the same compaction as topk_row keeps the sink, every
+// score > T and the lowest-index scores equal to T.  Rows where the bins do
+// not apply (all scores equal, a non-finite score, more than kBinCand scores
+// in b*) go through topk_row on the staged row, so the result is the same set
+// in every case.
+// ---------------------------------------------------------------------------
+constexpr int kBinCand = 64;
+
+// shared memory per warp: the row (ld floats), the histogram, the gathered bin
+__host__ __device__ inline int topk_bins_smem(int ld) {
+  return (kTopkThreads / 32) * (ld + 256 + kBinCand) * 4;
+}
+
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_bins_kernel(const float *__restrict__ scores, int N, int ld, int k_sel, int sink,
+                     size_t rows, int32_t *__restrict__ idx) {
+  extern __shared__ __align__(16) float tk_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * (kTopkThreads / 32) + warp;
+  if (row >= rows) return;
+  float *srow = tk_smem + (size_t)warp * (ld + 256 + kBinCand);
+  unsigned *hist = reinterpret_cast<unsigned *>(srow + ld);
+  float *cand = reinterpret_cast<float *>(hist + 256);
+  const float *sc = scores + row * ld;
+  int32_t *out = idx + row * k_sel;
+  const int need = k_sel - (sink >= 0 ? 1 : 0);
+  const int candidates = N - (sink >= 0 ? 1 : 0);
+  // stage the row (16-byte loads), and 1. the range of the candidates on the
+  // way; a NaN or infinite score sends the row to topk_row
+  const float inf = __int_as_float(0x7f800000);
+  float lo = inf, hi = -inf;
+  bool bad = false;
+#pragma unroll 2
+  for (int c = lane; c < ld / 4; c += 32) {
+    const float4 x4 = __ldcs(reinterpret_cast<const float4 *>(sc) + c);
+    *reinterpret_cast<float4 *>(srow + 4 * c) = x4;
+    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * c + e;
+      if (j < N && j != sink) {
+        bad |= !(fabsf(xs[e]) < inf);
+        lo = fminf(lo, xs[e]);
+        hi = fmaxf(hi, xs[e]);
+      }
+    }
+  }
+  __syncwarp();
+  if (need <= 0 || need >= candidates) {
+    topk_row(srow, N, k_sel, sink, hist, out, lane);
+    return;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const float span = hi - lo, w = 256.f / span;
+  if (__any_sync(0xffffffffu, bad) || !(span > 0.f && span < inf && w < inf)) {
+    topk_row(srow, N, k_sel, sink, hist, out, lane);
+    return;
+  }
+  auto bin_of = [&](float x) { return min((int)((x - lo) * w), 255); };
+  // 2. histogram and the boundary bin
+#pragma unroll
+  for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0u;
+  __syncwarp();
+#pragma unroll 2
+  for (int c = lane; c < ld / 4; c += 32) {
+    const float4 x4 = *reinterpret_cast<const float4 *>(srow + 4 * c);
+    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * c + e;
+      if (j < N && j != sink) atomicAdd(&hist[bin_of(xs[e])], 1u);
+    }
+  }
+  __syncwarp();
+  unsigned own = 0;                      // lane l owns bins 255-8l .. 248-8l
+#pragma unroll
+  for (int q = 0; q < 8; ++q) own += hist[255 - 8 * lane - q];
+  unsigned incl = own;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  const unsigned excl = incl - own;
+  const unsigned who = __ballot_sync(0xffffffffu, excl < (unsigned)need && (unsigned)need <= incl);
+  const int src = __ffs(who) - 1;
+  int bstar = 0, take = 0, cnt = 0;
+  if (lane == src) {
+    unsigned cum = excl;
+    for (int q = 0; q < 8; ++q) {
+      const int b = 255 - 8 * lane - q;
+      const unsigned c = hist[b];
+      if ((unsigned)need <= cum + c) {
+        bstar = b;
+        take = need - (int)cum;
+        cnt = (int)c;
+        break;
+      }
+      cum += c;
+    }
+  }
+  bstar = __shfl_sync(0xffffffffu, bstar, src);
+  take = __shfl_sync(0xffffffffu, take, src);
+  cnt = __shfl_sync(0xffffffffu, cnt, src);
+  if (cnt > kBinCand) {
+    topk_row(srow, N, k_sel, sink, hist, out, lane);
+    return;
+  }
+  // 3. the scores of b*, and T among them: the `take`-th largest; eq = how
+  //    many candidates equal T, rem = how many of those are kept
+  int base = 0;
+  for (int j0 = 0; j0 < N; j0 += 32) {
+    const int j = j0 + lane;
+    const float x = j < N ? srow[j] : 0.f;
+    const bool in = j < N && j != sink && bin_of(x) == bstar;
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (in) cand[base + __popc(bal & ((1u << lane) - 1u))] = x;
+    base += __popc(bal);
+  }
+  __syncwarp();
+  float T = 0.f;
+  int rem = 0, eq = 0;
+  bool found = false;
+  for (int m = lane; m < cnt; m += 32) {
+    const float xm = cand[m];
+    int gt = 0, ge = 0;
+    for (int n = 0; n < cnt; ++n) {
+      const float xn = cand[n];
+      gt += xn > xm;
+      ge += xn >= xm;
+    }
+    if (gt < take && take <= ge) {
+      found = true;
+      T = xm;
+      rem = take - gt;
+      eq = ge - gt;
+    }
+  }
+  const unsigned fb = __ballot_sync(0xffffffffu, found);
+  if (fb == 0u) {                        // cannot happen; keep the result exact anyway
+    topk_row(srow, N, k_sel, sink, hist, out, lane);
+    return;
+  }
+  const int fl = __ffs(fb) - 1;
+  T = __shfl_sync(0xffffffffu, T, fl);
+  rem = __shfl_sync(0xffffffffu, rem, fl);
+  eq = __shfl_sync(0xffffffffu, eq, fl);
+  // keep: the sink, every score > T, and the lowest-index `rem` scores equal
+  // to T (all of them when rem == eq, the usual case)
+  const bool ties = rem != eq;
+  int out_base = 0, eq_base = 0;
+  for (int j0 = 0; j0 < N; j0 += 32) {
+    const int j = j0 + lane;
+    const bool valid = j < N;
+    const float x = valid ? srow[j] : 0.f;
+    const bool cnd = valid && j != sink;
+    bool sel;
+    if (ties) {
+      const bool is_eq = cnd && x == T;
+      const unsigned eq_bal = __ballot_sync(0xffffffffu, is_eq);
+      sel = (cnd && x > T) || (is_eq && eq_base + __popc(eq_bal & ((1u << lane) - 1u)) < rem);
+      eq_base += __popc(eq_bal);
+    } else {
+      sel = cnd && x >= T;
+    }
+    sel = sel || (valid && j == sink);
+    const unsigned bal = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[out_base + __popc(bal & ((1u << lane) - 1u))] = j;
+    out_base += __popc(bal);
+  }
+  if (lane == 0 && out_base != k_sel) report_device_error(kDevErrRange);
 }
 
 // ---------------------------------------------------------------------------
 // Fused scores + top-k for a group of kSelRows query blocks: the group's score
-// rows live in shared memory only (no N x N matrix in HBM).  Each score is the
-// same fp32 computation as in scores_kernel (head dimension summed in ascending
-// order, then scale * acc + lambda * M_j), so both paths select the same sets.
+// rows live in shared memory only (no N x N matrix in HBM).  Each score is a
+// float32 FMA chain over the head dimension in ascending order, then
+// scale * acc + lambda * M_j.
 // 384 threads compute 4 x 4 score blocks from k-bar chunks of 256 blocks x 32
 // dimensions staged transposed in shared memory; then 12 warps take two rows
 // each through the radix select.

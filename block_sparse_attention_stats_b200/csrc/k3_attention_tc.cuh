@@ -51,8 +51,12 @@ namespace pisa {
 
 // Selection inside the fused kernel (128-token blocks only, where a CTA is one
 // query block and needs no partner): the CTA scores its own pooled query
-// against every block centroid, in the same float32 order as scores_kernel,
-// and takes the top k_sel with the sink forced in, exactly as pisa_select.
+// against every block centroid (a float32 FMA chain over the head dimension,
+// as select_fused_kernel does) and takes the top k_sel with the sink forced
+// in, by the same rule as pisa_select.  Up to 512 blocks the sets are the
+// separate step's bit for bit; on longer rows the separate step's scores come
+// from the tensor cores and may order two blocks whose scores agree to float32
+// rounding the other way.
 struct FusedSelect {
   const float *qbar;   // [BH, Nc, D] (NULL: the selection comes from idx)
   const float *kbar;   // [BH, Nc, D]

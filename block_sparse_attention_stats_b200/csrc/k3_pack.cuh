@@ -73,34 +73,61 @@ __global__ void selection_bitmap_kernel(const int32_t *__restrict__ idx, int N, 
 }
 
 // ov[bh][i][d-1] = |S_i n S_{i+d}| for d = 1 .. kPairWindow (0 past the end).
-__global__ void pair_overlap_kernel(const uint32_t *__restrict__ bm, int N, int nwords,
-                                    uint16_t *__restrict__ ov) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * (blockDim.x >> 5) + warp;
-  const int bh = blockIdx.y;
-  if (i >= N) return;
-  const uint32_t *a = bm + ((size_t)bh * N + i) * nwords;
-  for (int dd = lane; dd < kPairWindow; dd += 32) {
-    const int j = i + 1 + dd;
-    int cnt = 0;
-    if (j < N) {
-      const uint32_t *b = bm + ((size_t)bh * N + j) * nwords;
-      for (int w = 0; w < nwords; ++w) cnt += __popc(a[w] & b[w]);
+// One CTA per 8 consecutive blocks i (a warp each, lane l takes d = l + 1 and
+// l + 33).  The 72 bitmap rows they touch are staged in shared memory 32
+// words at a time with coalesced loads; the row stride of 33 words keeps the
+// lanes' reads of 32 different rows on 32 different banks.
+static_assert(kPairWindow == 64, "two window positions per lane");
+constexpr int kOvRows = 8 + kPairWindow;
+
+__global__ void __launch_bounds__(256)
+    pair_overlap_kernel(const uint32_t *__restrict__ bm, int N, int nwords,
+                        uint16_t *__restrict__ ov) {
+  __shared__ uint32_t rows[kOvRows][33];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i0 = blockIdx.x * 8, bh = blockIdx.y;
+  const int i = i0 + warp;
+  int c0 = 0, c1 = 0;
+  for (int w0 = 0; w0 < nwords; w0 += 32) {
+    __syncthreads();
+    for (int t = tid; t < kOvRows * 32; t += 256) {
+      const int r = t >> 5, w = t & 31, row = i0 + r;
+      rows[r][w] = (row < N && w0 + w < nwords) ? bm[((size_t)bh * N + row) * nwords + w0 + w] : 0u;
     }
-    ov[((size_t)bh * N + i) * kPairWindow + dd] = (uint16_t)cnt;
+    __syncthreads();
+    const int nw = min(32, nwords - w0);
+    for (int w = 0; w < nw; ++w) {
+      const uint32_t a = rows[warp][w];
+      c0 += __popc(a & rows[warp + 1 + lane][w]);
+      c1 += __popc(a & rows[warp + 33 + lane][w]);
+    }
+  }
+  if (i < N) {
+    uint16_t *o = ov + ((size_t)bh * N + i) * kPairWindow;
+    o[lane] = (uint16_t)(i + 1 + lane < N ? c0 : 0);
+    o[lane + 32] = (uint16_t)(i + 33 + lane < N ? c1 : 0);
   }
 }
 
-// One warp per head; pairs[bh][p] = (i0, i1), i1 = -1 for an unpaired block.
+// One CTA per head; pairs[bh][p] = (i0, i1), i1 = -1 for an unpaired block.
 // Writes exactly ceil(N / 2) entries.  The head's overlap table is staged in
 // shared memory first (N * kPairWindow * 2 bytes), then the greedy pass runs
-// from shared memory only.
-// With staged == 0 (tables too large for shared memory) the table is read
-// from global memory instead.
-__global__ void pairing_kernel(const uint16_t *__restrict__ ov, int N, int staged,
-                               int2 *__restrict__ pairs) {
+// from shared memory only; with staged == 0 (tables too large for shared
+// memory) the table is read from global memory instead.
+// Greedy in block order: an unpaired block i takes the unpaired block in
+// i + 1 .. i + kPairWindow with the largest overlap (the nearer one on equal
+// overlap), else the first unpaired block past the window.  Which blocks of
+// the window are paired already is a 64-bit mask in registers (bit d: block
+// i + 1 + d), shifted by one per step; only partners found past the window
+// go through shared memory (`used`), entering the mask when the window
+// reaches them.  Each step is one warp max-reduction (redux.sync).
+constexpr int kPairThreads = 256;   // all stage the table; warp 0 pairs
+
+__global__ void __launch_bounds__(kPairThreads)
+    pairing_kernel(const uint16_t *__restrict__ ov, int N, int staged,
+                   int2 *__restrict__ pairs) {
   extern __shared__ __align__(16) unsigned char pair_smem[];
-  const int bh = blockIdx.x, lane = threadIdx.x;
+  const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   const uint16_t *head = ov + (size_t)bh * N * kPairWindow;
   const uint16_t *o = head;
   unsigned char *used = pair_smem;
@@ -108,41 +135,52 @@ __global__ void pairing_kernel(const uint16_t *__restrict__ ov, int N, int stage
     uint16_t *t = reinterpret_cast<uint16_t *>(pair_smem);
     const uint4 *src = reinterpret_cast<const uint4 *>(head);
     uint4 *dst = reinterpret_cast<uint4 *>(t);
-    for (int i = lane; i < N * kPairWindow / 8; i += 32) dst[i] = src[i];
+#pragma unroll 4
+    for (int i = tid; i < N * kPairWindow / 8; i += kPairThreads) dst[i] = src[i];
     o = t;
     used = pair_smem + (size_t)N * kPairWindow * 2;
   }
-  for (int i = lane; i < N; i += 32) used[i] = 0;
-  __syncwarp();
+  for (int i = tid; i < N; i += kPairThreads) used[i] = 0;
+  __syncthreads();
+  if (tid >= 32) return;
   int2 *out = pairs + (size_t)bh * ((N + 1) / 2);
   int np = 0;
+  uint64_t ahead = 0ull;       // bit d: block i + 1 + d is paired already
+  bool self = false;           // block i is paired already
+  // the overlaps of the current block's window positions lane and lane + 32
+  unsigned o0 = o[lane], o1 = o[32 + lane];
   for (int i = 0; i < N; ++i) {
-    if (used[i]) continue;  // uniform: every lane reads the same byte
-    // key: overlap high, then nearer partner first; lane l looks at distances
-    // l + 1 and l + 33
-    int best = -1;
-    for (int dd = lane; dd < kPairWindow; dd += 32) {
-      const int j = i + 1 + dd;
-      if (j < N && !used[j])
-        best = max(best, ((int)o[(size_t)i * kPairWindow + dd] << 8) | (255 - dd));
+    const unsigned n0 = i + 1 < N ? o[(size_t)(i + 1) * kPairWindow + lane] : 0u;
+    const unsigned n1 = i + 1 < N ? o[(size_t)(i + 1) * kPairWindow + 32 + lane] : 0u;
+    if (!self) {
+      // key + 1: overlap high, then nearer partner first; 0 = no candidate
+      const int j0 = i + 1 + lane, j1 = i + 33 + lane;
+      unsigned key = 0u;
+      if (j0 < N && !((ahead >> lane) & 1ull)) key = ((o0 << 8) | (255u - lane)) + 1u;
+      if (j1 < N && !((ahead >> (32 + lane)) & 1ull))
+        key = max(key, ((o1 << 8) | (255u - 32u - lane)) + 1u);
+      const unsigned best = __reduce_max_sync(0xffffffffu, key);
+      int partner = -1;
+      if (best > 0u) {
+        const int dd = 255 - (int)((best - 1u) & 255u);
+        partner = i + 1 + dd;
+        ahead |= 1ull << dd;
+      } else {
+        for (int jj = i + 1 + kPairWindow; jj < N; ++jj)
+          if (!used[jj]) { partner = jj; break; }
+        __syncwarp();
+        if (lane == 0 && partner >= 0) used[partner] = 1;
+      }
+      if (lane == 0) out[np] = make_int2(i, partner);
+      ++np;
     }
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, s));
-    int partner = -1;
-    if (best >= 0) {
-      partner = i + 1 + (255 - (best & 255));
-    } else {
-      for (int jj = i + 1 + kPairWindow; jj < N; ++jj)
-        if (!used[jj]) { partner = jj; break; }
-    }
+    // slide the window by one block
     __syncwarp();
-    if (lane == 0) {
-      used[i] = 1;
-      if (partner >= 0) used[partner] = 1;
-      out[np] = make_int2(i, partner);
-    }
-    __syncwarp();
-    ++np;
+    self = ahead & 1ull;
+    ahead >>= 1;
+    if (i + 1 + kPairWindow < N && used[i + 1 + kPairWindow]) ahead |= 1ull << (kPairWindow - 1);
+    o0 = n0;
+    o1 = n1;
   }
 }
 

@@ -467,6 +467,26 @@ __global__ void __launch_bounds__(352, 1)
         tmem_ld_x32(dp_addr, r[2]);
         tmem_ld_x32(dp_addr + 32, r[3]);
         tmem_wait_ld();
+        if (second && !centroid && __all_sync(0xffffffffu, keep == ~0ull)) {
+          // an exact tile every row of the warp keeps whole: weight 1, no mask
+          // (the same arithmetic as below with on = true, w = 1)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(r[h][i]), sl2, -lse2));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(r[h][i + 1]), sl2, -lse2));
+              pk[i / 2] = pack_bf16x2(p0 * (__uint_as_float(r[2 + h][i]) - dfull),
+                                      p1 * (__uint_as_float(r[2 + h][i + 1]) - dfull));
+            }
+            tmem_st_x16(ds_addr + 16 * h, pk);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(C::kBarPFull + g));
+          continue;
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[16];

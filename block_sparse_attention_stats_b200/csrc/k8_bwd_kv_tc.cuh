@@ -37,28 +37,32 @@ namespace pisa {
 // ---------------------------------------------------------------------------
 // query-block lists of key-block pairs (CSR per head)
 // ---------------------------------------------------------------------------
-// entry = (t << 2) | (flag: key tile 2p selected) | (flag: key tile 2p+1) << 1,
+// entry = (t << 2) | (flag: key tile j0 selected) | (flag: key tile j1) << 1,
 // ascending query tile t (64 tokens).  bm: the selection bitmap at block level
 // [BH, Nc, cwords].  With 64-token blocks (bsub = 1) query and key tiles are
-// blocks: pair p holds blocks 2p, 2p+1, each flagged on its own.  With 128-token
-// blocks (bsub = 2) pair p is block p and a selecting query block i contributes
-// its two query tiles 2i, 2i+1, with both key halves flagged.
+// blocks and pair p is (j0, j1) = kpairs[bh][p] (j1 = -1: a single block), each
+// flagged on its own.  With 128-token blocks (bsub = 2) pair p is block p and a
+// selecting query block i contributes its two query tiles 2i, 2i+1, with both
+// key halves flagged.
 // fill == 0: counts[bh * P + p] = list length; fill == 1: write the entries at
 // entries + bh * cap + offsets[bh * P + p].  One warp per (p, bh).
 __global__ void kvlist_kernel(const uint32_t *__restrict__ bm, int N, int Nc, int cwords,
-                              int bsub, int P, int fill, int *__restrict__ counts,
-                              const long long *__restrict__ offsets, long long cap,
-                              int *__restrict__ entries) {
+                              int bsub, int P, const int2 *__restrict__ kpairs, int fill,
+                              int *__restrict__ counts, const long long *__restrict__ offsets,
+                              long long cap, int *__restrict__ entries) {
   const int p = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
-  const int jb = bsub == 1 ? 2 * p : p;                 // first block of the pair
-  const int w = jb >> 5, sh = jb & 31;
-  const uint32_t fmask = (2 * p + 1 < N) ? 3u : 1u;     // key tiles that exist
-  const uint32_t bmask = bsub == 1 ? fmask : 1u;
+  const int2 pr = bsub == 1 ? kpairs[(size_t)bh * P + p] : make_int2(p, -1);
+  const uint32_t fmask = (2 * p + 1 < N) ? 3u : 1u;     // key tiles of a 128-token block
   int total = 0;
   int *out = fill ? entries + bh * cap + offsets[(size_t)bh * P + p] : nullptr;
   for (int i0 = 0; i0 < Nc; i0 += 32) {
     const int i = i0 + lane;
-    const uint32_t bits = i < Nc ? (bm[((size_t)bh * Nc + i) * cwords + w] >> sh) & bmask : 0u;
+    uint32_t bits = 0u;
+    if (i < Nc) {
+      const uint32_t *row = bm + ((size_t)bh * Nc + i) * cwords;
+      bits = (row[pr.x >> 5] >> (pr.x & 31)) & 1u;
+      if (pr.y >= 0) bits |= ((row[pr.y >> 5] >> (pr.y & 31)) & 1u) << 1;
+    }
     // query tiles this lane contributes, in order
     int n = 0;
     if (bits) n = bsub == 1 ? 1 : (2 * i + 1 < N ? 2 : 1);
@@ -80,6 +84,21 @@ __global__ void kvlist_kernel(const uint32_t *__restrict__ bm, int N, int Nc, in
     total += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (!fill && lane == 0) counts[(size_t)bh * P + p] = total;
+}
+
+// bmT[bh][j][w]: bit l of word w set iff key block j is in S_(32w + l), the
+// transpose of bm (one warp per 32 x 32 bit square).
+__global__ void bitmap_transpose_kernel(const uint32_t *__restrict__ bm, int N, int nwords,
+                                        uint32_t *__restrict__ bmT) {
+  const int wi = blockIdx.x, wj = blockIdx.y, bh = blockIdx.z, lane = threadIdx.x;
+  const int i = 32 * wi + lane;
+  const uint32_t word = i < N ? bm[((size_t)bh * N + i) * nwords + wj] : 0u;
+#pragma unroll 4
+  for (int b = 0; b < 32; ++b) {
+    const uint32_t col = __ballot_sync(0xffffffffu, (word >> b) & 1u);
+    const int j = 32 * wj + b;
+    if (lane == b && j < N) bmT[((size_t)bh * N + j) * nwords + wi] = col;
+  }
 }
 
 // offsets[bh * P + p] = exclusive prefix sum of counts over p (one CTA per head)
@@ -110,7 +129,8 @@ __global__ void kvlist_scan_kernel(const int *__restrict__ counts, int P,
   }
 }
 
-// lse_pad[bh, t] = lse[bh, t] for t < L, +inf up to the padded length
+// lse_pad[bh, t] = lse[bh, t] * log2(e) for t < L, +inf up to the padded length
+// (the kernels exponentiate with ex2)
 __global__ void pad_lse_kernel(const float *__restrict__ lse, int L, int Lpad, int BH,
                                float *__restrict__ lse_pad) {
   const size_t n = (size_t)BH * Lpad;
@@ -118,7 +138,7 @@ __global__ void pad_lse_kernel(const float *__restrict__ lse, int L, int Lpad, i
        e += (size_t)gridDim.x * blockDim.x) {
     const size_t bh = e / Lpad;
     const int t = (int)(e % Lpad);
-    lse_pad[e] = t < L ? lse[bh * L + t] : INFINITY;
+    lse_pad[e] = t < L ? lse[bh * L + t] * kLog2e : INFINITY;
   }
 }
 
@@ -173,6 +193,7 @@ __global__ void __launch_bounds__(320, 1)
                      const __grid_constant__ CUtensorMap tm_delta,
                      const int *__restrict__ counts, const long long *__restrict__ offsets,
                      long long cap, const int *__restrict__ entries,
+                     const int2 *__restrict__ kpairs,
                      const uint32_t *__restrict__ bm, int cwords, int bsub, int Nc, int L,
                      int N, float scale,
                      float *__restrict__ dkbar, float *__restrict__ dvbar, int Npad,
@@ -191,7 +212,11 @@ __global__ void __launch_bounds__(320, 1)
   const int P = (N + 1) / 2;
   // row chunks (64 rows each) of this CTA: key blocks, or 64-centroid chunks
   const int nchunk = CENT ? Npad / 64 : N;
-  const int j0 = 2 * p, j1 = 2 * p + 1 < nchunk ? 2 * p + 1 : -1;
+  // 64-row chunks of this CTA: a key-block pair (64-token blocks), the two
+  // tiles of one 128-token block, or 128 consecutive centroids
+  const int2 kp = kpairs ? kpairs[(size_t)bh * P + p] : make_int2(-1, -1);
+  const int j0 = kpairs ? kp.x : 2 * p;
+  const int j1 = kpairs ? kp.y : (2 * p + 1 < nchunk ? 2 * p + 1 : -1);
   const int T = CENT ? N : counts[(size_t)bh * P + p];
   const int *list = CENT ? nullptr : entries + bh * cap + offsets[(size_t)bh * P + p];
   const int row_end = CENT ? Npad : L;   // first row past the K / V (or centroid) rows
@@ -382,7 +407,7 @@ __global__ void __launch_bounds__(320, 1)
       const bool on = CENT ? (kvalid && !((selw >> (key & 31)) & 1u))
                            : (kvalid && (((list[u] & 3) >> half) & 1));
       const float wrow = CENT ? wn : 1.f;
-      const float *ls = vec + sl * (C::kVecBytes / 4);     // lse of the 64 query rows
+      const float *ls = vec + sl * (C::kVecBytes / 4);     // lse * log2 e of the 64 query rows
       const float *dl = ls + 64;                            // Delta of the 64 query rows
       uint32_t pp[32], pd[32];
       if (__any_sync(0xffffffffu, on)) {
@@ -403,7 +428,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
               const float pr = on ? wrow * ex2_approx(fmaf(__uint_as_float(r[h][i + x]), sl2,
-                                                           -lv[x] * kLog2e))
+                                                           -lv[x]))
                                   : 0.f;
               pv[x] = pr;
               zv[x] = pr * (__uint_as_float(r[2 + h][i + x]) - dv4[x]);

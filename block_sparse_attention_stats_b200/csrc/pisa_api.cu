@@ -15,6 +15,7 @@
 #include "pisa_common.cuh"
 #include "k1_block_stats.cuh"
 #include "k2_select.cuh"
+#include "k2_scores_tc.cuh"
 #include "k3_pack.cuh"
 #include "k3_attention_tc.cuh"
 #include "k5_tail_histogram.cuh"
@@ -95,9 +96,22 @@ static size_t stats_ws(int B, int H, int L, int d, int block_size) {
   const int parts = std::max(stats_num_chunks(BH, N), stats_max_segments(BH, N));
   return align_up((size_t)BH * parts * d * d * sizeof(float), 256);
 }
-static size_t select_ws(int B, int H, int N) {
-  return align_up((size_t)B * H * N * N * sizeof(float), 256);
+// two-pass selection: the score matrix (rows padded to a multiple of 32 floats),
+// then the three-part bf16 splits of qbar and kbar (sized for d = 128)
+static int score_ld(int N) { return ceil_div(N, 32) * 32; }
+struct SelectLayout {
+  size_t qs, ks, total;
+};
+static SelectLayout select_layout(int B, int H, int N) {
+  const size_t BH = (size_t)B * H;
+  SelectLayout p;
+  p.qs = align_up(BH * N * score_ld(N) * sizeof(float), 256);
+  const size_t planes = align_up(BH * 3 * N * 128 * 2, 256);
+  p.ks = p.qs + planes;
+  p.total = p.ks + planes;
+  return p;
 }
+static size_t select_ws(int B, int H, int N) { return select_layout(B, H, N).total; }
 // scratch of the fused-attention step: bf16 kbar/vsum/hbar, query-block
 // pairing (selection bitmaps, overlaps, pairs), bf16 copies of f32 inputs
 struct SparseLayout {
@@ -252,13 +266,44 @@ static pisa_status launch_select(const float *qbar, const float *kbar, const flo
         qbar, kbar, cov, cov_weight, scale, N, d, k_sel, sink, idx);
     return check_launch();
   }
-  dim3 g1(ceil_div(N, kScoreTile), ceil_div(N, kScoreTile), BH);
-  scores_kernel<<<g1, 256, 0, st>>>(qbar, kbar, cov, cov_weight, scale, N, d, scores);
+  // pass 1: three-part bf16 splits of the centroids, then the score tiles on
+  // the tensor cores
+  const SelectLayout lay = select_layout(1, BH, N);
+  __nv_bfloat16 *qs = (__nv_bfloat16 *)(ws + lay.qs), *ks = (__nv_bfloat16 *)(ws + lay.ks);
+  const long long rows = (long long)BH * N;
+  centroid_split_kernel<<<grid_1d((size_t)rows * d / 4, 256), 256, 0, st>>>(qbar, kbar, rows, N,
+                                                                             d, qs, ks);
   PISA_TRY(check_launch());
-  const size_t rows = (size_t)BH * N;
+  CUtensorMap mqs, mks;
+  PISA_TRY(make_map(&mqs, qs, d, N, (uint64_t)BH * 3, ScoreTcCfg<128>::kRows));
+  PISA_TRY(make_map(&mks, ks, d, N, (uint64_t)BH * 3, ScoreTcCfg<128>::kCols));
+  const int ld = score_ld(N);
+  const dim3 g1(ceil_div(N, ScoreTcCfg<128>::kRows), BH);
+  if (d == 128) {
+    PISA_CUDA(cudaFuncSetAttribute(scores_tc_kernel<128>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   ScoreTcCfg<128>::kSmem));
+    scores_tc_kernel<128><<<g1, ScoreTcCfg<128>::kThreads, ScoreTcCfg<128>::kSmem, st>>>(
+        mqs, mks, cov, cov_weight, scale, N, ld, scores);
+  } else {
+    PISA_CUDA(cudaFuncSetAttribute(scores_tc_kernel<64>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   ScoreTcCfg<64>::kSmem));
+    scores_tc_kernel<64><<<g1, ScoreTcCfg<64>::kThreads, ScoreTcCfg<64>::kSmem, st>>>(
+        mqs, mks, cov, cov_weight, scale, N, ld, scores);
+  }
+  PISA_TRY(check_launch());
+  // pass 2: one warp per query block, its row staged in shared memory (rows
+  // too long for eight of them in shared memory: the radix select from L2)
   const int per_cta = kTopkThreads / 32;
-  topk_kernel<<<(unsigned)((rows + per_cta - 1) / per_cta), kTopkThreads, 0, st>>>(
-      scores, N, k_sel, sink, rows, idx);
+  const unsigned g2 = (unsigned)((rows + per_cta - 1) / per_cta);
+  const int tsmem = topk_bins_smem(ld);
+  if (tsmem <= 227 * 1024) {
+    PISA_CUDA(cudaFuncSetAttribute(topk_bins_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   tsmem));
+    topk_bins_kernel<<<g2, kTopkThreads, tsmem, st>>>(scores, N, ld, k_sel, sink, rows, idx);
+  } else
+    topk_kernel<<<g2, kTopkThreads, 0, st>>>(scores, N, ld, k_sel, sink, rows, idx);
   return check_launch();
 }
 
@@ -376,7 +421,7 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
     if (pair_smem > 48 * 1024)
       PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      pair_smem));
-    pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
+    pairing_kernel<<<BH, kPairThreads, pair_smem, st>>>(ov, N, staged, pairs);
     PISA_TRY(check_launch());
   } else {
     pairs = nullptr;   // the two 64-row halves of one 128-token query block share S_i
@@ -409,8 +454,8 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
 
 // ---- backward of the zeroth-order variant ------------------------------------
 struct BwdLayout {
-  size_t lse_pad, delta, kbar16, vbar16, bm, ov, pairs, dkbar, dvbar, counts, offsets, entries,
-      total;
+  size_t lse_pad, delta, kbar16, vbar16, bm, ov, pairs, bmT, kpairs, dkbar, dvbar, counts,
+      offsets, entries, total;
   long long cap;   // list entries per head
 };
 static BwdLayout bwd_layout(int B, int H, int L, int d, int k_sel, int block_size) {
@@ -428,6 +473,10 @@ static BwdLayout bwd_layout(int B, int H, int L, int d, int k_sel, int block_siz
   p.bm = o; o += align_up(BH * N * nwords * 4, 256);
   p.ov = o; o += align_up(BH * N * kPairWindow * 2, 256);
   p.pairs = o; o += align_up(BH * P * 8, 256);
+  // key-block pairs of the dk / dv pass (64-token blocks): the transposed
+  // bitmap, then pairs chosen like the query pairs (ov is reused)
+  p.bmT = o; o += block_size == 64 ? align_up(BH * N * nwords * 4, 256) : 0;
+  p.kpairs = o; o += block_size == 64 ? align_up(BH * P * 8, 256) : 0;
   p.dkbar = o; o += align_up(BH * Npad * d * 4, 256);
   p.dvbar = o; o += align_up(BH * Npad * d * 4, 256);
   p.counts = o; o += align_up(BH * P * 4, 256);
@@ -498,7 +547,7 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
     if (pair_smem > 48 * 1024)
       PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      pair_smem));
-    pairing_kernel<<<BH, 32, pair_smem, st>>>(ov, N, staged, pairs);
+    pairing_kernel<<<BH, kPairThreads, pair_smem, st>>>(ov, N, staged, pairs);
     PISA_TRY(check_launch());
   }
   const int dq_smem = DqTcCfg<D>::smem_bytes(N, Nc);
@@ -533,20 +582,40 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kvtc_smem));
   bwd_kv_tc_kernel<D, true><<<dim3(ceil_div(Ncpad, 128), BH), KvTcCfg<D>::kThreads, kvtc_smem,
                               st>>>(
-      mq, mdo, mkb, mvb, mlse, mdel, nullptr, nullptr, 0, nullptr, bm, cwords, bsub, Nc, L, N,
-      scale, dkbar, dvbar, Ncpad, nullptr, nullptr);
+      mq, mdo, mkb, mvb, mlse, mdel, nullptr, nullptr, 0, nullptr, nullptr, bm, cwords, bsub, Nc,
+      L, N, scale, dkbar, dvbar, Ncpad, nullptr, nullptr);
   PISA_TRY(check_launch());
-  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, 0, counts, offsets,
-                                            lay.cap, entries);
+  // 64-token blocks: key blocks paired by how many query blocks select both
+  // (the dk / dv tiles of a query block that selected only one of the two are
+  // half wasted), with the query pairing's greedy over the transposed bitmap
+  int2 *kpairs = nullptr;
+  if (bsub == 1) {
+    uint32_t *bmT = (uint32_t *)(ws + lay.bmT);
+    uint16_t *ov = (uint16_t *)(ws + lay.ov);
+    kpairs = (int2 *)(ws + lay.kpairs);
+    bitmap_transpose_kernel<<<dim3(cwords, cwords, BH), 32, 0, st>>>(bm, N, cwords, bmT);
+    PISA_TRY(check_launch());
+    pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bmT, N, cwords, ov);
+    PISA_TRY(check_launch());
+    const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
+    const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
+    if (pair_smem > 48 * 1024)
+      PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     pair_smem));
+    pairing_kernel<<<BH, kPairThreads, pair_smem, st>>>(ov, N, staged, kpairs);
+    PISA_TRY(check_launch());
+  }
+  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, kpairs, 0, counts,
+                                            offsets, lay.cap, entries);
   PISA_TRY(check_launch());
   kvlist_scan_kernel<<<BH, 1024, 0, st>>>(counts, P, offsets);
   PISA_TRY(check_launch());
-  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, 1, counts, offsets,
-                                            lay.cap, entries);
+  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, kpairs, 1, counts,
+                                            offsets, lay.cap, entries);
   PISA_TRY(check_launch());
   bwd_kv_tc_kernel<D, false><<<dim3(P, BH), KvTcCfg<D>::kThreads, kvtc_smem, st>>>(
-      mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, bm, cwords, bsub, Nc, L, N,
-      scale, dkbar, dvbar, Ncpad, dk, dv);
+      mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, kpairs, bm, cwords, bsub,
+      Nc, L, N, scale, dkbar, dvbar, Ncpad, dk, dv);
   return check_launch();
 }
 

@@ -124,9 +124,12 @@ def test_block_size_128(P, L, d, sink, mode, cov):
 ])
 def test_block_size_128_selection_in_fused_kernel(P, L, d, sink, mode, cov):
     """With 128-token blocks the fused kernel can select inside (each CTA is
-    one query block): the sets equal the separate selection step's bit for
-    bit (same float32 scores and tie rule), so does the output, and both
-    match the oracle."""
+    one query block).  Up to 512 blocks the separate step scores with the same
+    float32 FMA chain, so the sets and the outputs are equal bit for bit.  On
+    longer rows the separate step's scores come from the tensor cores: a row
+    may differ only where the oracle certifies a rounding tie, and rows that
+    agree give the same output rows bit for bit.  The fused sets match the
+    oracle."""
     wl = WORKLOADS["flux"].with_(B=1, H=2, L=L, d=d, block_size=128, sink_idx=sink, mode=mode,
                                  cov_weight=cov, cluster_kind="block", density=0.2)
     Q, K, V = generate_qkv(wl, "cpu")
@@ -140,8 +143,24 @@ def test_block_size_128_selection_in_fused_kernel(P, L, d, sink, mode, cov):
     out_s = P.pisa_attention_ex(q, k, v, wl.density, 128, sink, mode, cov_weight=cov,
                                 idx_out=idx_s)
     P.pisa_device_status()
-    assert torch.equal(idx_f, idx_s)
-    assert torch.equal(out_f, out_s)
+    if N <= 512:
+        assert torch.equal(idx_f, idx_s)
+        assert torch.equal(out_f, out_s)
+    else:
+        for h in range(2):
+            diff = (idx_f[0, h] != idx_s[0, h]).any(-1).cpu().numpy()
+            if diff.any():
+                st = O.block_stats(to64(Q[0, h]), to64(K[0, h]), to64(V[0, h]), 128)
+                rows = list(range(N))
+                sc = O.selection_scores(st["qbar"], st["kbar"], wl.scale, None, 0.0, rows)
+                orc = dict(qbar=st["qbar"], kbar=st["kbar"], cov=None, rows=np.asarray(rows),
+                           idx=O.select_blocks(sc, k_sel, sink), scores=sc)
+                rep = compare_selection(idx_s[0, h].cpu().numpy(), orc, wl.scale, 0.0, sink)
+                assert not rep.bad_rows, rep.bad_rows
+                assert set(np.nonzero(diff)[0]) <= set(rep.tie_rows)
+            same = np.repeat(~diff, 128)[:L]
+            assert torch.equal(out_f[0, h][torch.from_numpy(same).cuda()],
+                               out_s[0, h][torch.from_numpy(same).cuda()])
     heads = [(0, 0), (0, 1)] if L < 20000 else [(0, 1)]
     for (b, h) in heads:
         r = O.pisa_attention_head(to64(Q[b, h]), to64(K[b, h]), to64(V[b, h]), 128, wl.density,
