@@ -48,9 +48,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the fused attention kernel, from an ncu capture,
 # keyed by the sha1 of the kernel source it was taken on (see profiles/).
 K3_TRAFFIC = {
-    # H=4 ncu capture (dram read 240.1 MB + write 60.8 MB per launch) scaled by
+    # H=4 ncu capture (dram read 240.4 MB + write 61.1 MB per launch) scaled by
     # 10 to the 40 heads; profiles/piecewise_attention_tc_wan_h4.md
-    "6d5287a9c780": {"wan": 3.009e9},
+    "a0503d7f1a2e": {"wan": 3.016e9},
 }
 
 

@@ -405,21 +405,24 @@ __global__ void __launch_bounds__(192, 2)
     constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
     bool ok = uwait(bar(C::kBarQ), 0);
     tc_fence_after();
+    // descriptors are built once per buffer; a K step adds its byte offset / 16
+    // to the start-address field (the field cannot carry: shared memory is
+    // below 256 KB)
+    const uint64_t qd0 = smem_desc_sw128(sbase + C::kOffQ, 16, 1024);
     auto q_desc = [&](int k) -> uint64_t {
-      return smem_desc_sw128(sbase + C::kOffQ + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
+      return qd0 + (uint64_t)(((k >> 2) * C::kBoxQBytes + (k & 3) * 32) >> 4);
     };
     auto issue_pv = [&](int u) -> bool {
       const int bu = u & 1, sv = u % C::kVStages;
       if (!uwait(bar(C::kBarPFull + bu), (u >> 1) & 1)) return false;
       if (!uwait(bar(C::kBarVFull + sv), (u / C::kVStages) & 1)) return false;
       tc_fence_after();
-      const uint32_t vst = sbase + C::kOffV + sv * C::kTileBytes;
+      const uint64_t vd0 = smem_desc_sw128(sbase + C::kOffV + sv * C::kTileBytes, C::kBoxKBytes, 1024);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tmem + C::kColO, tmem + C::kColS + 64 * bu + kk * 8,
-                 smem_desc_sw128(vst + kk * 2048, C::kBoxKBytes, 1024), kIdPV,
-                 (u > 0 || kk > 0) ? 1u : 0u);
+                 vd0 + (uint64_t)((kk * 2048) >> 4), kIdPV, (u > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(C::kBarVEmpty + sv));
         tc_commit(bar(C::kBarODone));
       }
@@ -431,12 +434,12 @@ __global__ void __launch_bounds__(192, 2)
       const int sk = t % C::kKStages, b = t & 1;
       if (!uwait(bar(C::kBarKFull + sk), (t / C::kKStages) & 1)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t kst = sbase + C::kOffK + sk * C::kTileBytes;
+      const uint64_t kd0 = smem_desc_sw128(sbase + C::kOffK + sk * C::kTileBytes, 16, 1024);
       if (elect_one()) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem + C::kColS + 64 * b, q_desc(k),
-                 smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024), kIdQK,
+                 kd0 + (uint64_t)(((k >> 2) * C::kBoxKBytes + (k & 3) * 32) >> 4), kIdQK,
                  k > 0 ? 1u : 0u);
         tc_commit(bar(C::kBarSFull + b));
         tc_commit(bar(C::kBarKEmpty + sk));
