@@ -681,12 +681,12 @@ def run_pisa(args, wl):
         p_sus_b = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         p_burst_b = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         ex_tf = f_exec_b / (bms * 1e-3) / 1e12 if f_exec_b else None
-        bwd = {"ms": bms, "mode": "0th", "launches": 12 if wl.block_size == 64 else 10,
+        bwd = {"ms": bms, "mode": "0th", "launches": 15 if wl.block_size == 64 else 10,
                "delta": "dout . o from the forward's float32 output (bwd_delta_kernel)",
                "kernels": "dq: bwd_dq_tc (tcgen05, one sweep); dk/dv of exact keys: "
                           "bwd_kv_tc<false> (tcgen05); centroid gradients: bwd_kv_tc<true> "
                           "(tcgen05, centroid rows weighted by n_j); "
-                          "packing, bitmap, pairing, padding, list kernels",
+                          "packing, bitmap, query- and key-block pairing, padding, list kernels",
                "roofline": {"bound": "tensor", "achieved": f_alg_b / (bms * 1e-3) / 1e12,
                             "peak": p_burst_b, "peak_kind": "bf16 dense, burst",
                             "unit": "TFLOP/s",
@@ -780,11 +780,12 @@ def run_pisa(args, wl):
     src = _k3_source_hash()
     traffic = K3_TRAFFIC.get(src, {}).get(wl.name)
     # statistics: pass 1 + hbar reduction (+ covariance pass); selection: one
-    # fused kernel, or split + score tiles + top-k; fused step: statistics packing (+ bitmap, overlaps, pairing with
-    # 64-token blocks) (+ three f32 -> bf16 copies) + the fused kernel
+    # fused kernel, or split + score tiles + top-k; fused step: with 64-token
+    # blocks packing + bitmap (one launch), overlaps, pairing; with 128-token
+    # blocks packing; (+ three f32 -> bf16 copies) + the fused kernel
     n_sel = 1 if N <= 512 else 3
     launches_per_step = (2 + (1 if want_cov else 0) + n_sel
-                         + (5 if wl.block_size == 64 else 2) + (3 if wl.dtype == "f32" else 0))
+                         + (4 if wl.block_size == 64 else 2) + (3 if wl.dtype == "f32" else 0))
     line = {
         "metric": METRIC,
         "value": weak_scaling_value(world, dense_flops(wl), t_step),

@@ -72,6 +72,49 @@ __global__ void selection_bitmap_kernel(const int32_t *__restrict__ idx, int N, 
   for (int w = threadIdx.x; w < nwords; w += blockDim.x) bm[row * nwords + w] = words[w];
 }
 
+// The two preparation steps of the 64-token fused step in one launch: CTAs
+// 0 .. N*BH-1 build the selection bitmap rows (as selection_bitmap_kernel),
+// the rest pack the statistics (as pack_stats_kernel, grid-stride).
+constexpr int kPackThreads = 128;
+__global__ void __launch_bounds__(kPackThreads)
+    pack_and_bitmap_kernel(const float *__restrict__ kbar, const float *__restrict__ vsum,
+                           const float *__restrict__ hbar, int N, int Npad, int D, int BH,
+                           __nv_bfloat16 *__restrict__ kbar16, __nv_bfloat16 *__restrict__ vsum16,
+                           __nv_bfloat16 *__restrict__ hbar16, const int32_t *__restrict__ idx,
+                           int k_sel, int nwords, uint32_t *__restrict__ bm) {
+  extern __shared__ uint32_t words[];
+  const size_t nbm = (size_t)N * BH;
+  if (blockIdx.x < nbm) {
+    const size_t row = blockIdx.x;     // bh * N + i
+    for (int w = threadIdx.x; w < nwords; w += blockDim.x) words[w] = 0u;
+    __syncthreads();
+    for (int t = threadIdx.x; t < k_sel; t += blockDim.x) {
+      const int j = idx[row * k_sel + t];
+      if (j >= 0 && j < N) atomicOr(&words[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
+    for (int w = threadIdx.x; w < nwords; w += blockDim.x) bm[row * nwords + w] = words[w];
+    return;
+  }
+  const size_t nrow = (size_t)BH * Npad * D;
+  const size_t nh = (size_t)BH * D * D;
+  const size_t stride = (size_t)(gridDim.x - nbm) * blockDim.x;
+  for (size_t e = (blockIdx.x - nbm) * (size_t)blockDim.x + threadIdx.x; e < nrow + nh;
+       e += stride) {
+    if (e < nrow) {
+      const size_t bh = e / ((size_t)Npad * D), rem = e % ((size_t)Npad * D);
+      const int j = (int)(rem / D), c = (int)(rem % D);
+      const bool ok = j < N;
+      const size_t src = (bh * N + j) * D + c;
+      kbar16[e] = __float2bfloat16_rn(ok ? kbar[src] : 0.f);
+      vsum16[e] = __float2bfloat16_rn(ok ? vsum[src] : 0.f);
+    } else {
+      const size_t h = e - nrow;
+      hbar16[h] = __float2bfloat16_rn(hbar[h]);
+    }
+  }
+}
+
 // ov[bh][i][d-1] = |S_i n S_{i+d}| for d = 1 .. kPairWindow (0 past the end).
 // One CTA per 8 consecutive blocks i (a warp each, lane l takes d = l + 1 and
 // l + 33).  The 72 bitmap rows they touch are staged in shared memory 32
@@ -147,18 +190,22 @@ __global__ void __launch_bounds__(kPairThreads)
   int np = 0;
   uint64_t ahead = 0ull;       // bit d: block i + 1 + d is paired already
   bool self = false;           // block i is paired already
+  const uint64_t bit_lo = 1ull << lane, bit_hi = 1ull << (32 + lane);
   // the overlaps of the current block's window positions lane and lane + 32
   unsigned o0 = o[lane], o1 = o[32 + lane];
   for (int i = 0; i < N; ++i) {
     const unsigned n0 = i + 1 < N ? o[(size_t)(i + 1) * kPairWindow + lane] : 0u;
     const unsigned n1 = i + 1 < N ? o[(size_t)(i + 1) * kPairWindow + 32 + lane] : 0u;
+    // the block entering the window next; re-read below if this step pairs
+    // past the window (the only writes to `used`)
+    const bool in_next = i + 1 + kPairWindow < N;
+    bool next_used = in_next && used[i + 1 + kPairWindow];
     if (!self) {
       // key + 1: overlap high, then nearer partner first; 0 = no candidate
-      const int j0 = i + 1 + lane, j1 = i + 33 + lane;
       unsigned key = 0u;
-      if (j0 < N && !((ahead >> lane) & 1ull)) key = ((o0 << 8) | (255u - lane)) + 1u;
-      if (j1 < N && !((ahead >> (32 + lane)) & 1ull))
-        key = max(key, ((o1 << 8) | (255u - 32u - lane)) + 1u);
+      if (i + 1 + lane < N && !(ahead & bit_lo)) key = ((o0 << 8) | (255u - lane)) + 1u;
+      if (i + 33 + lane < N && !(ahead & bit_hi))
+        key = max(key, ((o1 << 8) | (223u - lane)) + 1u);
       const unsigned best = __reduce_max_sync(0xffffffffu, key);
       int partner = -1;
       if (best > 0u) {
@@ -170,15 +217,16 @@ __global__ void __launch_bounds__(kPairThreads)
           if (!used[jj]) { partner = jj; break; }
         __syncwarp();
         if (lane == 0 && partner >= 0) used[partner] = 1;
+        __syncwarp();
+        next_used = in_next && used[i + 1 + kPairWindow];
       }
       if (lane == 0) out[np] = make_int2(i, partner);
       ++np;
     }
     // slide the window by one block
-    __syncwarp();
     self = ahead & 1ull;
     ahead >>= 1;
-    if (i + 1 + kPairWindow < N && used[i + 1 + kPairWindow]) ahead |= 1ull << (kPairWindow - 1);
+    if (next_used) ahead |= 1ull << (kPairWindow - 1);
     o0 = n0;
     o1 = n1;
   }

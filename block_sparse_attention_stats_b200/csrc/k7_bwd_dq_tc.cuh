@@ -311,8 +311,15 @@ __global__ void __launch_bounds__(352, 1)
     const bool s_warp = warp == 1;
     bool ok = uwait(bar(C::kBarQ), 0);
     tc_fence_after();
-    auto a_desc = [&](uint32_t off, int k) -> uint64_t {
-      return smem_desc_sw128(sbase + off + (k >> 2) * C::kBoxQBytes + (k & 3) * 32, 16, 1024);
+    // descriptors are built once per buffer; a K step adds its byte offset / 16
+    // to the start-address field (which cannot carry below 256 KB)
+    const uint64_t qd0 = smem_desc_sw128(sbase + C::kOffQ, 16, 1024);
+    const uint64_t dod0 = smem_desc_sw128(sbase + C::kOffDO, 16, 1024);
+    auto a_step = [](int k) -> uint64_t {
+      return (uint64_t)(((k >> 2) * C::kBoxQBytes + (k & 3) * 32) >> 4);
+    };
+    auto b_step = [](int k) -> uint64_t {
+      return (uint64_t)(((k >> 2) * C::kBoxKBytes + (k & 3) * 32) >> 4);
     };
     // warp 10: the second-sweep product for tile w once its dS is in TMEM (in
     // the first sweep only the wait for the dS warpgroup)
@@ -322,13 +329,12 @@ __global__ void __launch_bounds__(352, 1)
       if (w >= T1) {
         tc_fence_after();
         const int db = (w - T1) & 1;
-        const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
+        const uint64_t kd = smem_desc_sw128(sbase + C::kOffK + sl * C::kTileBytes, C::kBoxKBytes, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + C::kColDQ, tmem + C::kColDS + 32 * db + kk * 8,
-                   smem_desc_sw128(kst + kk * 2048, C::kBoxKBytes, 1024), kIdDQ,
-                   (w > T1 || kk > 0) ? 1u : 0u);
+                   kd + (uint64_t)((kk * 2048) >> 4), kIdDQ, (w > T1 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::kBarKEmpty + sl));
           tc_commit(bar(C::kBarDsFree + db));
         }
@@ -343,13 +349,12 @@ __global__ void __launch_bounds__(352, 1)
         if (u >= 2 && !uwait(bar(C::kBarPFull + b), ((u - 2) >> 1) & 1)) { ok = false; break; }
         if (!uwait(bar(C::kBarKFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t kst = sbase + C::kOffK + sl * C::kTileBytes;
+        const uint64_t kd = smem_desc_sw128(sbase + C::kOffK + sl * C::kTileBytes, 16, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b, a_desc(C::kOffQ, k),
-                   smem_desc_sw128(kst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024),
-                   kIdQK, k > 0 ? 1u : 0u);
+            mma_ss(tmem + C::kColBuf + 128 * b, qd0 + a_step(k), kd + b_step(k), kIdQK,
+                   k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarSFull + b));
           if (u < T1) tc_commit(bar(C::kBarKEmpty + sl));
         }
@@ -357,13 +362,12 @@ __global__ void __launch_bounds__(352, 1)
       } else {
         if (!uwait(bar(C::kBarVFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t vst = sbase + C::kOffV + sl * C::kTileBytes;
+        const uint64_t vd = smem_desc_sw128(sbase + C::kOffV + sl * C::kTileBytes, 16, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b + 64, a_desc(C::kOffDO, k),
-                   smem_desc_sw128(vst + (k >> 2) * C::kBoxKBytes + (k & 3) * 32, 16, 1024),
-                   kIdQK, k > 0 ? 1u : 0u);
+            mma_ss(tmem + C::kColBuf + 128 * b + 64, dod0 + a_step(k), vd + b_step(k), kIdQK,
+                   k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarSFull + b));
           tc_commit(bar(C::kBarVEmpty + sl));
         }

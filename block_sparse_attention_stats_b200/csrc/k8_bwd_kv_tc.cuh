@@ -318,27 +318,34 @@ __global__ void __launch_bounds__(320, 1)
     if (T > 0) {
       ok = uwait(bar(C::kBarKV), 0);
       tc_fence_after();
-      auto a_desc = [&](uint32_t off, int k) -> uint64_t {
-        return smem_desc_sw128(sbase + off + (k >> 2) * C::kBoxPairBytes + (k & 3) * 32, 16, 1024);
+      // descriptors are built once per buffer; a K step adds its byte offset /
+      // 16 to the start-address field (which cannot carry below 256 KB)
+      const uint64_t kd0 = smem_desc_sw128(sbase + C::kOffK, 16, 1024);
+      const uint64_t vd0 = smem_desc_sw128(sbase + C::kOffV, 16, 1024);
+      auto a_step = [](int k) -> uint64_t {
+        return (uint64_t)(((k >> 2) * C::kBoxPairBytes + (k & 3) * 32) >> 4);
+      };
+      auto b_step = [](int k) -> uint64_t {
+        return (uint64_t)(((k >> 2) * C::kBoxRowBytes + (k & 3) * 32) >> 4);
       };
       // dV and dK products of tile w once P^T and dS^T are in TMEM
       auto finish = [&](int w) -> bool {
         const int b = w & 1, sl = w % C::kStages;
         if (!uwait(bar(C::kBarPFull + b), (w >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t qst = sbase + C::kOffQ + sl * C::kTileBytes;
-        const uint32_t dst_ = sbase + C::kOffDO + sl * C::kTileBytes;
+        const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + sl * C::kTileBytes,
+                                            C::kBoxRowBytes, 1024);
+        const uint64_t dd = smem_desc_sw128(sbase + C::kOffDO + sl * C::kTileBytes,
+                                            C::kBoxRowBytes, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + C::kColDV, tmem + C::kColBuf + 128 * b + kk * 8,
-                   smem_desc_sw128(dst_ + kk * 2048, C::kBoxRowBytes, 1024), kIdAcc,
-                   (w > 0 || kk > 0) ? 1u : 0u);
+                   dd + (uint64_t)((kk * 2048) >> 4), kIdAcc, (w > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + C::kColDK, tmem + C::kColBuf + 128 * b + 64 + kk * 8,
-                   smem_desc_sw128(qst + kk * 2048, C::kBoxRowBytes, 1024), kIdAcc,
-                   (w > 0 || kk > 0) ? 1u : 0u);
+                   qd + (uint64_t)((kk * 2048) >> 4), kIdAcc, (w > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::kBarQEmpty + sl));
         }
         __syncwarp();
@@ -349,19 +356,17 @@ __global__ void __launch_bounds__(320, 1)
         const int sl = u % C::kStages, b = u & 1;
         if (!uwait(bar(C::kBarQFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t qst = sbase + C::kOffQ + sl * C::kTileBytes;
-        const uint32_t dst_ = sbase + C::kOffDO + sl * C::kTileBytes;
+        const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + sl * C::kTileBytes, 16, 1024);
+        const uint64_t dd = smem_desc_sw128(sbase + C::kOffDO + sl * C::kTileBytes, 16, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b, a_desc(C::kOffK, k),
-                   smem_desc_sw128(qst + (k >> 2) * C::kBoxRowBytes + (k & 3) * 32, 16, 1024),
-                   kIdS, k > 0 ? 1u : 0u);
+            mma_ss(tmem + C::kColBuf + 128 * b, kd0 + a_step(k), qd + b_step(k), kIdS,
+                   k > 0 ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b + 64, a_desc(C::kOffV, k),
-                   smem_desc_sw128(dst_ + (k >> 2) * C::kBoxRowBytes + (k & 3) * 32, 16, 1024),
-                   kIdS, k > 0 ? 1u : 0u);
+            mma_ss(tmem + C::kColBuf + 128 * b + 64, vd0 + a_step(k), dd + b_step(k), kIdS,
+                   k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarSFull + b));
         }
         __syncwarp();

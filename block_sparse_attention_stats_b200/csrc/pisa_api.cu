@@ -406,13 +406,13 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
   uint32_t *bm = (uint32_t *)(ws + lay.bm);
   uint16_t *ov = (uint16_t *)(ws + lay.ov);
   int2 *pairs = (int2 *)(ws + lay.pairs);
-  pack_stats_kernel<<<grid_1d((size_t)BH * (Ncpad * d + d * d), 256), 256, 0, st>>>(
-      kbar, vsum, hbar, Nc, Ncpad, d, BH, kbar16, vsum16, hbar16);
-  PISA_TRY(check_launch());
   if (bsub == 1) {
+    // statistics packing and the selection bitmap in one launch; then the
     // schedule: pair query blocks whose exact sets overlap most
-    selection_bitmap_kernel<<<dim3(N, BH), 64, nwords * sizeof(uint32_t), st>>>(idx, N, k_sel,
-                                                                                nwords, bm);
+    const unsigned npack = grid_1d((size_t)BH * (Ncpad * d + d * d), kPackThreads);
+    pack_and_bitmap_kernel<<<(unsigned)((size_t)N * BH) + npack, kPackThreads,
+                             nwords * sizeof(uint32_t), st>>>(
+        kbar, vsum, hbar, Nc, Ncpad, d, BH, kbar16, vsum16, hbar16, idx, k_sel, nwords, bm);
     PISA_TRY(check_launch());
     pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bm, N, nwords, ov);
     PISA_TRY(check_launch());
@@ -424,6 +424,9 @@ static pisa_status run_sparse_attention(const void *q, const void *k, const void
     pairing_kernel<<<BH, kPairThreads, pair_smem, st>>>(ov, N, staged, pairs);
     PISA_TRY(check_launch());
   } else {
+    pack_stats_kernel<<<grid_1d((size_t)BH * (Ncpad * d + d * d), 256), 256, 0, st>>>(
+        kbar, vsum, hbar, Nc, Ncpad, d, BH, kbar16, vsum16, hbar16);
+    PISA_TRY(check_launch());
     pairs = nullptr;   // the two 64-row halves of one 128-token query block share S_i
   }
   const __nv_bfloat16 *q16 = (const __nv_bfloat16 *)q, *k16 = (const __nv_bfloat16 *)k,

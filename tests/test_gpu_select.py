@@ -75,6 +75,14 @@ def test_long_row_selection_clustered(P, L, density, sink, cov):
     assert ties <= wl.H * (L // 64) // 100, f"{ties} certified rounding ties"
 
 
+def test_long_row_selection_head_dim_64(P):
+    """d = 64: one 64-column box per split plane in the score kernel."""
+    wl = WORKLOADS["flux"].with_(H=2, L=64 * 700 + 33, d=64, density=0.125, sink_idx=-1,
+                                 cov_weight=0.1, cluster_kind="block")
+    Q, K, V = generate_qkv(wl, "cpu")
+    assert _check(P, wl, Q, K, V) <= wl.H * (wl.L // 64) // 100
+
+
 @pytest.mark.parametrize("cov", [0.0, 0.1])
 def test_long_row_selection_zero_queries(P, cov):
     """q = 0 makes every relevance term exactly 0: without the covariance term
