@@ -164,9 +164,10 @@ __global__ void __launch_bounds__(kTopkThreads)
 //  2. One histogram of the candidates' bins; scanning from the top bin gives
 //     the bin b* that holds the `need`-th largest key and how many keys of b*
 //     are still to be taken.
-//  3. The (at most kBinCand) scores of b* are gathered and T is the one whose
-//     count of larger scores is below, and whose count of larger or equal
-//     scores reaches, the number still to be taken.
+//  3. The (at most kBinCand) scores of b* are gathered (in any order: only
+//     their multiset matters) and T is the one whose count of larger scores is
+//     below, and whose count of larger or equal scores reaches, the number
+//     still to be taken.
 // Comparing floats gives the key order (only -0 and +0 share a key, and they
 // compare equal).  Then the same compaction as topk_row keeps the sink, every
 // score > T and the lowest-index scores equal to T.  Rows where the bins do
@@ -239,10 +240,15 @@ __global__ void __launch_bounds__(kTopkThreads)
   for (int c = lane; c < ld / 4; c += 32) {
     const float4 x4 = *reinterpret_cast<const float4 *>(srow + 4 * c);
     const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+    if (4 * c + 3 < N && (unsigned)(sink - 4 * c) > 3u) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = 4 * c + e;
-      if (j < N && j != sink) atomicAdd(&hist[bin_of(xs[e])], 1u);
+      for (int e = 0; e < 4; ++e) atomicAdd(&hist[bin_of(xs[e])], 1u);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * c + e;
+        if (j < N && j != sink) atomicAdd(&hist[bin_of(xs[e])], 1u);
+      }
     }
   }
   __syncwarp();
@@ -282,14 +288,21 @@ __global__ void __launch_bounds__(kTopkThreads)
   }
   // 3. the scores of b*, and T among them: the `take`-th largest; eq = how
   //    many candidates equal T, rem = how many of those are kept
-  int base = 0;
-  for (int j0 = 0; j0 < N; j0 += 32) {
-    const int j = j0 + lane;
-    const float x = j < N ? srow[j] : 0.f;
-    const bool in = j < N && j != sink && bin_of(x) == bstar;
-    const unsigned bal = __ballot_sync(0xffffffffu, in);
-    if (in) cand[base + __popc(bal & ((1u << lane) - 1u))] = x;
-    base += __popc(bal);
+  // (the order of the gathered scores does not matter: T and the counts
+  // depend only on their multiset)
+  unsigned *ncand = hist;                // the histogram is no longer needed
+  __syncwarp();
+  if (lane == 0) *ncand = 0u;
+  __syncwarp();
+#pragma unroll 2
+  for (int c = lane; c < ld / 4; c += 32) {
+    const float4 x4 = *reinterpret_cast<const float4 *>(srow + 4 * c);
+    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * c + e;
+      if (j < N && j != sink && bin_of(xs[e]) == bstar) cand[atomicAdd(ncand, 1u)] = xs[e];
+    }
   }
   __syncwarp();
   float T = 0.f;
@@ -323,6 +336,39 @@ __global__ void __launch_bounds__(kTopkThreads)
   // to T (all of them when rem == eq, the usual case)
   const bool ties = rem != eq;
   int out_base = 0, eq_base = 0;
+  if (!ties) {
+    // lane l holds blocks 4 (32 it + l) .. +3; its kept count goes into the
+    // warp's exclusive prefix as three bit-plane ballots
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll 2
+    for (int c0 = 0; c0 < ld / 4; c0 += 32) {
+      const int c = c0 + lane;
+      const float4 x4 = c < ld / 4 ? *reinterpret_cast<const float4 *>(srow + 4 * c)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+      unsigned keep = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * c + e;
+        if (j < N && (j == sink || xs[e] >= T)) keep |= 1u << e;
+      }
+      const unsigned n = __popc(keep);
+      const unsigned b0 = __ballot_sync(0xffffffffu, n & 1u);
+      const unsigned b1 = __ballot_sync(0xffffffffu, n & 2u);
+      const unsigned b2 = __ballot_sync(0xffffffffu, n & 4u);
+      int pos = out_base + __popc(b0 & lt) + 2 * __popc(b1 & lt) + 4 * __popc(b2 & lt);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((keep >> e) & 1u) {
+          if (pos < k_sel) out[pos] = 4 * c + e;
+          else report_device_error(kDevErrRange);
+          ++pos;
+        }
+      out_base += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+    }
+    if (lane == 0 && out_base != k_sel) report_device_error(kDevErrRange);
+    return;
+  }
   for (int j0 = 0; j0 < N; j0 += 32) {
     const int j = j0 + lane;
     const bool valid = j < N;
