@@ -60,6 +60,10 @@ template <int D> struct DqTcCfg {
   static constexpr uint32_t kColDQ = 0;
   static constexpr uint32_t kColBuf = D;                        // + 128 b
   static constexpr uint32_t kColDS = D + 256;                   // + 32 b: packed bf16 dS
+  // Q as packed bf16 pairs (D / 2 columns), the A operand of the S products:
+  // read from tensor memory, an N = 64 product needs only its 2 KB of K tile
+  // from shared memory instead of 6 KB, which bounds it at ~52 pipe cycles
+  static constexpr uint32_t kColQ = D + 320;
   static constexpr int kBarQ = 0;
   static constexpr int kBarKFull = 1;                           // + slot
   static constexpr int kBarKEmpty = kBarKFull + kStages;
@@ -71,7 +75,9 @@ template <int D> struct DqTcCfg {
   static constexpr int kBarDelta = kBarDsFree + 2;
   static constexpr int kBarFinal = kBarDelta + 1;
   static constexpr int kBarTeardown = kBarFinal + 1;
-  static_assert(kBarTeardown < kNumBars, "barrier slots");
+  static constexpr int kBarQT = kBarTeardown + 1;                // Q copied into TMEM
+  static_assert(kBarQT < kNumBars, "barrier slots");
+  static_assert(kColQ + D / 2 <= kTmemCols, "tensor memory columns");
 
   // N 64-token tiles, Nc blocks (= centroids)
   __host__ __device__ static int smem_bytes(int N, int Nc) {
@@ -156,6 +162,7 @@ __global__ void __launch_bounds__(352, 1)
     mbar_init(bar(C::kBarDelta), 256);
     mbar_init(bar(C::kBarFinal), 1);
     mbar_init(bar(C::kBarTeardown), 2);
+    mbar_init(bar(C::kBarQT), 4);
     fence_mbar_init();
     misc[1] = 0;
   }
@@ -313,8 +320,9 @@ __global__ void __launch_bounds__(352, 1)
     tc_fence_after();
     // descriptors are built once per buffer; a K step adds its byte offset / 16
     // to the start-address field (which cannot carry below 256 KB)
-    const uint64_t qd0 = smem_desc_sw128(sbase + C::kOffQ, 16, 1024);
     const uint64_t dod0 = smem_desc_sw128(sbase + C::kOffDO, 16, 1024);
+    if (s_warp && ok) ok = uwait(bar(C::kBarQT), 0);   // Q in tensor memory
+    tc_fence_after();
     auto a_step = [](int k) -> uint64_t {
       return (uint64_t)(((k >> 2) * C::kBoxQBytes + (k & 3) * 32) >> 4);
     };
@@ -353,7 +361,7 @@ __global__ void __launch_bounds__(352, 1)
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b, qd0 + a_step(k), kd + b_step(k), kIdQK,
+            mma_ts(tmem + C::kColBuf + 128 * b, tmem + C::kColQ + 8 * k, kd + b_step(k), kIdQK,
                    k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarSFull + b));
           if (u < T1) tc_commit(bar(C::kBarKEmpty + sl));
@@ -408,6 +416,34 @@ __global__ void __launch_bounds__(352, 1)
     auto warp_wait = [&](uint32_t b_addr, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b_addr, parity));
     };
+    if (g == 0) {
+      // this thread's query row of Q, from the 128-byte-swizzled TMA boxes
+      // (16-byte chunk c of row r sits at chunk c ^ (r & 7)) into tensor
+      // memory as packed bf16 pairs; every warp arrives, even after a timeout
+      if (warp_wait(bar(C::kBarQ), 0)) {
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          uint32_t w[32];
+          const unsigned char *box = smem + C::kOffQ + h * C::kBoxQBytes + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(box + ((c ^ (row & 7)) << 4));
+            w[4 * c] = v.x;
+            w[4 * c + 1] = v.y;
+            w[4 * c + 2] = v.z;
+            w[4 * c + 3] = v.w;
+          }
+          tmem_st_x32(lane_addr + C::kColQ + 32 * h, w);
+        }
+        tmem_wait_st();
+      } else {
+        ok = false;
+        misc[1] = 1;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::kBarQT));
+    }
     // combine the two warpgroups' Delta partial sums (once, before the first
     // second-sweep tile of this warpgroup, or after its loop)
     auto exchange = [&]() -> bool {
