@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(32 * 10, 1)
     const bool sums = p < 3 * (D / 2);
     const uint32_t col_off = (uint32_t)(tns * T::kTileBytes + (lp / 32) * T::kBoxBytes);
     const int chunk = (lp % 32) / 4, inword = (lp % 4) * 4;
-    float cs0 = 0.f, cs1 = 0.f;
+    float ps0[4] = {0.f, 0.f, 0.f, 0.f}, ps1[4] = {0.f, 0.f, 0.f, 0.f};
     auto flush = [&](int bh) {
       const int seg = c - stats_cta_of((long long)bh * N, total, nc);
       float *P = partial + ((size_t)bh * maxseg + seg) * D * D + (size_t)arow * D + ch * kH;
@@ -476,15 +476,15 @@ __global__ void __launch_bounds__(32 * 10, 1)
           break;
         }
         if (sums) {
-          const uint32_t base = sbase + slot * T::kStageBytes + col_off + inword;
-#pragma unroll 8
+          // four interleaved partial sums (rows r % 4) keep four load-add
+          // chains in flight; they are combined in a fixed order at block end
+          const unsigned char *tile = smem + slot * T::kStageBytes + col_off + inword;
+#pragma unroll 16
           for (int r = 0; r < kBlk; ++r) {
-            uint32_t w;
-            asm volatile("ld.shared.b32 %0, [%1];"
-                         : "=r"(w)
-                         : "r"(base + r * 128 + ((chunk ^ (r & 7)) << 4)));
-            cs0 += __uint_as_float(w << 16);
-            cs1 += __uint_as_float(w & 0xffff0000u);
+            const uint32_t w =
+                *reinterpret_cast<const uint32_t *>(tile + r * 128 + ((chunk ^ (r & 7)) << 4));
+            ps0[r & 3] += __uint_as_float(w << 16);
+            ps1[r & 3] += __uint_as_float(w & 0xffff0000u);
           }
         }
         __syncwarp();
@@ -494,6 +494,8 @@ __global__ void __launch_bounds__(32 * 10, 1)
       const int n_j = min(sub * kBlk, L - j * sub * kBlk);
       const float inv_n = 1.f / (float)n_j;
       float *kv = reinterpret_cast<float *>(smem + T::kOffKV) + g * 2 * D;   // kbar, vsum
+      const float cs0 = (ps0[0] + ps0[1]) + (ps0[2] + ps0[3]);
+      const float cs1 = (ps1[0] + ps1[1]) + (ps1[2] + ps1[3]);
       if (sums && !bad) {
         const size_t so = ((size_t)bh * N + j) * D + 2 * lp;
         if (tns == 0) {
@@ -508,7 +510,8 @@ __global__ void __launch_bounds__(32 * 10, 1)
           kv[D + 2 * lp + 1] = cs1;
         }
       }
-      cs0 = cs1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ps0[k] = ps1[k] = 0.f;
       if (!__all_sync(0xffffffffu, mbar_wait(gfull(g), (blk >> 1) & 1))) bad = true;
       // every consumer warp takes the same decision: the flag of this block's
       // parity is written only before this barrier and read only after it
