@@ -142,7 +142,12 @@ pisa_status pisa_block_stats(const void *q, const void *k, const void *v, pisa_d
  * scores, ties going to the lower block index; with sink_idx 0 / -1 the block
  * 0 / N-1 is always kept and the other k_sel-1 are the best of the rest.
  * idx [B,H,N,k_sel] int32, each row ascending.  cov may be NULL when
- * cov_weight == 0.  `workspace`: pisa_select_workspace_bytes(B,H,N) bytes. */
+ * cov_weight == 0.  `workspace`: pisa_select_workspace_bytes(B,H,N) bytes.
+ * The scores are formed to float32 accuracy: with a float32 FMA chain over d
+ * for N <= 512, and on the tensor cores from three-part bf16 splits of qbar
+ * and kbar (six cross products) for longer rows.  Two blocks whose scores
+ * agree to float32 rounding may therefore be ordered differently from an
+ * fp64 evaluation; exact float32 ties go to the lower index. */
 pisa_status pisa_select(const float *qbar, const float *kbar, const float *cov,
                         float cov_weight, float scale, int B, int H, int N, int d,
                         double density, int sink_idx, int32_t *idx,
