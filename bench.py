@@ -50,7 +50,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 K3_TRAFFIC = {
     # H=4 ncu capture (dram read 240.4 MB + write 61.1 MB per launch) scaled by
     # 10 to the 40 heads; profiles/piecewise_attention_tc_wan_h4.md
-    "a0503d7f1a2e": {"wan": 3.016e9},
+    "09e7bbbd5e4f": {"wan": 3.016e9},
 }
 
 
@@ -93,13 +93,21 @@ def select_roofline(wl, N, k_sel, ms, peaks):
 
 
 def _k3_source_hash():
-    # the files the fused kernel's own code comes from (the kernel, the
-    # in-kernel selection's top-k, the tcgen05 / TMA primitives)
+    # the fused kernel's own code: its file, the top-k row routine it takes from
+    # k2_select.cuh for the in-kernel selection (float_key .. topk_row), and
+    # the tcgen05 / TMA primitives
+    d = os.path.join(ROOT, "block_sparse_attention_stats_b200", "csrc")
     h = hashlib.sha1()
     for n in ("k3_attention_tc.cuh", "k2_select.cuh", "sm100_primitives.cuh"):
-        fn = os.path.join(ROOT, "block_sparse_attention_stats_b200", "csrc", n)
-        if os.path.exists(fn):
-            h.update(open(fn, "rb").read())
+        fn = os.path.join(d, n)
+        if not os.path.exists(fn):
+            continue
+        txt = open(fn).read()
+        if n == "k2_select.cuh":
+            a = txt.find("// Order-preserving map float32 -> uint32")
+            b = txt.find("// One warp per query block over the score matrix")
+            txt = txt[a:b] if 0 <= a < b else txt
+        h.update(txt.encode())
     return h.hexdigest()[:12]
 
 
