@@ -547,6 +547,228 @@ __global__ void __launch_bounds__(32 * 10, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Streamed pass 3 (bf16, d = 128): cov_j = ||G_j - kbar_j^T vsum_j - hbar||_F
+// with G_j = K_j^T V_j formed again on tcgen05.  Same CTA ranges as pass 1.
+// Warp 0 streams K and V tiles through a four-stage TMA ring, warp 1 issues
+// the K^T V products into two TMEM buffers, warps 2-9 read each block's G
+// back (thread = row arow of G, half ch of its columns), subtract
+// kbar_j[arow] vsum_j and the thread's 64 entries of hbar (kept in registers
+// per head), and sum the squares; the 256 partial sums meet in a fixed order
+// (warp shuffles, then the eight warps in index order), so cov is bitwise
+// reproducible.
+// ---------------------------------------------------------------------------
+template <int D> struct CovTmaCfg {
+  static constexpr int kThreads = 32 * 10;
+  static constexpr int kTileBytes = kBlk * D * 2;           // one 64-token tile of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;        // K, V
+  static constexpr int kBoxBytes = kBlk * 128;              // 64 tokens x 64 columns
+  static constexpr int kOffRed = kStatsStages * kStageBytes;   // [2][8] warp sums
+  static constexpr int kOffBar = kOffRed + 2 * 8 * 4;
+  // bars: full[4], empty[4], gfull[2], gempty[2], teardown
+  static constexpr int kNumBars = 2 * kStatsStages + 5;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kOffMisc = kOffTmemSlot + 16;
+  static constexpr int kSmem = kOffMisc + 16 + 1024;        // + alignment slack
+  static constexpr uint32_t kTmemCols = 2 * D;              // two G buffers
+};
+
+template <int D>
+__global__ void __launch_bounds__(32 * 10, 1)
+    cov_pass_tma_kernel(const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, int L, int N, int sub, int BH,
+                        const float *__restrict__ kbar, const float *__restrict__ vsum,
+                        const float *__restrict__ hbar, float *__restrict__ cov) {
+  using T = CovTmaCfg<D>;
+  using namespace sm100;
+  static_assert(D == 128, "the consumer layout assumes 128 rows of G");
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  unsigned char *smem = smem_raw + (sbase - raw);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + T::kOffMisc);
+  volatile int *cflag = abort_flag + 1;   // [2]: consumers' abort, by block parity
+  float *red = reinterpret_cast<float *>(smem + T::kOffRed);
+  auto bar = [&](int i) -> uint32_t { return sbase + T::kOffBar + 8 * i; };
+  auto full = [&](int s) { return bar(s); };
+  auto empty = [&](int s) { return bar(kStatsStages + s); };
+  auto gfull = [&](int g) { return bar(2 * kStatsStages + g); };
+  auto gempty = [&](int g) { return bar(2 * kStatsStages + 2 + g); };
+  const uint32_t teardown = bar(2 * kStatsStages + 4);
+
+  const long long total = (long long)BH * N;
+  const int nc = gridDim.x, c = blockIdx.x;
+  const long long g0 = stats_first_block(c, total, nc), g1 = stats_first_block(c + 1, total, nc);
+  const int ntile = ceil_div(L, kBlk);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
+  auto tiles_of = [&](long long G) -> int {
+    const int j = (int)(G % N);
+    return min(sub, ntile - j * sub);
+  };
+
+  if (warp == 1) {
+    tmem_alloc(sbase + T::kOffTmemSlot, T::kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStatsStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);         // the MMA commit
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(gfull(g), 1);
+      mbar_init(gempty(g), 8);
+    }
+    mbar_init(teardown, 1);
+    fence_mbar_init();
+    abort_flag[0] = 0;
+    abort_flag[1] = 0;
+    abort_flag[2] = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + T::kOffTmemSlot);
+
+  if (warp == 0) {
+    // ======================= TMA producer =====================================
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int t = 0;
+      bool ok = true;
+      for (long long G = g0; ok && G < g1; ++G) {
+        const int bh = (int)(G / N), j = (int)(G % N);
+        const int nt = tiles_of(G);
+        for (int s = 0; s < nt; ++s, ++t) {
+          const int slot = t % kStatsStages;
+          if (t >= kStatsStages && !mbar_wait(empty(slot), ((t / kStatsStages) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          if (*abort_flag) { ok = false; break; }
+          const uint32_t dst = sbase + slot * T::kStageBytes;
+          const int row = (j * sub + s) * kBlk;
+          mbar_expect_tx(full(slot), T::kStageBytes);
+#pragma unroll
+          for (int b = 0; b < D / 64; ++b) {
+            tma_load_3d(dst + b * T::kBoxBytes, &tm_k, full(slot), 64 * b, row, bh);
+            tma_load_3d(dst + T::kTileBytes + b * T::kBoxBytes, &tm_v, full(slot), 64 * b, row,
+                        bh);
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        for (int u = (t >= kStatsStages ? t - kStatsStages : 0); u < t; ++u)
+          mbar_wait(full(u % kStatsStages), (u / kStatsStages) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================================
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16_f32(128, D, 1, 1);
+      int t = 0, blk = 0;
+      bool ok = true;
+      for (long long G = g0; ok && G < g1; ++G, ++blk) {
+        const int g = blk & 1;
+        if (blk >= 2 && !mbar_wait(gempty(g), ((blk >> 1) - 1) & 1)) { ok = false; break; }
+        const int nt = tiles_of(G);
+        for (int s = 0; s < nt; ++s, ++t) {
+          const int slot = t % kStatsStages;
+          if (!mbar_wait(full(slot), (t / kStatsStages) & 1)) { ok = false; break; }
+          if (*abort_flag) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kst = sbase + slot * T::kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBlk / 16; ++kk)
+            mma_ss(tmem + D * g, smem_desc_sw128(kst + kk * 2048, T::kBoxBytes, 1024),
+                   smem_desc_sw128(kst + T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kId,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(empty(slot));
+        }
+        if (ok) tc_commit(gfull(g));
+      }
+      if (!ok) *abort_flag = 1;
+      tc_commit(teardown);
+      mbar_wait(teardown, 0);
+    }
+    __syncwarp();
+  } else {
+    // ======================= consumers ========================================
+    const int cw = warp - 2, ctid = tid - 64;
+    const int sp = warp & 3, ch = cw >> 2;      // TMEM sub-partition, column half of G
+    const int arow = sp * 32 + lane;            // row of G (a key dimension)
+    constexpr int kH = D / 2;                   // columns of G per thread
+    float hb[kH];
+    int cur_bh = -1;
+    int blk = 0;
+    bool ok = true;
+    for (long long G = g0; ok && G < g1; ++G, ++blk) {
+      const int bh = (int)(G / N), g = blk & 1;
+      if (bh != cur_bh) {
+        const float4 *h4 =
+            reinterpret_cast<const float4 *>(hbar + ((size_t)bh * D + arow) * D + ch * kH);
+#pragma unroll
+        for (int i = 0; i < kH / 4; ++i) {
+          const float4 x = h4[i];
+          hb[4 * i] = x.x;
+          hb[4 * i + 1] = x.y;
+          hb[4 * i + 2] = x.z;
+          hb[4 * i + 3] = x.w;
+        }
+        cur_bh = bh;
+      }
+      const float ka = kbar[(size_t)G * D + arow];
+      const float *vs = vsum + (size_t)G * D + ch * kH;
+      bool bad = !__all_sync(0xffffffffu, mbar_wait(gfull(g), (blk >> 1) & 1));
+      float ss = 0.f;
+      if (!bad) {
+        tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(sp * 32) << 16) + D * g + ch * kH;
+#pragma unroll
+        for (int q = 0; q < kH / 32; ++q) {
+          uint32_t r[32];
+          tmem_ld_x32(taddr + 32 * q, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float e = __uint_as_float(r[i]) - ka * vs[32 * q + i] - hb[32 * q + i];
+            ss = fmaf(e, e, ss);
+          }
+        }
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(gempty(g));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) red[g * 8 + cw] = ss;
+      // every consumer warp takes the same decision: the flag of this block's
+      // parity is written only before this barrier and read only after it
+      if (bad) {
+        cflag[blk & 1] = 1;
+        *abort_flag = 1;
+      }
+      stats_consumer_barrier();
+      if (cflag[blk & 1]) { ok = false; break; }
+      if (ctid == 0) {
+        const float *rg = red + g * 8;
+        const float tot = ((rg[0] + rg[1]) + (rg[2] + rg[3])) + ((rg[4] + rg[5]) + (rg[6] + rg[7]));
+        cov[G] = sqrtf(tot);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, T::kTmemCols);
+  }
+}
+
 // pass 2 of the streamed pass: hbar = (1/N) sum of the head's segment partials,
 // in segment order.
 __global__ void hbar_reduce_seg_kernel(const float *__restrict__ partial, int maxseg, int DD,

@@ -203,6 +203,15 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
       hbar_reduce_seg_kernel<<<dim3(ceil_div(D * D, 256), BH), 256, 0, st>>>(
           partial, maxseg, D * D, N, BH, nc, hbar);
       PISA_TRY(check_launch());
+      if (want_cov) {
+        // pass 3 on the same ranges: K and V again, G_j on tcgen05
+        PISA_CUDA(cudaFuncSetAttribute(cov_pass_tma_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       CovTmaCfg<D>::kSmem));
+        cov_pass_tma_kernel<D><<<nc, CovTmaCfg<D>::kThreads, CovTmaCfg<D>::kSmem, st>>>(
+            mk, mv, L, N, sub, BH, kbar, vsum, hbar, cov);
+        PISA_TRY(check_launch());
+      }
     }
   }
   if (streamed) {
@@ -231,7 +240,7 @@ static pisa_status launch_stats(const void *q, const void *k, const void *v, pis
                                                                         N, hbar);
     PISA_TRY(check_launch());
   }
-  if (want_cov) {
+  if (want_cov && !streamed) {
     if (dt == PISA_BF16) {
       const int smem = 2 * 2 * StatsMmaCfg<D>::kTileBytes + 32 * (int)sizeof(float);
       PISA_CUDA(cudaFuncSetAttribute(cov_pass_bf16_kernel<D>,
