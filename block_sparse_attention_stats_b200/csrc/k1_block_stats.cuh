@@ -781,6 +781,8 @@ __global__ void hbar_reduce_seg_kernel(const float *__restrict__ partial, int ma
   const int c1 = stats_cta_of((long long)(bh + 1) * N - 1, total, nc);
   const float *p = partial + (size_t)bh * maxseg * DD + e;
   float s = 0.f;
+  // the loads of four segments go out together; the sum stays in segment order
+#pragma unroll 4
   for (int seg = 0; seg <= c1 - c0; ++seg) s += p[(size_t)seg * DD];
   hbar[(size_t)bh * DD + e] = s / (float)N;
 }
