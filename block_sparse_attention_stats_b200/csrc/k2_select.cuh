@@ -412,7 +412,7 @@ __host__ __device__ inline int select_fused_smem(int N, int D) {
   return kSelRows * N * 4 + (stage > hist ? stage : hist);
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1)
+__global__ void __launch_bounds__(kSelThreads, 2)
     select_fused_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar,
                         const float *__restrict__ cov, float cov_weight, float scale, int N,
                         int D, int k_sel, int sink, int32_t *__restrict__ idx) {
@@ -431,34 +431,56 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     const int r = e % kSelRows, dd = e / kSelRows;
     qT[e] = i0 + r < N ? qb[(size_t)(i0 + r) * D + dd] : 0.f;
   }
+  // the k-bar chunk of the next head-dimension step is fetched into registers
+  // while the current one is used
+  constexpr int kPf = (kSelCols * kSelDims / 4 + kSelThreads - 1) / kSelThreads;
+  float4 pf[kPf];
+  auto fetch = [&](int c0, int e0) {
+#pragma unroll
+    for (int h = 0; h < kPf; ++h) {
+      const int f = tid + kSelThreads * h;
+      const int c = f % kSelCols, e4 = (f / kSelCols) * 4, j = c0 + c;
+      pf[h] = (f < kSelCols * kSelDims / 4 && j < N)
+                  ? *reinterpret_cast<const float4 *>(kb + (size_t)j * D + e0 + e4)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  // warp w computes columns 128 (w & 1) .. +127 of a chunk: none of them may
+  // exist on short rows
+  const int wcol = 128 * ((tid >> 5) & 1);
   for (int c0 = 0; c0 < N; c0 += kSelCols) {
     float acc[4][4];
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
       for (int x = 0; x < 4; ++x) acc[r][x] = 0.f;
+    fetch(c0, 0);
     for (int e0 = 0; e0 < D; e0 += kSelDims) {
       __syncthreads();   // qT written / the previous chunk consumed
-      for (int f = tid; f < kSelCols * kSelDims / 4; f += kSelThreads) {
-        const int c = f % kSelCols, e4 = (f / kSelCols) * 4;
-        const int j = c0 + c;
-        const float4 v = j < N ? *reinterpret_cast<const float4 *>(kb + (size_t)j * D + e0 + e4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-        kT[(e4 + 0) * kSelCols + c] = v.x;
-        kT[(e4 + 1) * kSelCols + c] = v.y;
-        kT[(e4 + 2) * kSelCols + c] = v.z;
-        kT[(e4 + 3) * kSelCols + c] = v.w;
+#pragma unroll
+      for (int h = 0; h < kPf; ++h) {
+        const int f = tid + kSelThreads * h;
+        if (f < kSelCols * kSelDims / 4) {
+          const int c = f % kSelCols, e4 = (f / kSelCols) * 4;
+          kT[(e4 + 0) * kSelCols + c] = pf[h].x;
+          kT[(e4 + 1) * kSelCols + c] = pf[h].y;
+          kT[(e4 + 2) * kSelCols + c] = pf[h].z;
+          kT[(e4 + 3) * kSelCols + c] = pf[h].w;
+        }
       }
       __syncthreads();
+      if (e0 + kSelDims < D) fetch(c0, e0 + kSelDims);
+      if (c0 + wcol < N) {
 #pragma unroll 8
-      for (int e = 0; e < kSelDims; ++e) {
-        const float4 a = *reinterpret_cast<const float4 *>(qT + (e0 + e) * kSelRows + 4 * rg);
-        const float4 b = *reinterpret_cast<const float4 *>(kT + e * kSelCols + 4 * cg);
-        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+        for (int e = 0; e < kSelDims; ++e) {
+          const float4 a = *reinterpret_cast<const float4 *>(qT + (e0 + e) * kSelRows + 4 * rg);
+          const float4 b = *reinterpret_cast<const float4 *>(kT + e * kSelCols + 4 * cg);
+          const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+          for (int r = 0; r < 4; ++r)
 #pragma unroll
-          for (int x = 0; x < 4; ++x) acc[r][x] = fmaf(av[r], bv[x], acc[r][x]);
+            for (int x = 0; x < 4; ++x) acc[r][x] = fmaf(av[r], bv[x], acc[r][x]);
+        }
       }
     }
 #pragma unroll
