@@ -157,12 +157,10 @@ __global__ void __launch_bounds__(kTopkThreads)
 // The same selection with one histogram pass instead of four radix passes.
 // Each warp copies its row into shared memory, then finds the k-th largest key
 // T and the number of keys equal to T to keep:
-//  1. lo / hi = the smallest / largest of 64 scores sampled at even strides
-//     from the staged row; bin(x) = clamp(int((x - lo) * (256 / (hi - lo))),
-//     0, 255).  Every step of bin() is a monotone float32 operation (the
-//     conversion saturates, so infinite scores land in the end bins), so
-//     x >= y implies bin(x) >= bin(y): the bins order the keys whatever the
-//     range; the sample only sets how evenly a row spreads over them.
+//  1. lo / hi = the smallest / largest candidate score; bin(x) =
+//     min(255, int((x - lo) * (256 / (hi - lo)))).  Every step of bin() is a
+//     monotone float32 operation, so x >= y implies bin(x) >= bin(y): the bins
+//     order the keys.
 //  2. One histogram of the candidates' bins; scanning from the top bin gives
 //     the bin b* that holds the `need`-th largest key and how many keys of b*
 //     are still to be taken.
@@ -173,9 +171,9 @@ __global__ void __launch_bounds__(kTopkThreads)
 // Comparing floats gives the key order (only -0 and +0 share a key, and they
 // compare equal).  Then the same compaction as topk_row keeps the sink, every
 // score > T and the lowest-index scores equal to T.  Rows where the bins do
-// not apply (a degenerate sample, a NaN score, more than kBinCand scores in
-// b*) go through topk_row on the staged row, so the result is the same set in
-// every case.
+// not apply (all scores equal, a non-finite score, more than kBinCand scores
+// in b*) go through topk_row on the staged row, so the result is the same set
+// in every case.
 // ---------------------------------------------------------------------------
 constexpr int kBinCand = 64;
 
@@ -198,64 +196,60 @@ __global__ void __launch_bounds__(kTopkThreads)
   int32_t *out = idx + row * k_sel;
   const int need = k_sel - (sink >= 0 ? 1 : 0);
   const int candidates = N - (sink >= 0 ? 1 : 0);
+  // stage the row (16-byte loads), and 1. the range of the candidates on the
+  // way; a NaN or infinite score sends the row to topk_row
+  const float inf = __int_as_float(0x7f800000);
+  float lo = inf, hi = -inf;
+  bool bad = false;
+#pragma unroll 2
+  for (int c = lane; c < ld / 4; c += 32) {
+    const float4 x4 = __ldcs(reinterpret_cast<const float4 *>(sc) + c);
+    *reinterpret_cast<float4 *>(srow + 4 * c) = x4;
+    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * c + e;
+      if (j < N && j != sink) {
+        bad |= !(fabsf(xs[e]) < inf);
+        lo = fminf(lo, xs[e]);
+        hi = fmaxf(hi, xs[e]);
+      }
+    }
+  }
+  __syncwarp();
   if (need <= 0 || need >= candidates) {
-    topk_row(sc, N, k_sel, sink, hist, out, lane);
+    topk_row(srow, N, k_sel, sink, hist, out, lane);
     return;
   }
-  // stage the row (16-byte loads only, so many are in flight)
-#pragma unroll 4
-  for (int c = lane; c < ld / 4; c += 32)
-    *reinterpret_cast<float4 *>(srow + 4 * c) = __ldcs(reinterpret_cast<const float4 *>(sc) + c);
-  __syncwarp();
-  // 1. the bin range from a strided sample of 64 scores (two per lane).  Any
-  //    range gives monotone bins once they are clamped to 0 .. 255 (scores
-  //    outside it fall into the end bins); the sample only decides how evenly
-  //    the row spreads over the bins.  A degenerate sample sends the row to
-  //    topk_row.
-  const float inf = __int_as_float(0x7f800000);
-  const float s0 = srow[(int)(((long long)lane * N) >> 5)];
-  const float s1 = srow[(int)(((long long)(2 * lane + 1) * N) >> 6)];
-  float lo = fminf(s0, s1), hi = fmaxf(s0, s1);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
     hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
   const float span = hi - lo, w = 256.f / span;
-  if (!(span > 0.f && span < inf && w < inf)) {
+  if (__any_sync(0xffffffffu, bad) || !(span > 0.f && span < inf && w < inf)) {
     topk_row(srow, N, k_sel, sink, hist, out, lane);
     return;
   }
-  auto bin_of = [&](float x) { return min(max((int)((x - lo) * w), 0), 255); };
-  // 2. histogram and the boundary bin; a NaN score (unordered) sends the row
-  //    to topk_row
+  auto bin_of = [&](float x) { return min((int)((x - lo) * w), 255); };
+  // 2. histogram and the boundary bin
 #pragma unroll
   for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0u;
   __syncwarp();
-  bool bad = false;
 #pragma unroll 2
   for (int c = lane; c < ld / 4; c += 32) {
     const float4 x4 = *reinterpret_cast<const float4 *>(srow + 4 * c);
     const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
     if (4 * c + 3 < N && (unsigned)(sink - 4 * c) > 3u) {
-      bad |= (xs[0] != xs[0]) | (xs[1] != xs[1]) | (xs[2] != xs[2]) | (xs[3] != xs[3]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) atomicAdd(&hist[bin_of(xs[e])], 1u);
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = 4 * c + e;
-        if (j < N && j != sink) {
-          bad |= xs[e] != xs[e];
-          atomicAdd(&hist[bin_of(xs[e])], 1u);
-        }
+        if (j < N && j != sink) atomicAdd(&hist[bin_of(xs[e])], 1u);
       }
     }
-  }
-  __syncwarp();
-  if (__any_sync(0xffffffffu, bad)) {
-    topk_row(srow, N, k_sel, sink, hist, out, lane);
-    return;
   }
   __syncwarp();
   unsigned own = 0;                      // lane l owns bins 255-8l .. 248-8l
