@@ -299,8 +299,11 @@ template <int D> struct StatsTmaCfg {
   static constexpr uint32_t kTmemCols = 2 * D < 32 ? 32 : 2 * D;   // two G buffers
 };
 
-__device__ __forceinline__ void stats_consumer_barrier() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
+// named barrier 1 over the consumer warps of one kernel (every warp from
+// index 2 up): kCount = 32 x that kernel's consumer warps
+template <int kCount> __device__ __forceinline__ void stats_consumer_barrier() {
+  static_assert(kCount % 32 == 0, "whole warps");
+  asm volatile("bar.sync 1, %0;" ::"n"(kCount) : "memory");
 }
 
 template <int D>
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(32 * 10, 1)
         cflag[blk & 1] = 1;
         *abort_flag = 1;
       }
-      stats_consumer_barrier();
+      stats_consumer_barrier<T::kThreads - 64>();
       if (cflag[blk & 1]) { ok = false; break; }
       tc_fence_after();
       const float ka = kv[arow];
@@ -752,7 +755,7 @@ __global__ void __launch_bounds__(32 * 10, 1)
         cflag[blk & 1] = 1;
         *abort_flag = 1;
       }
-      stats_consumer_barrier();
+      stats_consumer_barrier<T::kThreads - 64>();
       if (cflag[blk & 1]) { ok = false; break; }
       if (ctid == 0) {
         const float *rg = red + g * 8;
