@@ -23,13 +23,18 @@
 //   warps 2-9   two warpgroups of 4 warps; warpgroup g takes the tiles with
 //               u & 1 == g (buffer g), one thread per query row (TMEM lane):
 //               P and dP from TMEM, Delta partial sums (Delta sweep) or dS
-//               written to a dS buffer as bf16 (dq sweep); the two Delta
-//               partials are combined through shared memory between sweeps
-//               (with Delta given, each thread reads its row's value);
-//               the epilogue scales dQ by s and stores it (half the columns
-//               each).
+//               written as bf16 over the dP columns it was formed from (dq
+//               sweep); the two Delta partials are combined through shared
+//               memory between sweeps (with Delta given, each thread reads its
+//               row's value); the epilogue scales dQ by s and stores it (half
+//               the columns each).  Before the loop warpgroup 0 copies Q and
+//               warpgroup 1 copies dout into tensor memory.
 // TMEM columns: dQ [0, D); buffer b: S [D + 128 b, D + 128 b + 64), dP the next
-// 64; dS buffers (packed bf16) [D + 256 + 32 c, D + 256 + 32 c + 32).
+// 64 (dS, packed bf16, over its first 32); dout [D + 256, D + 256 + D / 2) and
+// Q [D + 320, D + 320 + D / 2) as packed bf16 pairs, the A operands of the dP
+// and S products.  dP_u + 2 rewrites the dS of tile u only after dQ_u has read
+// it: warp 10 issues both, in that order, and one thread's tcgen05 products
+// run in issue order; the commit that signals dP_u also covers dQ_u - 2.
 // Every mbarrier wait is bounded; on a timeout the CTA records the error,
 // stops issuing, drains its copies and MMAs, frees TMEM and exits.
 #pragma once
@@ -59,10 +64,11 @@ template <int D> struct DqTcCfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColDQ = 0;
   static constexpr uint32_t kColBuf = D;                        // + 128 b
-  static constexpr uint32_t kColDS = D + 256;                   // + 32 b: packed bf16 dS
-  // Q as packed bf16 pairs (D / 2 columns), the A operand of the S products:
-  // read from tensor memory, an N = 64 product needs only its 2 KB of K tile
-  // from shared memory instead of 6 KB, which bounds it at ~52 pipe cycles
+  // dout and Q as packed bf16 pairs (D / 2 columns each), the A operands of
+  // the dP and S products: read from tensor memory, an N = 64 product needs
+  // only its 2 KB of V or K tile from shared memory instead of 6 KB, which
+  // bounds it at ~52 pipe cycles
+  static constexpr uint32_t kColDO = D + 256;
   static constexpr uint32_t kColQ = D + 320;
   static constexpr int kBarQ = 0;
   static constexpr int kBarKFull = 1;                           // + slot
@@ -71,12 +77,13 @@ template <int D> struct DqTcCfg {
   static constexpr int kBarVEmpty = kBarVFull + kStages;
   static constexpr int kBarSFull = kBarVEmpty + kStages;        // + buffer
   static constexpr int kBarPFull = kBarSFull + 2;               // + buffer
-  static constexpr int kBarDsFree = kBarPFull + 2;             // + dS buffer
-  static constexpr int kBarDelta = kBarDsFree + 2;
+  static constexpr int kBarDelta = kBarPFull + 2;
   static constexpr int kBarFinal = kBarDelta + 1;
   static constexpr int kBarTeardown = kBarFinal + 1;
   static constexpr int kBarQT = kBarTeardown + 1;                // Q copied into TMEM
-  static_assert(kBarQT < kNumBars, "barrier slots");
+  static constexpr int kBarDOT = kBarQT + 1;                     // dout copied into TMEM
+  static_assert(kBarDOT < kNumBars, "barrier slots");
+  static_assert(kColDO + D / 2 <= kColQ, "tensor memory columns");
   static_assert(kColQ + D / 2 <= kTmemCols, "tensor memory columns");
 
   // N 64-token tiles, Nc blocks (= centroids)
@@ -157,12 +164,12 @@ __global__ void __launch_bounds__(352, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(C::kBarSFull + b), 2);       // S from warp 1, dP from warp 10
       mbar_init(bar(C::kBarPFull + b), 128);
-      mbar_init(bar(C::kBarDsFree + b), 1);
     }
     mbar_init(bar(C::kBarDelta), 256);
     mbar_init(bar(C::kBarFinal), 1);
     mbar_init(bar(C::kBarTeardown), 2);
     mbar_init(bar(C::kBarQT), 4);
+    mbar_init(bar(C::kBarDOT), 4);
     fence_mbar_init();
     misc[1] = 0;
   }
@@ -311,8 +318,8 @@ __global__ void __launch_bounds__(352, 1)
     // One warp issues tcgen05.mma at a bounded rate, so the products are
     // split: warp 1 issues S_u = Q K_u^T; warp 10 issues dP_u = dout V_u^T and,
     // in the second sweep, dQ += dS_u K_u.  Buffer u & 1 is rewritten by S_u
-    // once the dS warpgroup has read tile u - 2 from it (PFull); dS lives in
-    // its own pair of buffers, released by the dQ products (DsFree).
+    // once the dS warpgroup has read tile u - 2 from it (PFull); its dP half,
+    // which then holds dS_u - 2, by dP_u after dQ_u - 2 (warp 10's order).
     constexpr uint32_t kIdQK = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t kIdDQ = idesc_bf16_f32(128, D, 0, 1);
     const bool s_warp = warp == 1;
@@ -320,12 +327,8 @@ __global__ void __launch_bounds__(352, 1)
     tc_fence_after();
     // descriptors are built once per buffer; a K step adds its byte offset / 16
     // to the start-address field (which cannot carry below 256 KB)
-    const uint64_t dod0 = smem_desc_sw128(sbase + C::kOffDO, 16, 1024);
-    if (s_warp && ok) ok = uwait(bar(C::kBarQT), 0);   // Q in tensor memory
+    if (ok) ok = uwait(bar(s_warp ? C::kBarQT : C::kBarDOT), 0);   // Q / dout in tensor memory
     tc_fence_after();
-    auto a_step = [](int k) -> uint64_t {
-      return (uint64_t)(((k >> 2) * C::kBoxQBytes + (k & 3) * 32) >> 4);
-    };
     auto b_step = [](int k) -> uint64_t {
       return (uint64_t)(((k >> 2) * C::kBoxKBytes + (k & 3) * 32) >> 4);
     };
@@ -336,15 +339,13 @@ __global__ void __launch_bounds__(352, 1)
       if (!uwait(bar(C::kBarPFull + b), (w >> 1) & 1)) return false;
       if (w >= T1) {
         tc_fence_after();
-        const int db = (w - T1) & 1;
         const uint64_t kd = smem_desc_sw128(sbase + C::kOffK + sl * C::kTileBytes, C::kBoxKBytes, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + C::kColDQ, tmem + C::kColDS + 32 * db + kk * 8,
+            mma_ts(tmem + C::kColDQ, tmem + C::kColBuf + 128 * b + 64 + kk * 8,
                    kd + (uint64_t)((kk * 2048) >> 4), kIdDQ, (w > T1 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::kBarKEmpty + sl));
-          tc_commit(bar(C::kBarDsFree + db));
         }
         __syncwarp();
       }
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(352, 1)
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b + 64, dod0 + a_step(k), vd + b_step(k), kIdQK,
+            mma_ts(tmem + C::kColBuf + 128 * b + 64, tmem + C::kColDO + 8 * k, vd + b_step(k), kIdQK,
                    k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarSFull + b));
           tc_commit(bar(C::kBarVEmpty + sl));
@@ -416,15 +417,18 @@ __global__ void __launch_bounds__(352, 1)
     auto warp_wait = [&](uint32_t b_addr, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b_addr, parity));
     };
-    if (g == 0) {
-      // this thread's query row of Q, from the 128-byte-swizzled TMA boxes
-      // (16-byte chunk c of row r sits at chunk c ^ (r & 7)) into tensor
-      // memory as packed bf16 pairs; every warp arrives, even after a timeout
+    {
+      // this thread's query row of Q (warpgroup 0) or dout (warpgroup 1), from
+      // the 128-byte-swizzled TMA boxes (16-byte chunk c of row r sits at
+      // chunk c ^ (r & 7)) into tensor memory as packed bf16 pairs; every warp
+      // arrives, even after a timeout
+      const int src = g == 0 ? C::kOffQ : C::kOffDO;
+      const uint32_t dst = lane_addr + (g == 0 ? C::kColQ : C::kColDO);
       if (warp_wait(bar(C::kBarQ), 0)) {
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
           uint32_t w[32];
-          const unsigned char *box = smem + C::kOffQ + h * C::kBoxQBytes + row * 128;
+          const unsigned char *box = smem + src + h * C::kBoxQBytes + row * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 v = *reinterpret_cast<const uint4 *>(box + ((c ^ (row & 7)) << 4));
@@ -433,7 +437,7 @@ __global__ void __launch_bounds__(352, 1)
             w[4 * c + 2] = v.z;
             w[4 * c + 3] = v.w;
           }
-          tmem_st_x32(lane_addr + C::kColQ + 32 * h, w);
+          tmem_st_x32(dst + 32 * h, w);
         }
         tmem_wait_st();
       } else {
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::kBarQT));
+      if (lane == 0) mbar_arrive(bar(g == 0 ? C::kBarQT : C::kBarDOT));
     }
     // combine the two warpgroups' Delta partial sums (once, before the first
     // second-sweep tile of this warpgroup, or after its loop)
@@ -469,14 +473,10 @@ __global__ void __launch_bounds__(352, 1)
       tc_fence_after();
       const int e = tiles[second ? u - T1 : u];
       const bool centroid = e < 0;
-      // dS of second-sweep tile u goes to dS buffer (u - T1) & 1, free once the
-      // dQ product of tile u - 2 has completed
-      const int r2 = u - T1;
-      const uint32_t ds_addr = lane_addr + C::kColDS + 32 * (r2 & 1);
-      if (second && r2 >= 2 && !warp_wait(bar(C::kBarDsFree + (r2 & 1)), ((r2 - 2) >> 1) & 1)) {
-        ok = false;
-        break;
-      }
+      // dS of second-sweep tile u goes over the first 32 dP columns of its
+      // buffer (read above into registers); dQ_u - 2 has read the dS there
+      // before dP_u completed (SFull covers it)
+      const uint32_t ds_addr = dp_addr;
       uint64_t keep = 0ull;
       float w_full = 1.f, w_last = 0.f;
       int last_col = -1;
