@@ -402,6 +402,30 @@ def oracle_sample(wl, n_heads: int, n_blocks: int, seed: int = 7):
 # arms
 # ----------------------------------------------------------------------------
 
+def gpu_local_cpus(dev) -> set | None:
+    """The CPUs NVML reports as local to this GPU, within the process's allowed set.
+
+    Pinned host buffers allocated from one of them sit on the GPU's NUMA node.
+    None when NVML or the PCI ids are unavailable or the sets do not meet.
+    """
+    try:
+        import pynvml
+        p = torch.cuda.get_device_properties(dev)
+        pynvml.nvmlInit()
+        try:
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(
+                f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0")
+            words = (os.cpu_count() + 63) // 64
+            masks = pynvml.nvmlDeviceGetCpuAffinity(h, words)
+        finally:
+            pynvml.nvmlShutdown()
+        cpus = {64 * i + b for i, m in enumerate(masks) for b in range(64) if (int(m) >> b) & 1}
+        cpus &= os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
 def max_over_ranks(values, world: int, device="cpu"):
     """Element-wise maximum of per-rank timings (ms) over all ranks (the slowest
     rank defines the step time); a no-op with one rank."""
@@ -708,6 +732,13 @@ def run_pisa(args, wl):
     # ---- e2e: public API with pinned host buffers ------------------------------
     e2e = None
     if not args.no_e2e:
+        # the pinned buffers are allocated (and their pages placed) from CPUs on
+        # the GPU's NUMA node when NVML names them; the thread's affinity is
+        # restored afterwards
+        cpus0 = os.sched_getaffinity(0)
+        local = None if args.no_numa_pin else gpu_local_cpus(dev)
+        if local and local != cpus0:
+            os.sched_setaffinity(0, local)
         hq = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
         hk = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
         hv = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
@@ -761,7 +792,10 @@ def run_pisa(args, wl):
         t_e2e = a.elapsed_time(b2) / e2e_steps
         nbytes = Q.numel() * Q.element_size()
         e2e = {"t_ms": t_e2e, "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
-               "chunks": nchunks}
+               "chunks": nchunks,
+               "host_cpus": (f"{len(local)} GPU-local CPUs of {len(cpus0)}" if local and local != cpus0
+                             else f"all {len(cpus0)} allowed CPUs")}
+        os.sched_setaffinity(0, cpus0)
         # sanity: the chunked result agrees with one call over all heads (the
         # statistics' reduction order depends on the batch, so not bit for bit)
         ref = P.pisa_attention(Q, K, V, wl.density, wl.block_size, wl.sink_idx, wl.mode)
@@ -852,7 +886,8 @@ def run_pisa(args, wl):
                        "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
                        "api": "pisa_attention (C ABI) from pinned host buffers, on "
                               f"{e2e['chunks']} head chunks with H2D, compute and D2H "
-                              "overlapped on three streams"}
+                              "overlapped on three streams",
+                       "pinned_from": e2e["host_cpus"]}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         big = wl.L > 20000
         full, spent, desc = oracle_sample(wl, 2 if big else wl.H,
@@ -877,6 +912,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-numa-pin", action="store_true",
+                    help="allocate the e2e leg's pinned buffers from any allowed CPU")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip timing the step replayed from a CUDA graph")
     ap.add_argument("--no-backward", action="store_true",
