@@ -68,3 +68,57 @@ def test_block_wise_first_order_reads_every_key():
     wl = WORKLOADS["flux"].with_(B=1, H=3, L=1000, d=64, mode="1st")
     idx = _idx(1, 3, 16, 4, 3)
     assert bench.k3_algorithmic_flops(wl, idx) == 4.0 * 64 * 1000 * 1000 * 3
+
+
+class _FakeNvml:
+    """Stands in for pynvml: one GPU whose local CPUs are given as 64-bit words."""
+
+    def __init__(self, words):
+        self.words = words
+        self.bus_ids = []
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlShutdown(self):
+        pass
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus_id):
+        self.bus_ids.append(bus_id)
+        return object()
+
+    def nvmlDeviceGetCpuAffinity(self, handle, n):
+        return self.words[:n] + [0] * max(0, n - len(self.words))
+
+
+class _Props:
+    pci_domain_id, pci_bus_id, pci_device_id = 0, 0x1B, 0
+
+
+def _local_cpus(monkeypatch, words, allowed, ncpu=128):
+    import sys
+    fake = _FakeNvml(words)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda dev: _Props())
+    monkeypatch.setattr(bench.os, "cpu_count", lambda: ncpu)
+    monkeypatch.setattr(bench.os, "sched_getaffinity", lambda pid: set(allowed))
+    return bench.gpu_local_cpus(0), fake
+
+
+def test_gpu_local_cpus_decodes_the_mask_and_keeps_allowed_cpus(monkeypatch):
+    # CPUs 0-15 and 64-79 are local to the GPU; the process may run on 8-71
+    words = [0xFFFF, 0xFFFF]
+    got, fake = _local_cpus(monkeypatch, words, range(8, 72))
+    assert got == set(range(8, 16)) | set(range(64, 72))
+    assert fake.bus_ids == ["00000000:1B:00.0"]
+
+
+def test_gpu_local_cpus_none_when_the_sets_do_not_meet(monkeypatch):
+    got, _ = _local_cpus(monkeypatch, [0xFF], range(32, 48))
+    assert got is None
+
+
+def test_gpu_local_cpus_none_without_nvml(monkeypatch):
+    import sys
+    monkeypatch.setitem(sys.modules, "pynvml", None)    # import fails
+    assert bench.gpu_local_cpus(0) is None
