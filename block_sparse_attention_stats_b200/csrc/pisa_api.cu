@@ -523,6 +523,73 @@ static pisa_status make_map_f32_rows(CUtensorMap *m, const void *base, uint64_t 
   return PISA_OK;
 }
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (cuCtxGetId: ids are never
+// reused within a process), or 0 when there is none or the driver lacks the call.
+static unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// A second stream of this thread on the current device, with two events, for
+// work of one call that may run beside the work on the caller's stream: it
+// starts after an event recorded on that stream and the caller's stream waits
+// for it before going on, so to the caller everything stays ordered on its
+// stream (graph capture included).  Created once, kept for the process.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  unsigned long long ctx = 0;   // context the handles belong to
+};
+
+static pisa_status side_stream(SideStream **out) {
+  int dev = 0;
+  PISA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) {
+    t_last_error = "side stream: device ordinal " + std::to_string(dev) + " out of range";
+    return PISA_ERR_UNSUPPORTED;
+  }
+  static thread_local SideStream cache[64];
+  SideStream &ss = cache[dev];
+  // after cudaDeviceReset the old handles died with their context: make new ones
+  const unsigned long long ctx = current_context_id();
+  if (ss.s == nullptr || ctx == 0 || ctx != ss.ctx) {
+    int lo = 0, hi = 0;
+    PISA_CUDA(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+    cudaStream_t s = nullptr;
+    PISA_CUDA(cudaStreamCreateWithPriority(&s, cudaStreamNonBlocking, hi));
+    cudaEvent_t f = nullptr, j = nullptr;
+    PISA_CUDA(cudaEventCreateWithFlags(&f, cudaEventDisableTiming));
+    PISA_CUDA(cudaEventCreateWithFlags(&j, cudaEventDisableTiming));
+    ss.s = s;
+    ss.fork = f;
+    ss.join = j;
+    ss.ctx = ctx;
+  }
+  *out = &ss;
+  return PISA_OK;
+}
+
 template <int D>
 static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                               const __nv_bfloat16 *v, const __nv_bfloat16 *dout, const float *lse,
@@ -581,6 +648,34 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                                                           BH, delta);
     PISA_TRY(check_launch());
   }
+  // With Delta given, the centroid gradients, the key-block pairing and the
+  // query-tile lists need nothing from dq: they run on a side stream beside it
+  // (high priority, so their few CTAs are placed as dq's CTAs retire), and the
+  // exact keys' dk, dv wait for both.  With the Delta sweep, dq writes Delta
+  // and everything runs in order on the caller's stream.
+  cudaStream_t ss = st;
+  SideStream *side = nullptr;
+  if (o32) {
+    PISA_TRY(side_stream(&side));
+    PISA_CUDA(cudaEventRecord(side->fork, st));
+    PISA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    ss = side->s;
+  }
+  // on every return from here on, the caller's stream waits for the side
+  // stream's work (so an early error never leaves kernels running on a
+  // workspace the caller may free)
+  struct JoinGuard {
+    SideStream *side;
+    cudaStream_t ss, st;
+    cudaError_t join() {
+      if (!side) return cudaSuccess;
+      cudaError_t e = cudaEventRecord(side->join, ss);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
+      side = nullptr;
+      return e;
+    }
+    ~JoinGuard() { join(); }
+  } guard{side, ss, st};
   bwd_dq_tc_kernel<D><<<dim3(P, BH), DqTcCfg<D>::kThreads, dq_smem, st>>>(
       mq, mdo, mk, mv, mkb, mvb, idx, pairs, k_sel, L, N, bsub, Nc, scale, lse, delta,
       o32 != nullptr, Lpad, dq);
@@ -593,7 +688,7 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
   PISA_CUDA(cudaFuncSetAttribute(bwd_kv_tc_kernel<D, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kvtc_smem));
   bwd_kv_tc_kernel<D, true><<<dim3(ceil_div(Ncpad, 128), BH), KvTcCfg<D>::kThreads, kvtc_smem,
-                              st>>>(
+                              ss>>>(
       mq, mdo, mkb, mvb, mlse, mdel, nullptr, nullptr, 0, nullptr, nullptr, bm, cwords, bsub, Nc,
       L, N, scale, dkbar, dvbar, Ncpad, nullptr, nullptr);
   PISA_TRY(check_launch());
@@ -605,26 +700,27 @@ static pisa_status launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
     uint32_t *bmT = (uint32_t *)(ws + lay.bmT);
     uint16_t *ov = (uint16_t *)(ws + lay.ov);
     kpairs = (int2 *)(ws + lay.kpairs);
-    bitmap_transpose_kernel<<<dim3(cwords, cwords, BH), 32, 0, st>>>(bm, N, cwords, bmT);
+    bitmap_transpose_kernel<<<dim3(cwords, cwords, BH), 32, 0, ss>>>(bm, N, cwords, bmT);
     PISA_TRY(check_launch());
-    pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, st>>>(bmT, N, cwords, ov);
+    pair_overlap_kernel<<<dim3(ceil_div(N, 8), BH), 256, 0, ss>>>(bmT, N, cwords, ov);
     PISA_TRY(check_launch());
     const int staged = N * (kPairWindow * 2 + 1) <= 200 * 1024;
     const int pair_smem = staged ? N * (kPairWindow * 2 + 1) : N;
     if (pair_smem > 48 * 1024)
       PISA_CUDA(cudaFuncSetAttribute(pairing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      pair_smem));
-    pairing_kernel<<<BH, kPairThreads, pair_smem, st>>>(ov, N, staged, kpairs);
+    pairing_kernel<<<BH, kPairThreads, pair_smem, ss>>>(ov, N, staged, kpairs);
     PISA_TRY(check_launch());
   }
-  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, kpairs, 0, counts,
+  kvlist_kernel<<<dim3(P, BH), 32, 0, ss>>>(bm, N, Nc, cwords, bsub, P, kpairs, 0, counts,
                                             offsets, lay.cap, entries);
   PISA_TRY(check_launch());
-  kvlist_scan_kernel<<<BH, 1024, 0, st>>>(counts, P, offsets);
+  kvlist_scan_kernel<<<BH, 1024, 0, ss>>>(counts, P, offsets);
   PISA_TRY(check_launch());
-  kvlist_kernel<<<dim3(P, BH), 32, 0, st>>>(bm, N, Nc, cwords, bsub, P, kpairs, 1, counts,
+  kvlist_kernel<<<dim3(P, BH), 32, 0, ss>>>(bm, N, Nc, cwords, bsub, P, kpairs, 1, counts,
                                             offsets, lay.cap, entries);
   PISA_TRY(check_launch());
+  PISA_CUDA(guard.join());
   bwd_kv_tc_kernel<D, false><<<dim3(P, BH), KvTcCfg<D>::kThreads, kvtc_smem, st>>>(
       mq, mdo, mk, mv, mlse, mdel, counts, offsets, lay.cap, entries, kpairs, bm, cwords, bsub,
       Nc, L, N, scale, dkbar, dvbar, Ncpad, dk, dv);
@@ -650,34 +746,6 @@ std::mutex g_noalloc_mutex;
 // was looked up in (0 = not looked up yet)
 void *g_noalloc_ptr[kMaxDevices] = {nullptr};
 unsigned long long g_noalloc_ctx[kMaxDevices] = {0};
-
-using CtxGetCurrentFn = CUresult (*)(CUcontext *);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
-
-// Unique id of the calling thread's current context (cuCtxGetId: ids are never
-// reused within a process), or 0 when there is none or the driver lacks the call.
-unsigned long long current_context_id() {
-  static CtxGetCurrentFn get_current = nullptr;
-  static CtxGetIdFn get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<CtxGetIdFn>(p);
-  });
-  if (!get_current || !get_id) return 0;
-  CUcontext ctx = nullptr;
-  unsigned long long id = 0;
-  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
-  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
-  return id;
-}
 
 // Device address of g_noalloc_scratch on the current device.  Looked up with
 // the device current on the first call on each device, and again whenever the

@@ -214,7 +214,13 @@ size_t pisa_sparse_attention_bwd_workspace_bytes(int B, int H, int L, int d, int
  * its rounding, amplified by the cancellation in P (dP - Delta), can move dq
  * by several per cent on short sequences.  dq, dk, dv must not overlap any
  * input or one another.  No atomics: bitwise reproducible.
- * `workspace`: pisa_sparse_attention_bwd_workspace_bytes(...) bytes. */
+ * `workspace`: pisa_sparse_attention_bwd_workspace_bytes(...) bytes.
+ * With out_f32, part of the work (the centroid gradients and the key-block
+ * lists, which need nothing from dq) runs beside dq on a second stream that
+ * the library keeps per calling thread and device; it starts after the work
+ * already on `stream` and `stream` waits for it before the call's last
+ * kernel, so to the caller every effect is ordered on `stream` (also under
+ * stream capture), whatever the call returns. */
 pisa_status pisa_sparse_attention_bwd(const void *q, const void *k, const void *v,
                                       const void *dout, const float *lse, const float *out_f32,
                                       const float *kbar, const float *vsum, const int32_t *idx,
