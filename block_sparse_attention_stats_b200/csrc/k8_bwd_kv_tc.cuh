@@ -12,14 +12,17 @@
 // The epilogue adds the centroid chain terms dkbar_j / n_j, dvbar_j / n_j of
 // the key's block and stores bf16.
 //
-// Roles (320 threads):
+// Roles (352 threads):
 //   warp 0      TMA producer: K and V of the two key blocks once, then Q_i,
 //               dout_i, lse_i and Delta_i of every listed query block into a
 //               3-stage ring;
-//   warp 1      TMEM allocation; one elected lane issues every tcgen05.mma:
-//               S^T_u = K Q_i^T and dP^T_u = V dout_i^T into TMEM buffer u & 1,
-//               then dV += P^T_u dout_i and dK += dS^T_u Q_i with P^T and dS^T
-//               read from TMEM;
+//   warp 1      TMEM allocation; issues S^T_u = K Q_i^T into TMEM buffer u & 1
+//               and, once P^T_u is back in it, dV += P^T_u dout_i;
+//   warp 10     issues dP^T_u = V dout_i^T into the same buffer and dK +=
+//               dS^T_u Q_i (one warp's issue rate, about 70 cycles per
+//               tcgen05.mma, would otherwise bound the kernel at 24 products
+//               per tile).  Each half of a buffer is rewritten only by the warp
+//               that also reads its bf16 overwrite, in that warp's issue order;
 //   warps 2-9   two warpgroups of 4 warps; warpgroup g takes the tiles with
 //               u & 1 == g, one thread per key row (TMEM lane): P^T and dS^T
 //               written back as bf16 over S^T and dP^T; the epilogue (half of
@@ -146,7 +149,7 @@ __global__ void pad_lse_kernel(const float *__restrict__ lse, int L, int Lpad, i
 // the tensor-core dk / dv kernel
 // ---------------------------------------------------------------------------
 template <int D> struct KvTcCfg {
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;
   static constexpr int kStages = 3;
   static constexpr int kPairBytes = 128 * D * 2;   // K or V of the two key blocks
   static constexpr int kBoxPairBytes = 128 * 128;  // one 64-column box of 128 rows
@@ -184,7 +187,7 @@ template <int D> struct KvTcCfg {
 // elsewhere), and the epilogue writes dkbar_j / n_j and dvbar_j / n_j (float32)
 // for the exact pass's chain terms.
 template <int D, bool CENT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_do,
                      const __grid_constant__ CUtensorMap tm_k,
@@ -231,14 +234,14 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(bar(C::kBarKV), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bar(C::kBarQFull + s), 1);
-      mbar_init(bar(C::kBarQEmpty + s), 1);
+      mbar_init(bar(C::kBarQEmpty + s), 2);      // dV from warp 1, dK from warp 10
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::kBarSFull + b), 1);
+      mbar_init(bar(C::kBarSFull + b), 2);       // S^T from warp 1, dP^T from warp 10
       mbar_init(bar(C::kBarPFull + b), 128);
     }
-    mbar_init(bar(C::kBarFinal), 1);
-    mbar_init(bar(C::kBarTeardown), 1);
+    mbar_init(bar(C::kBarFinal), 2);
+    mbar_init(bar(C::kBarTeardown), 2);
     fence_mbar_init();
     misc[1] = 0;
   }
@@ -310,42 +313,45 @@ __global__ void __launch_bounds__(320, 1)
       for (int u = issued - C::kStages; u < issued; ++u)
         if (u >= 0) uwait(bar(C::kBarQFull + u % C::kStages), (u / C::kStages) & 1);
     }
-  } else if (warp == 1) {
-    // ======================= MMA issuer =======================================
+  } else if (warp == 1 || warp == 10) {
+    // ======================= MMA issuers ======================================
+    // warp 1: S^T_u into the S half of buffer u & 1, dV += P^T_w dout_w from
+    // it; warp 10: dP^T_u into the dP half, dK += dS^T_w Q_w from it.  A half
+    // is rewritten (by the product of tile w + 2) only after the same warp
+    // has issued the product that reads tile w's overwrite, and one thread's
+    // tcgen05 products run in issue order.
     constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t kIdAcc = idesc_bf16_f32(128, D, 0, 1);
+    const bool s_warp = warp == 1;
+    const uint32_t half_col = s_warp ? 0u : 64u;     // S^T or dP^T half of a buffer
+    const uint32_t acc_col = s_warp ? C::kColDV : C::kColDK;
     bool ok = true;
     if (T > 0) {
       ok = uwait(bar(C::kBarKV), 0);
       tc_fence_after();
       // descriptors are built once per buffer; a K step adds its byte offset /
       // 16 to the start-address field (which cannot carry below 256 KB)
-      const uint64_t kd0 = smem_desc_sw128(sbase + C::kOffK, 16, 1024);
-      const uint64_t vd0 = smem_desc_sw128(sbase + C::kOffV, 16, 1024);
+      const uint64_t ad0 = smem_desc_sw128(sbase + (s_warp ? C::kOffK : C::kOffV), 16, 1024);
+      const int b_off = s_warp ? C::kOffQ : C::kOffDO;    // B of S^T / dP^T
+      const int acc_b_off = s_warp ? C::kOffDO : C::kOffQ;  // B of dV / dK
       auto a_step = [](int k) -> uint64_t {
         return (uint64_t)(((k >> 2) * C::kBoxPairBytes + (k & 3) * 32) >> 4);
       };
       auto b_step = [](int k) -> uint64_t {
         return (uint64_t)(((k >> 2) * C::kBoxRowBytes + (k & 3) * 32) >> 4);
       };
-      // dV and dK products of tile w once P^T and dS^T are in TMEM
+      // the accumulating product of tile w once its bf16 overwrite is in TMEM
       auto finish = [&](int w) -> bool {
         const int b = w & 1, sl = w % C::kStages;
         if (!uwait(bar(C::kBarPFull + b), (w >> 1) & 1)) return false;
         tc_fence_after();
-        const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + sl * C::kTileBytes,
-                                            C::kBoxRowBytes, 1024);
-        const uint64_t dd = smem_desc_sw128(sbase + C::kOffDO + sl * C::kTileBytes,
+        const uint64_t bd = smem_desc_sw128(sbase + acc_b_off + sl * C::kTileBytes,
                                             C::kBoxRowBytes, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + C::kColDV, tmem + C::kColBuf + 128 * b + kk * 8,
-                   dd + (uint64_t)((kk * 2048) >> 4), kIdAcc, (w > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + C::kColDK, tmem + C::kColBuf + 128 * b + 64 + kk * 8,
-                   qd + (uint64_t)((kk * 2048) >> 4), kIdAcc, (w > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + acc_col, tmem + C::kColBuf + 128 * b + half_col + kk * 8,
+                   bd + (uint64_t)((kk * 2048) >> 4), kIdAcc, (w > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::kBarQEmpty + sl));
         }
         __syncwarp();
@@ -356,16 +362,11 @@ __global__ void __launch_bounds__(320, 1)
         const int sl = u % C::kStages, b = u & 1;
         if (!uwait(bar(C::kBarQFull + sl), (u / C::kStages) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + sl * C::kTileBytes, 16, 1024);
-        const uint64_t dd = smem_desc_sw128(sbase + C::kOffDO + sl * C::kTileBytes, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(sbase + b_off + sl * C::kTileBytes, 16, 1024);
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b, kd0 + a_step(k), qd + b_step(k), kIdS,
-                   k > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k)
-            mma_ss(tmem + C::kColBuf + 128 * b + 64, vd0 + a_step(k), dd + b_step(k), kIdS,
+            mma_ss(tmem + C::kColBuf + 128 * b + half_col, ad0 + a_step(k), bd + b_step(k), kIdS,
                    k > 0 ? 1u : 0u);
           tc_commit(bar(C::kBarSFull + b));
         }
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     if (!ok) misc[1] = 1;
-    // every MMA issued must finish before TMEM is released
+    // every MMA this warp issued must finish before TMEM is released
     if (elect_one()) tc_commit(bar(C::kBarTeardown));
     __syncwarp();
     uwait(bar(C::kBarTeardown), 0);
